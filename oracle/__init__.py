@@ -1,0 +1,190 @@
+"""ctypes wrapper around the CPU oracle (test infrastructure only).
+
+Only tests/, the smoke check in __graft_entry__ and bench.py's CPU baseline may
+import this package. It works on host numpy arrays and never touches the CUDA
+library. bf16 tensors are passed as their raw uint16 words.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+FLOOR = 0
+RCEIL = 1
+ERR_ARG = 1
+ERR_OFFSETS = 2
+
+_lib = None
+
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        sig = {
+            "oracle_e4m3_value": (ctypes.c_double, [ctypes.c_uint8]),
+            "oracle_e4m3_from_float": (ctypes.c_uint8, [ctypes.c_float]),
+            "oracle_e4m3_from_float_array": (None, [_f32p, _i64, _u8p]),
+            "oracle_fp8_scale": (ctypes.c_float, [ctypes.c_float]),
+            "oracle_fp8_inv_scale": (ctypes.c_float, [ctypes.c_float]),
+            "oracle_e8m0_floor": (ctypes.c_uint8, [ctypes.c_float]),
+            "oracle_e8m0_rceil": (ctypes.c_uint8, [ctypes.c_float]),
+            "oracle_e8m0": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_int]),
+            "oracle_mx_element": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_uint8]),
+            "oracle_blocked_offset": (_i64, [_i64, _i64, _i64]),
+            "oracle_blocked_grouped_rows_bound": (_i64, [_i64, _i32]),
+            "oracle_fp8_quant_jagged_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _i64, _i32p, _i32, _u8p, _f32p]),
+            "oracle_fp8_quant_jagged_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _i64, _i32p, _i32, _u8p, _f32p]),
+            "oracle_fp8_quant_blockwise": (ctypes.c_int, [_u16p, _i64, _i64, _i32, _i32, _u8p, _f32p]),
+            "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
+            "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
+            "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _words(x):
+    """Raw uint16 words of a bf16 array given as a torch tensor or uint16 numpy array."""
+    if hasattr(x, "view") and hasattr(x, "dtype") and "bfloat16" in str(x.dtype):
+        import torch
+        return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    a = np.asarray(x)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code):
+        super().__init__(f"oracle error {code}")
+        self.code = code
+
+
+def _check(rc):
+    if rc != 0:
+        raise OracleError(rc)
+
+
+# ---- scalars --------------------------------------------------------------
+
+def e4m3_value(code):
+    return lib().oracle_e4m3_value(int(code))
+
+
+def e4m3_from_float(v):
+    return lib().oracle_e4m3_from_float(float(v))
+
+
+def e4m3_from_float_array(v):
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_from_float_array(_p(v, _f32p), v.size, _p(out, _u8p))
+    return out
+
+
+def fp8_scale(amax):
+    return lib().oracle_fp8_scale(float(amax))
+
+
+def fp8_inv_scale(amax):
+    return lib().oracle_fp8_inv_scale(float(amax))
+
+
+def e8m0(amax, mode):
+    return lib().oracle_e8m0(float(amax), int(mode))
+
+
+def mx_element(x, byte):
+    return lib().oracle_mx_element(float(x), int(byte))
+
+
+def blocked_offset(r, c, cols_padded):
+    return lib().oracle_blocked_offset(int(r), int(c), int(cols_padded))
+
+
+def blocked_grouped_rows_bound(rows, groups):
+    return lib().oracle_blocked_grouped_rows_bound(int(rows), int(groups))
+
+
+# ---- ops ------------------------------------------------------------------
+# Strided inputs: `words` is the flat uint16 storage, strides are in elements.
+
+def fp8_quant_jagged_rowwise(words, rows, cols, stride_row, stride_col, offs):
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    out = np.zeros((rows, cols), dtype=np.uint8)
+    inv = np.zeros((len(o), rows), dtype=np.float32)
+    _check(lib().oracle_fp8_quant_jagged_rowwise(_p(w, _u16p), rows, cols, stride_row, stride_col,
+                                                 _p(o, _i32p), len(o), _p(out, _u8p), _p(inv, _f32p)))
+    return out, inv
+
+
+def fp8_quant_jagged_colwise(words, rows, cols, stride_row, stride_col, offs):
+    """Returns (out, inv) with out the column-major buffer viewed as (cols, rows)."""
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    out = np.zeros((cols, rows), dtype=np.uint8)
+    inv = np.zeros((len(o), cols), dtype=np.float32)
+    _check(lib().oracle_fp8_quant_jagged_colwise(_p(w, _u16p), rows, cols, stride_row, stride_col,
+                                                 _p(o, _i32p), len(o), _p(out, _u8p), _p(inv, _f32p)))
+    return out, inv
+
+
+def fp8_quant_blockwise(x, br, bc):
+    w = np.ascontiguousarray(_words(x))
+    rows, cols = w.shape
+    out = np.zeros((rows, cols), dtype=np.uint8)
+    inv = np.zeros((rows // br, cols // bc), dtype=np.float32)
+    _check(lib().oracle_fp8_quant_blockwise(_p(w, _u16p), rows, cols, br, bc, _p(out, _u8p), _p(inv, _f32p)))
+    return out, inv
+
+
+def mx_quant_3d_colwise(x, mode):
+    """x: (E, N, K) bf16. Returns out viewed as (E, K, N) and scales (E, K, N/32)."""
+    w = np.ascontiguousarray(_words(x))
+    E, N, K = w.shape
+    out = np.zeros((E, K, N), dtype=np.uint8)
+    sc = np.zeros((E, K, N // 32), dtype=np.uint8)
+    _check(lib().oracle_mx_quant_3d_colwise(_p(w, _u16p), E, N, K, mode, _p(out, _u8p), _p(sc, _u8p)))
+    return out, sc
+
+
+def mx_quant_rowwise(x, mode):
+    w = np.ascontiguousarray(_words(x))
+    rows, cols = w.shape
+    out = np.zeros((rows, cols), dtype=np.uint8)
+    sc = np.zeros((rows, cols // 32), dtype=np.uint8)
+    _check(lib().oracle_mx_quant_rowwise(_p(w, _u16p), rows, cols, mode, _p(out, _u8p), _p(sc, _u8p)))
+    return out, sc
+
+
+def mx_scales_to_blocked_grouped(scales, offs, capacity_rows=None):
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, cols = s.shape
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    if capacity_rows is None:
+        capacity_rows = blocked_grouped_rows_bound(rows, len(o))
+    cols_p = (cols + 3) // 4 * 4
+    out = np.full((capacity_rows * cols_p,), 0xAB, dtype=np.uint8)
+    starts = np.zeros((len(o),), dtype=np.int32)
+    _check(lib().oracle_mx_scales_to_blocked_grouped(_p(s, _u8p), rows, cols, _p(o, _i32p), len(o),
+                                                     _p(out, _u8p), capacity_rows, _p(starts, _i32p)))
+    return out, starts
