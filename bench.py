@@ -1,0 +1,597 @@
+"""Benchmark of the MoE quantization path on B200.
+
+One step = one pass of the whole path, every op at its full-size workload:
+  blockwise   fp8 1x128 on activations (16384, 4096) and 128x128 on the
+              weight (14336, 4096)                        (Llama-3-8B MLP shapes)
+  jagged      rowwise on grad_out^T and colwise on input, both (65536, 4096),
+              G=16 Dirichlet(0.5) groups along M          (grouped-GEMM backward)
+  MX 3-D      expert weights (E, 8192, 5120), E=64 by default, floor mode
+  MX act      tokens (65536, 7168) rowwise 1x32, then per-group (G=64,
+              Dirichlet(0.3)) 128x4 blocked layout of its E8M0 scales
+Inputs are seeded synthetic tensors resident in HBM; every step moves more
+than 12 GB, far above the 126 MB L2, so no flush is needed between steps.
+
+Metric: achieved HBM GB/s = algorithmic bytes (2 B read + 1 B written per
+element, plus scales) / device time, CUDA events on the launch stream, max
+over ranks. Also printed: per-op us/call and GB/s, a per-shape sweep (L2
+flushed before every rep), the dominant kernel's roofline against the
+measured copy bandwidth, the CPU oracle on a bounded sample, an end-to-end
+figure through the public API from pinned host buffers, and SM clocks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mxq|reference]
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "achieved HBM GB/s and % of B200 peak per quant kernel; µs/call per shape"
+WORKLOAD = "moe_quant_path"
+KERNEL_NAMES = {
+    "blockwise_1x128": "k_fp8_1x128",
+    "blockwise_128x128": "k_fp8_128x128",
+    "jagged_rowwise": "k_jagged_fused",
+    "jagged_colwise": "k_jagged_fused",
+    "mx_3d_colwise": "k_mx_3d_colwise",
+    "mx_rowwise": "k_mx_1x32",
+    "blocked_grouped": "k_blocked_grouped",
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
+    p.add_argument("--experts", type=int, default=64, help="E of the MX 3-D expert-weight op")
+    p.add_argument("--mx3d-mode", default="floor", choices=["floor", "rceil"])
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--no-per-shape", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--reps", type=int, default=20, help="reps per shape in the per-shape sweep")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mxfp8_quantization_moe_device_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("source_hash") != kernel_source_hash():
+            return None
+        return d["kernels"][kernel]["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                 hw=f[5] == "Active", hwt=f[6] == "Active", swt=f[7] == "Active",
+                                 pcap=f[8] == "Active"))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 300] or rows
+        reasons = []
+        for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                          ("pcap", "sw_power_cap")):
+            if any(r[key] for r in loaded):
+                reasons.append(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": reasons, "samples": len(loaded)}
+
+
+# ----------------------------------------------------------------- workload
+
+class Workload:
+    """Device tensors, outputs and the per-op launch closures of one step."""
+
+    def __init__(self, dev, experts, mx3d_mode, with_outputs=True):
+        import torch
+        from mxfp8_quantization_moe_device_b200 import binding as mxq
+        from mxfp8_quantization_moe_device_b200 import synth
+        self.torch, self.mxq = torch, mxq
+        self.dev = dev
+        self.experts = experts
+        self.mx3d_mode = mx3d_mode
+        t = torch
+        self.act = synth.blockwise_act(device=dev)
+        self.wt = synth.blockwise_weight(device=dev)
+        self.grad_out, self.inp, offs16 = synth.jagged_bwd(device=dev)
+        self.offs16 = offs16.to(dev)
+        self.w3 = synth.mx3d_weight(experts, device=dev)
+        self.tok, offs64 = synth.mx_act(device=dev)
+        self.offs64 = offs64.to(dev)
+        M, D = self.inp.shape
+        E, N, K = self.w3.shape
+        T, KT = self.tok.shape
+        u8 = dict(dtype=t.uint8, device=dev)
+        f32 = dict(dtype=t.float32, device=dev)
+        self.o = dict(
+            act_q=t.empty(self.act.shape, **u8), act_s=t.empty((16384, 32), **f32),
+            wt_q=t.empty(self.wt.shape, **u8), wt_s=t.empty((112, 32), **f32),
+            go_q=t.empty((D, M), **u8), go_s=t.empty((16, D), **f32),
+            in_q=t.empty((D, M), **u8), in_s=t.empty((16, D), **f32),
+            w3_q=t.empty((E, K, N), **u8), w3_s=t.empty((E, K, N // 32), **u8),
+            tok_q=t.empty((T, KT), **u8), tok_s=t.empty((T, KT // 32), **u8),
+        )
+        cap = mxq.blocked_grouped_rows_bound(T, 64)
+        self.cap = cap
+        self.o["blk"] = t.empty(cap * ((KT // 32 + 3) // 4 * 4), **u8)
+        self.o["blk_starts"] = t.empty(64, dtype=t.int32, device=dev)
+        ws_r = mxq.jagged_workspace_bytes(D, M, 1, D, 16, False)
+        ws_c = mxq.jagged_workspace_bytes(M, D, D, 1, 16, True)
+        self.ws_r = t.empty(max(ws_r, 1), **u8)
+        self.ws_c = t.empty(max(ws_c, 1), **u8)
+        self.ops = self._ops()
+
+    def _ops(self):
+        mxq, o = self.mxq, self.o
+        E, N, K = self.w3.shape
+        T, KT = self.tok.shape
+        M, D = self.inp.shape
+        G16 = 16
+        ops = [
+            ("blockwise_1x128", lambda: mxq.fp8_quant_blockwise(self.act, 1, 128, out=o["act_q"], inv_scales=o["act_s"]),
+             16384 * 4096 * 3 + 16384 * 32 * 4),
+            ("blockwise_128x128", lambda: mxq.fp8_quant_blockwise(self.wt, 128, 128, out=o["wt_q"], inv_scales=o["wt_s"]),
+             14336 * 4096 * 3 + 112 * 32 * 4),
+            ("jagged_rowwise", lambda: mxq.fp8_quant_jagged_rowwise(self.grad_out.t(), self.offs16, out=o["go_q"],
+                                                                   inv_scales=o["go_s"], workspace=self.ws_r),
+             M * D * 3 + G16 * D * 4),
+            ("jagged_colwise", lambda: mxq.fp8_quant_jagged_colwise(self.inp, self.offs16, out=o["in_q"],
+                                                                   inv_scales=o["in_s"], workspace=self.ws_c),
+             M * D * 3 + G16 * D * 4),
+            ("mx_3d_colwise", lambda: mxq.mx_quant_3d_colwise(self.w3, self.mx3d_mode, out=o["w3_q"], scales=o["w3_s"]),
+             E * N * K * 3 + E * K * N // 32),
+            ("mx_rowwise", lambda: mxq.mx_quant_rowwise(self.tok, "floor", out=o["tok_q"], scales=o["tok_s"]),
+             T * KT * 3 + T * KT // 32),
+            ("blocked_grouped", lambda: mxq.mx_scales_to_blocked_grouped(o["tok_s"], self.offs64, capacity_rows=self.cap,
+                                                                        out=o["blk"], group_row_starts=o["blk_starts"]),
+             T * (KT // 32) + self.cap * ((KT // 32 + 3) // 4 * 4)),
+        ]
+        return ops
+
+    def step_bytes(self):
+        return sum(b for _, _, b in self.ops)
+
+
+def time_steps(wl, steps, warmup, per_op=True):
+    """Run warmup + timed steps on the current stream; returns (total_ms,
+    per-op list of per-step ms)."""
+    torch = wl.torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for _, fn, _ in wl.ops:
+            fn()
+    torch.cuda.synchronize()
+    n = len(wl.ops)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(steps):
+        ev[s][0].record(stream)
+        for i, (_, fn, _) in enumerate(wl.ops):
+            fn()
+            ev[s][i + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    per = [[ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)] for i in range(n)]
+    return total, per
+
+
+def flush_l2(torch, buf):
+    buf.zero_()
+
+
+def per_shape_sweep(wl, reps):
+    """us/call and GB/s per config shape, L2 flushed (256 MB write) before each rep."""
+    torch, mxq = wl.torch, wl.mxq
+    from mxfp8_quantization_moe_device_b200 import synth
+    dev = wl.dev
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, _ = load_peaks()
+    rows = []
+
+    def run(name, shape, fn, nbytes):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush_l2(torch, flush)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        us = statistics.median(ts)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        rows.append({"op": name, "shape": shape, "us": round(us, 3), "GB/s": round(gbs, 1),
+                     "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4)})
+
+    # tiny jagged
+    a, offs = synth.tiny_jagged(device=dev)
+    offs = offs.to(dev)
+    run("jagged_colwise", "(256,512) G=4", lambda: mxq.fp8_quant_jagged_colwise(a, offs), 256 * 512 * 3 + 4 * 512 * 4)
+    run("jagged_rowwise", "(512,256)^T G=4", lambda: mxq.fp8_quant_jagged_rowwise(a.t(), offs), 256 * 512 * 3 + 4 * 512 * 4)
+    by = {n: (f, b) for n, f, b in wl.ops}
+    run("blockwise_1x128", "(16384,4096)", *by["blockwise_1x128"])
+    run("blockwise_128x128", "(14336,4096)", *by["blockwise_128x128"])
+    run("jagged_rowwise", "(4096,65536)^T G=16", *by["jagged_rowwise"])
+    run("jagged_colwise", "(65536,4096) G=16", *by["jagged_colwise"])
+    E = wl.w3.shape[0]
+    for e in [x for x in (1, 2, 4, 8, 16, 64) if x <= E]:
+        w = wl.w3[:e]
+        for mode in ("floor", "rceil"):
+            out = wl.o["w3_q"][:e]
+            sc = wl.o["w3_s"][:e]
+            run("mx_3d_colwise", f"({e},8192,5120) {mode}",
+                lambda w=w, mode=mode, out=out, sc=sc: mxq.mx_quant_3d_colwise(w, mode, out=out, scales=sc),
+                e * 8192 * 5120 * 3 + e * 5120 * 256)
+    for mode in ("floor", "rceil"):
+        run("mx_rowwise", f"(65536,7168) {mode}",
+            lambda mode=mode: mxq.mx_quant_rowwise(wl.tok, mode, out=wl.o["tok_q"], scales=wl.o["tok_s"]),
+            65536 * 7168 * 3 + 65536 * 224)
+    run("blocked_grouped", "(65536,224) G=64", *by["blocked_grouped"])
+    for R in (8192, 5120, 7168, 2048):
+        for C in (512, 1024, 2048, 4096, 32768):
+            s, o = synth.scale_sweep(R, C, device="cpu")
+            s, o = s.to(dev), o.to(dev)
+            cap = mxq.blocked_grouped_rows_bound(R, 8)
+            out = torch.empty(cap * C, dtype=torch.uint8, device=dev)
+            st = torch.empty(8, dtype=torch.int32, device=dev)
+            run("blocked_grouped", f"({R},{C}) G=8",
+                lambda s=s, o=o, cap=cap, out=out, st=st: mxq.mx_scales_to_blocked_grouped(
+                    s, o, capacity_rows=cap, out=out, group_row_starts=st),
+                R * C + cap * C)
+    del flush
+    return rows
+
+
+# ----------------------------------------------------------------- oracle side
+
+def oracle_samples(wl):
+    """Bounded host samples of every op of the step, with the algorithmic
+    bytes each sample stands for: (name, fn, sample_bytes, full_bytes)."""
+    import numpy as np
+    import oracle
+    torch = wl.torch
+
+    def words(t):
+        return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    full = {n: b for n, _, b in wl.ops}
+    act = words(wl.act[:512])
+    wt = words(wl.wt[:256])
+    go = words(wl.grad_out[:, :96])        # (65536, 96): rowwise on its transpose
+    inp = words(wl.inp[:, :96])
+    w3 = words(wl.w3[0, :, :160]).reshape(1, 8192, 160)
+    tok = words(wl.tok[:256])
+    from mxfp8_quantization_moe_device_b200 import synth
+    scales = synth.uniform_u8((65536, 224), 0, 254, seed=9).numpy()  # synthetic, never a GPU output
+    offs16 = wl.offs16.cpu().numpy()
+    offs64 = wl.offs64.cpu().numpy()
+    M = go.shape[0]
+    return [
+        ("blockwise_1x128", lambda: oracle.fp8_quant_blockwise(act, 1, 128), act.size * 3 + act.size // 128 * 4,
+         full["blockwise_1x128"]),
+        ("blockwise_128x128", lambda: oracle.fp8_quant_blockwise(wt, 128, 128), wt.size * 3 + wt.size // 16384 * 4,
+         full["blockwise_128x128"]),
+        ("jagged_rowwise", lambda: oracle.fp8_quant_jagged_rowwise(go.reshape(-1), 96, M, 1, 96, offs16),
+         go.size * 3 + 16 * 96 * 4, full["jagged_rowwise"]),
+        ("jagged_colwise", lambda: oracle.fp8_quant_jagged_colwise(inp.reshape(-1), M, 96, 96, 1, offs16),
+         inp.size * 3 + 16 * 96 * 4, full["jagged_colwise"]),
+        ("mx_3d_colwise", lambda: oracle.mx_quant_3d_colwise(w3, 0 if wl.mx3d_mode == "floor" else 1),
+         w3.size * 3 + w3.size // 32, full["mx_3d_colwise"]),
+        ("mx_rowwise", lambda: oracle.mx_quant_rowwise(tok, 0), tok.size * 3 + tok.size // 32, full["mx_rowwise"]),
+        ("blocked_grouped", lambda: oracle.mx_scales_to_blocked_grouped(scales, offs64, wl.cap),
+         full["blocked_grouped"], full["blocked_grouped"]),
+    ]
+
+
+def run_oracle_samples(samples):
+    """Time each sample once; estimate the oracle's time for the full step
+    from each op's per-byte rate. Returns (GB/s, seconds spent, per-op)."""
+    est = 0.0
+    spent = 0.0
+    per = {}
+    for name, fn, sb, fb in samples:
+        t0 = time.perf_counter()
+        fn()
+        dt = time.perf_counter() - t0
+        spent += dt
+        est += dt * fb / sb
+        per[name] = round(sb / dt / 1e9, 4)
+    total = sum(fb for _, _, _, fb in samples)
+    return total / est / 1e9, spent, per
+
+
+SAMPLE_DESC = ("single-threaded C oracle on a slice of every op: act rows 0-511, weight rows 0-255, "
+               "grad_out/input columns 0-95 (all 65536 rows, G=16), expert 0 columns 0-159, tokens rows 0-255, "
+               "the full (65536,224) scale matrix; each op's time scaled to its full-size bytes")
+
+
+# ----------------------------------------------------------------- e2e
+
+def run_e2e(wl, steps):
+    """The same step through the public API from pinned host buffers: each step
+    copies its inputs host->device, runs every op, and copies every output
+    back to pinned host memory, all inside the timed region."""
+    torch = wl.torch
+    host_in = {}
+    for name in ("act", "wt", "grad_out", "inp", "w3", "tok"):
+        t = getattr(wl, name)
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        host_in[name] = h
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in wl.o.items()}
+    bi = sum(h.numel() * h.element_size() for h in host_in.values()) + 2 * 4 * (16 + 64)
+    bo = sum(h.numel() * h.element_size() for h in host_out.values())
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        for name, h in host_in.items():
+            getattr(wl, name).copy_(h, non_blocking=True)
+        for _, fn, _ in wl.ops:
+            fn()
+        for k, h in host_out.items():
+            h.copy_(wl.o[k], non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    del host_in, host_out
+    return ms, bi, bo
+
+
+# ----------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and "CUDA_VISIBLE_DEVICES" not in os.environ:
+        # one GPU per process: this process sees only its own device as cuda:0
+        os.environ["CUDA_VISIBLE_DEVICES"] = str(local)
+    import torch
+
+    if args.impl == "reference":
+        return main_reference(args, world, rank)
+
+    import torch.distributed as dist
+    if world > 1:
+        dev_index = 0 if os.environ.get("CUDA_VISIBLE_DEVICES", "").count(",") == 0 else local
+        torch.cuda.set_device(dev_index)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    from mxfp8_quantization_moe_device_b200 import binding as mxq
+    mxq.lib()
+
+    wl = Workload(dev, args.experts, args.mx3d_mode)
+    step_bytes = wl.step_bytes()
+    peak, peak_kind = load_peaks()
+
+    clk = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    total_ms, per = time_steps(wl, args.steps, args.warmup)
+    clocks = clk.stop()
+    status = mxq.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed steps")
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+
+    per_op = {}
+    for (name, _, nbytes), ts in zip(wl.ops, per):
+        us = statistics.mean(ts) * 1e3
+        gbs = nbytes / (us * 1e-6) / 1e9
+        per_op[name] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_measured": round(gbs / peak, 4),
+                        "frac_8TBs": round(gbs / 8000.0, 4), "bytes": nbytes, "share": 0.0}
+    tot_us = sum(v["us"] for v in per_op.values())
+    for v in per_op.values():
+        v["share"] = round(v["us"] / tot_us, 4)
+    dom = max(per_op, key=lambda k: per_op[k]["us"])
+    dom_bytes = per_op[dom]["bytes"]
+    achieved = per_op[dom]["GB/s"]
+    roofline = {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "op": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                "algorithmic_bytes_per_launch": dom_bytes, "traffic": load_traffic(KERNEL_NAMES[dom])}
+
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3 (fp32 scale math)",
+           "data": "synthetic (seeded; shapes and distributions of the source pages' workloads)",
+           "config": {"workload": WORKLOAD,
+                      "ops": ["fp8 blockwise 1x128 (16384,4096)", "fp8 blockwise 128x128 (14336,4096)",
+                              "fp8 jagged rowwise grad_out^T (65536,4096) G=16",
+                              "fp8 jagged colwise input (65536,4096) G=16",
+                              f"mx 3d colwise ({args.experts},8192,5120) {args.mx3d_mode}",
+                              "mx rowwise 1x32 (65536,7168) floor",
+                              "mx scales to blocked grouped (65536,224) G=64"],
+                      "step_bytes": step_bytes, "parallelism": f"replicas x{world}",
+                      "l2": "no flush: inputs larger than L2 (each step moves >12 GB)"},
+           "roofline": roofline, "per_op": per_op, "gpu_launches": len(wl.ops) * args.steps,
+           "clocks": clocks}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        samples = oracle_samples(wl)
+        gbs, spent, per_o = run_oracle_samples(samples)
+        out["cpu_baseline"] = {"value": round(gbs, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                               "sample": SAMPLE_DESC, "seconds": round(spent, 2), "per_op_GB/s": per_o}
+    if not args.no_e2e:
+        ms, bi, bo = run_e2e(wl, max(1, args.e2e_steps))
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        out["e2e"] = {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                      "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 3),
+                      "steps": max(1, args.e2e_steps)}
+    if not args.no_per_shape and rank == 0:
+        out["per_shape"] = per_shape_sweep(wl, args.reps)
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main_reference(args, world, rank):
+    """The CPU oracle as the reference arm: rank 0 times it on bounded samples
+    of the same workload, one pass over the samples per step."""
+    if rank != 0:
+        return
+    import torch
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    if dev.type == "cuda":
+        torch.cuda.set_device(dev)
+    wl = RefWorkload(dev, args.experts, args.mx3d_mode)
+    samples = wl.samples
+    for _ in range(args.warmup):
+        samples[0][1]()
+    times = []
+    t0 = time.perf_counter()
+    vals = []
+    for _ in range(args.steps):
+        gbs, spent, _ = run_oracle_samples(samples)
+        vals.append(gbs)
+        times.append(spent)
+    value = statistics.median(vals)
+    total = sum(fb for _, _, _, fb in samples)
+    out = {"metric": METRIC, "impl": "reference", "value": round(value, 5), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / (value * 1e9) * 1e3, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3 (fp32 scale math)",
+           "data": "synthetic (seeded)",
+           "config": {"workload": WORKLOAD, "step_bytes": total, "parallelism": "single-threaded CPU oracle"},
+           "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                            "sample": SAMPLE_DESC},
+           "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "wall_s": round(time.perf_counter() - t0, 1)}
+    print(json.dumps(out))
+
+
+class RefWorkload:
+    """Host-only view of the workload for the reference arm: the same seeded
+    tensors (drawn on the GPU when there is one), sliced to the oracle samples."""
+
+    def __init__(self, dev, experts, mx3d_mode):
+        import torch
+        from mxfp8_quantization_moe_device_b200 import synth
+        self.torch = torch
+        self.mx3d_mode = mx3d_mode
+        self.dev = dev
+        self.act = synth.blockwise_act(device=dev, rows=512)
+        self.wt = synth.blockwise_weight(device=dev, rows=256)
+        go, inp, offs16 = synth.jagged_bwd(device=dev)
+        self.grad_out, self.inp = go[:, :96].contiguous(), inp[:, :96].contiguous()
+        del go, inp
+        self.offs16 = offs16
+        self.w3 = synth.mx3d_weight(1, device=dev)[:, :, :160].contiguous()
+        tok, offs64 = synth.mx_act(device=dev)
+        self.tok = tok[:256].contiguous()
+        self.offs64 = offs64
+        self.cap = 128 * ((65536 + 127 * 64) // 128)
+        E = experts
+        full = {"blockwise_1x128": 16384 * 4096 * 3 + 16384 * 32 * 4,
+                "blockwise_128x128": 14336 * 4096 * 3 + 112 * 32 * 4,
+                "jagged_rowwise": 65536 * 4096 * 3 + 16 * 4096 * 4,
+                "jagged_colwise": 65536 * 4096 * 3 + 16 * 4096 * 4,
+                "mx_3d_colwise": E * 8192 * 5120 * 3 + E * 5120 * 256,
+                "mx_rowwise": 65536 * 7168 * 3 + 65536 * 224,
+                "blocked_grouped": 65536 * 224 + self.cap * 224}
+        self.ops = [(k, None, v) for k, v in full.items()]
+        self.samples = oracle_samples(self)
+
+
+if __name__ == "__main__":
+    main()

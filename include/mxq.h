@@ -1,0 +1,223 @@
+/*
+ * mxq.h - C ABI of libmxq, the sm_100a (B200) library for the dynamic
+ * low-precision quantization path that feeds scaled grouped GEMMs in
+ * mixture-of-experts training.
+ *
+ * Sources, pytorch/ao pull-request pages:
+ *   #2064 "[scaled grouped mm] add triton kernels for float8 rowwise
+ *          quantization with per-group/jagged scales" (Motivation, Summary)
+ *   #2827 "[fp8 blockwise] load 2d chunks for groupwise quant to enable
+ *          coalesced gmem accesses" (description, Kernel performance)
+ *   #3002 "[mxfp8 moe training] add CUDA kernel to quantize 3d tensor
+ *          colwise" (Summary, comments)
+ *   #3504 "[mxfp8 moe training] add CUDA kernel for per-group conversion of
+ *          scale factors to blocked layout" (title, Benchmarks)
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers, owned by the caller; the library never
+ *     frees or retains them. bf16 inputs are raw 16-bit words; float8 e4m3
+ *     and E8M0 outputs are raw bytes; scales written as fp32 are the
+ *     INVERSE scales (multiply the e4m3 value by them to dequantize).
+ *   - Work is enqueued on `stream`; nothing synchronizes the host, and the
+ *     group offsets are never read on the host.
+ *   - Calls return MXQ_OK after a successful enqueue. A call with no
+ *     elements to process returns MXQ_OK without launching, and its data
+ *     pointers may then be NULL. Problems visible on
+ *     the host (null pointer, bad shape, misalignment, small workspace) are
+ *     returned at once and nothing is launched. Problems only visible on the
+ *     device (malformed offsets, an expired wait) are recorded in a device
+ *     status word that mxq_device_status() reads and clears; in that case the
+ *     kernel writes none of its outputs (offsets) or stops early (timeout).
+ *   - Entry points are reentrant and may be called from several host
+ *     threads; calls on different streams run concurrently.
+ *   - Offsets: int32, `num_groups` cumulative group ENDS along the grouped
+ *     dimension: group g covers [offs[g-1], offs[g]) with offs[-1] = 0.
+ *     They must be non-decreasing and lie in [0, extent]. Empty groups are
+ *     allowed; elements past offs[num_groups-1] are not written.
+ *
+ * Numerics (bit-exact, no tolerance; every rule is computed in fp32):
+ *   e4m3 unit scale  s = 448 / max(amax, 1e-12f), stored inverse = 1 / s,
+ *                    element = e4m3(clamp(x * s)), round to nearest even.
+ *   MX (E8M0)        floor: 2^(floor(log2 amax) - 8);
+ *                    rceil: 2^ceil(log2(amax / 448)); both clamped to
+ *                    [2^-127, 2^127]; element = e4m3(x / scale).
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mxq_status {
+    MXQ_OK = 0,
+    MXQ_ERR_NULL = 1,        /* a required pointer is NULL                      */
+    MXQ_ERR_SHAPE = 2,       /* negative / non-divisible sizes                  */
+    MXQ_ERR_ALIGN = 3,       /* pointer or stride misaligned for the op         */
+    MXQ_ERR_UNSUPPORTED = 4, /* parameter combination not implemented           */
+    MXQ_ERR_LAUNCH = 5,      /* the CUDA launch failed                          */
+    MXQ_ERR_BAD_OFFSETS = 6, /* device: offsets decreasing, negative or > extent */
+    MXQ_ERR_TIMEOUT = 7,     /* device: a bounded wait expired                  */
+    MXQ_ERR_WORKSPACE = 8,   /* workspace missing or smaller than required      */
+    MXQ_ERR_CUDA = 9         /* another CUDA runtime error                      */
+} mxq_status;
+
+typedef enum mxq_scale_mode {
+    MXQ_E8M0_FLOOR = 0,
+    MXQ_E8M0_RCEIL = 1
+} mxq_scale_mode;
+
+/* ------------------------------------------------------------------------ *
+ * (a1) fp8_quant_jagged_rowwise - #2064 Summary, first kernel: float8 e4m3
+ * quantization with one scale per (row, group), the groups being column
+ * ranges given by `offs`, output row-major. Used on the left operand of the
+ * grad_weight grouped GEMM (grad_out^T).
+ *   in          logical (rows, cols) bf16; element (r, c) at
+ *               in[r * stride_row + c * stride_col] (strides in elements).
+ *               The transposed view of a row-major (M, N) tensor has
+ *               stride_row = 1, stride_col = N and takes the fast path.
+ *   offs        num_groups int32 ends along cols (device).
+ *   out         rows x cols e4m3 bytes, row-major: out[r * cols + c].
+ *   inv_scales  fp32 (num_groups, rows): inv_scales[g * rows + r].
+ *   workspace   device scratch of at least
+ *               fp8_quant_jagged_workspace_bytes(rows, cols, stride_row,
+ *               stride_col, num_groups) bytes (may be NULL when that is 0);
+ *               it is cleared and used by the call, so concurrent calls need
+ *               distinct workspaces.
+ * ------------------------------------------------------------------------ */
+int fp8_quant_jagged_rowwise(const void *in, int64_t rows, int64_t cols,
+                             int64_t stride_row, int64_t stride_col,
+                             const int32_t *offs, int32_t num_groups,
+                             void *out, float *inv_scales,
+                             void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * (a2) fp8_quant_jagged_colwise - #2064 Summary, second kernel: one scale per
+ * (column, group), the groups being row ranges, output column-major. Used on
+ * the right operand of the grad_weight grouped GEMM (input).
+ *   in          logical (rows, cols) bf16 with element strides; row-major
+ *               (stride_row = cols, stride_col = 1) takes the fast path.
+ *   offs        num_groups int32 ends along rows (device).
+ *   out         column-major e4m3: out[c * rows + r].
+ *   inv_scales  fp32 (num_groups, cols): inv_scales[g * cols + c].
+ *   workspace   as for the rowwise op.
+ * Rowwise on the transposed view of A and colwise on A give byte-identical
+ * buffers and scales.
+ * ------------------------------------------------------------------------ */
+int fp8_quant_jagged_colwise(const void *in, int64_t rows, int64_t cols,
+                             int64_t stride_row, int64_t stride_col,
+                             const int32_t *offs, int32_t num_groups,
+                             void *out, float *inv_scales,
+                             void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/* Workspace size for the jagged ops with these arguments (rowwise: pass the
+ * rowwise shape and strides; colwise: the colwise ones, with is_colwise = 1).
+ * Returns 0 when the call needs none. */
+size_t fp8_quant_jagged_workspace_bytes(int64_t rows, int64_t cols,
+                                        int64_t stride_row, int64_t stride_col,
+                                        int32_t num_groups, int32_t is_colwise);
+
+/* ------------------------------------------------------------------------ *
+ * (a3) fp8_quant_blockwise - #2827: one e4m3 scale per block of a row-major
+ * (rows, cols) bf16 matrix; block 1 x 128 (activations) or 128 x 128
+ * (weights).
+ *   block_rows  1 or 128; block_cols 128. rows % block_rows == 0,
+ *               cols % 128 == 0, else MXQ_ERR_SHAPE / MXQ_ERR_UNSUPPORTED.
+ *   in, out     16-byte aligned; out row-major e4m3 (rows, cols).
+ *   inv_scales  fp32 row-major (rows / block_rows, cols / 128).
+ * ------------------------------------------------------------------------ */
+int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols,
+                        int32_t block_rows, int32_t block_cols,
+                        void *out, float *inv_scales, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * (a4) mx_quant_3d_colwise - #3002 Summary: MXFP8 quantization of expert
+ * weights (E, N, K) along N in 32 x 1 blocks, written straight into each
+ * expert's column-major layout.
+ *   in          contiguous (E, N, K) bf16; K % 8 == 0; 16-byte aligned.
+ *   mode        MXQ_E8M0_FLOOR or MXQ_E8M0_RCEIL.
+ *   out         e4m3 with strides (N*K, 1, N): out[e*N*K + k*N + n];
+ *               16-byte aligned.
+ *   scales      E8M0 bytes (E, K, N/32) row-major.
+ *   N % 32 == 0, else MXQ_ERR_SHAPE.
+ * ------------------------------------------------------------------------ */
+int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K,
+                        int32_t mode, void *out, uint8_t *scales,
+                        cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * (a5) mx_quant_rowwise - MXFP8 1 x 32 quantization along the last dimension
+ * of a row-major (rows, cols) bf16 matrix (the last-dim scaling #3002's
+ * Summary describes for to_mx), used on MoE activations.
+ *   cols % 32 == 0; in and out 16-byte aligned.
+ *   out         e4m3 row-major (rows, cols).
+ *   scales      E8M0 bytes (rows, cols / 32) row-major.
+ * ------------------------------------------------------------------------ */
+int mx_quant_rowwise(const void *in, int64_t rows, int64_t cols, int32_t mode,
+                     void *out, uint8_t *scales, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * (a6) mx_scales_to_blocked_grouped - #3504 title: per-group conversion of an
+ * E8M0 scale matrix (rows, cols) to the 128 x 4 blocked layout, the groups
+ * being row ranges from `offs`, each padded to a multiple of 128 rows on its
+ * own.
+ *   Layout: group g's rows start at padded row P_g = sum_{h<g}
+ *   128*ceil(size_h/128); columns are padded to cols4 = 4*ceil(cols/4);
+ *   byte (R, c) of the padded matrix lives at
+ *   ((R/128)*(cols4/4) + c/4)*512 + (R%32)*16 + ((R%128)/32)*4 + c%4.
+ *   Every byte of out is written: pad bytes and all rows past the last group
+ *   are 0.
+ *   out_rows_capacity  a multiple of 128 and at least
+ *               mx_blocked_grouped_rows_bound(rows, num_groups); out holds
+ *               out_rows_capacity * cols4 bytes and is 16-byte aligned.
+ *   out_group_row_starts  optional (NULL allowed): P_g for each group, int32.
+ * ------------------------------------------------------------------------ */
+int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t cols,
+                                 const int32_t *offs, int32_t num_groups,
+                                 uint8_t *out, int64_t out_rows_capacity,
+                                 int32_t *out_group_row_starts,
+                                 cudaStream_t stream);
+
+/* Smallest capacity valid for any offsets: 128 * floor((rows + 127*G) / 128). */
+int64_t mx_blocked_grouped_rows_bound(int64_t rows, int32_t num_groups);
+
+/* ------------------------------------------------------------------------ *
+ * Status and housekeeping
+ * ------------------------------------------------------------------------ */
+
+/* Synchronizes `stream`, stores the first device-side error recorded since
+ * the last call (MXQ_OK if none) in *host_status and clears it. */
+int mxq_device_status(cudaStream_t stream, int32_t *host_status);
+
+/* Static text for a status code. */
+const char *mxq_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mxq_version(void);
+
+/* Test hooks (host-side settings read at launch time):
+ *   MXQ_TESTING_WAIT_LIMIT_NS  bound of every device-side wait, nanoseconds
+ *                              (default 1e9; 0 restores the default).
+ *   MXQ_TESTING_SKIP_ARRIVAL   when 1, one CTA of the single-pass jagged
+ *                              kernels skips its arrival on the amax barrier,
+ *                              so the others' bounded waits expire and report
+ *                              MXQ_ERR_TIMEOUT; 0 turns it off.
+ *   MXQ_TESTING_FORCE_PATH     jagged ops: 0 automatic, 1 single-pass
+ *                              barrier kernel, 2 generic kernel. */
+#define MXQ_TESTING_WAIT_LIMIT_NS 1
+#define MXQ_TESTING_SKIP_ARRIVAL 2
+#define MXQ_TESTING_FORCE_PATH 3
+int mxq_testing_set(int32_t what, int64_t value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

@@ -1,0 +1,241 @@
+"""Thin ctypes binding over libmxq.so (C ABI in include/mxq.h).
+
+Argument marshalling only: every step of the quantization path runs in the
+library's CUDA kernels. PyTorch provides the device memory (outputs and the
+jagged workspace are allocated here with torch.empty) and the stream (the
+current torch stream of the input's device). There is no CPU fallback: when
+the library is missing, or a tensor is not on a CUDA device, the call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxq.so")
+
+OK = 0
+ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_LAUNCH = 1, 2, 3, 4, 5
+ERR_BAD_OFFSETS, ERR_TIMEOUT, ERR_WORKSPACE, ERR_CUDA = 6, 7, 8, 9
+FLOOR, RCEIL = 0, 1
+TESTING_WAIT_LIMIT_NS, TESTING_SKIP_ARRIVAL, TESTING_FORCE_PATH = 1, 2, 3
+
+_lib = None
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/mxq.h
+SIGNATURES = {
+    "fp8_quant_jagged_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "fp8_quant_jagged_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "fp8_quant_jagged_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32]),
+    "fp8_quant_blockwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
+    "mx_blocked_grouped_rows_bound": (_i64, [_i64, _i32]),
+    "mxq_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(_i32)]),
+    "mxq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mxq_version": (ctypes.c_int, []),
+    "mxq_testing_set": (ctypes.c_int, [_i32, _i64]),
+}
+
+
+class MXQError(RuntimeError):
+    def __init__(self, fn, code):
+        msg = lib().mxq_status_string(code).decode() if _lib is not None else str(code)
+        super().__init__(f"{fn}: {msg} (status {code})")
+        self.code = code
+
+
+def lib():
+    """Load libmxq.so once. Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libmxq.so not found at {LIB_PATH}; build it with "
+                "`python -m mxfp8_quantization_moe_device_b200.build` (or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn, rc):
+    if rc != OK:
+        raise MXQError(fn, rc)
+
+
+def _cuda(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _mode(mode):
+    if mode in (FLOOR, "floor"):
+        return FLOOR
+    if mode in (RCEIL, "rceil"):
+        return RCEIL
+    raise ValueError(f"unknown scale mode {mode!r}")
+
+
+def _offsets(offs, dev):
+    _cuda(offs, "offs")
+    if offs.dtype != torch.int32 or offs.dim() != 1 or not offs.is_contiguous() or offs.device != dev:
+        raise TypeError("offs must be a contiguous 1-D int32 tensor on the input's device")
+    return offs
+
+
+# ---------------------------------------------------------------- jagged
+
+def jagged_workspace_bytes(rows, cols, stride_row, stride_col, num_groups, colwise):
+    return lib().fp8_quant_jagged_workspace_bytes(rows, cols, stride_row, stride_col, num_groups, 1 if colwise else 0)
+
+
+def _jagged(name, x, offs, colwise, out, inv_scales, workspace):
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    dev = x.device
+    _offsets(offs, dev)
+    rows, cols = x.shape
+    sr, sc = x.stride()
+    G = offs.numel()
+    if out is None:
+        out = torch.empty((cols, rows) if colwise else (rows, cols), dtype=torch.uint8, device=dev)
+    if inv_scales is None:
+        inv_scales = torch.empty((G, cols if colwise else rows), dtype=torch.float32, device=dev)
+    need = jagged_workspace_bytes(rows, cols, sr, sc, G, colwise)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    # the library reads x through its data pointer and element strides
+    rc = getattr(lib(), name)(_ptr(x), rows, cols, sr, sc, _ptr(offs), G, _ptr(out), _ptr(inv_scales),
+                              _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream(dev))
+    _check(name, rc)
+    q = out.view(torch.float8_e4m3fn)
+    return (q.t() if colwise else q), inv_scales
+
+
+def fp8_quant_jagged_rowwise(x, offs, *, out=None, inv_scales=None, workspace=None):
+    """e4m3 quantization of x (rows, cols), one scale per (row, group), groups
+    along cols. Returns (q row-major (rows, cols) float8_e4m3fn, inv (G, rows))."""
+    return _jagged("fp8_quant_jagged_rowwise", x, offs, False, out, inv_scales, workspace)
+
+
+def fp8_quant_jagged_colwise(x, offs, *, out=None, inv_scales=None, workspace=None):
+    """e4m3 quantization of x (rows, cols), one scale per (column, group),
+    groups along rows. Returns (q column-major (rows, cols) view, inv (G, cols))."""
+    return _jagged("fp8_quant_jagged_colwise", x, offs, True, out, inv_scales, workspace)
+
+
+# ---------------------------------------------------------------- blockwise
+
+def fp8_quant_blockwise(x, block_rows=1, block_cols=128, *, out=None, inv_scales=None):
+    """e4m3 quantization of row-major x with one scale per block_rows x 128 block.
+    Returns (q (rows, cols) float8_e4m3fn, inv (rows/block_rows, cols/128))."""
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if inv_scales is None:
+        inv_scales = torch.empty((rows // block_rows, cols // block_cols), dtype=torch.float32, device=x.device)
+    rc = lib().fp8_quant_blockwise(_ptr(x), rows, cols, block_rows, block_cols, _ptr(out), _ptr(inv_scales),
+                                   _stream(x.device))
+    _check("fp8_quant_blockwise", rc)
+    return out.view(torch.float8_e4m3fn), inv_scales
+
+
+# ---------------------------------------------------------------- MX
+
+def mx_quant_3d_colwise(w, mode="floor", *, out=None, scales=None):
+    """MXFP8 quantization of expert weights w (E, N, K) along N (32x1 blocks).
+    Returns (q (E, N, K) with strides (N*K, 1, N), scales (E, K, N/32) uint8 E8M0)."""
+    _cuda(w, "w")
+    if w.dtype != torch.bfloat16 or w.dim() != 3 or not w.is_contiguous():
+        raise TypeError("w must be a contiguous 3-D bfloat16 tensor")
+    E, N, K = w.shape
+    if out is None:
+        out = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((E, K, N // 32), dtype=torch.uint8, device=w.device)
+    rc = lib().mx_quant_3d_colwise(_ptr(w), E, N, K, _mode(mode), _ptr(out), _ptr(scales), _stream(w.device))
+    _check("mx_quant_3d_colwise", rc)
+    return out.view(torch.float8_e4m3fn).transpose(1, 2), scales
+
+
+def mx_quant_rowwise(x, mode="floor", *, out=None, scales=None):
+    """MXFP8 1x32 quantization of row-major x (rows, cols) along cols.
+    Returns (q (rows, cols) float8_e4m3fn, scales (rows, cols/32) uint8 E8M0)."""
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
+    rc = lib().mx_quant_rowwise(_ptr(x), rows, cols, _mode(mode), _ptr(out), _ptr(scales), _stream(x.device))
+    _check("mx_quant_rowwise", rc)
+    return out.view(torch.float8_e4m3fn), scales
+
+
+def blocked_grouped_rows_bound(rows, num_groups):
+    return lib().mx_blocked_grouped_rows_bound(rows, num_groups)
+
+
+def mx_scales_to_blocked_grouped(scales, offs, *, capacity_rows=None, out=None, group_row_starts=None,
+                                 with_starts=True):
+    """Per-group 128x4 blocked layout of a (rows, cols) uint8 scale matrix with
+    groups along rows. Returns (out flat uint8 of capacity_rows * pad4(cols)
+    bytes, padded group starts int32 (G) or None)."""
+    _cuda(scales, "scales")
+    if scales.dim() != 2 or not scales.is_contiguous() or scales.element_size() != 1:
+        raise TypeError("scales must be a contiguous 2-D 1-byte tensor")
+    dev = scales.device
+    _offsets(offs, dev)
+    rows, cols = scales.shape
+    G = offs.numel()
+    if capacity_rows is None:
+        capacity_rows = blocked_grouped_rows_bound(rows, G)
+    cols4 = (cols + 3) // 4 * 4
+    if out is None:
+        out = torch.empty(capacity_rows * cols4, dtype=torch.uint8, device=dev)
+    if group_row_starts is None and with_starts:
+        group_row_starts = torch.empty(G, dtype=torch.int32, device=dev)
+    rc = lib().mx_scales_to_blocked_grouped(_ptr(scales), rows, cols, _ptr(offs), G, _ptr(out), capacity_rows,
+                                            _ptr(group_row_starts), _stream(dev))
+    _check("mx_scales_to_blocked_grouped", rc)
+    return out, group_row_starts
+
+
+# ---------------------------------------------------------------- status
+
+def device_status(device=None):
+    """Synchronize the current stream and return (and clear) the first
+    device-side error recorded by the kernels (0 = none)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    v = _i32(0)
+    _check("mxq_device_status", lib().mxq_device_status(_stream(dev), ctypes.byref(v)))
+    return v.value
+
+
+def testing_set(what, value):
+    _check("mxq_testing_set", lib().mxq_testing_set(what, value))

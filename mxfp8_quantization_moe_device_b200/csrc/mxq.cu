@@ -1,0 +1,475 @@
+// mxq.cu - host side of libmxq: argument checks, TMA descriptor encoding,
+// launch configuration and the C ABI declared in include/mxq.h. All kernels
+// are compiled into this one translation unit for sm_100a.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "rowblock.cuh"
+#include "mx3d.cuh"
+#include "jagged.cuh"
+#include "blocked.cuh"
+
+using namespace mxq;
+
+namespace {
+
+std::atomic<int64_t> g_wait_ns{1000000000LL};
+std::atomic<int> g_skip_arrival{0};
+std::atomic<int> g_force_path{0};
+
+uint64_t wait_ns() { return (uint64_t)g_wait_ns.load(); }
+
+// ------------------------------------------------------------ driver entry
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// rank-N tiled map; dims/box innermost first, strides in bytes for dims 1..N-1
+int make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *ptr, const uint64_t *dims,
+             const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return MXQ_ERR_CUDA;
+    cuuint64_t d[5], s[5];
+    cuuint32_t b[5], e[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        e[i] = 1;
+        if (i + 1 < rank)
+            s[i] = strides[i];
+    }
+    const CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(ptr), d, s, b, e,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MXQ_OK : MXQ_ERR_ALIGN;
+}
+
+// ------------------------------------------------------------ device info
+struct DevInfo {
+    bool ready = false;
+    int sms = 0;
+    int smem_optin = 0;
+    int coop = 0;
+};
+
+DevInfo g_dev[128];
+std::mutex g_dev_mu;
+
+int device_info(const DevInfo **out)
+{
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 128)
+        return MXQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo &di = g_dev[d];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.coop, cudaDevAttrCooperativeLaunch, d) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        if (cudaFuncSetAttribute(mx3d::k_mx_3d_colwise<MXQ_E8M0_FLOOR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mx3d::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(mx3d::k_mx_3d_colwise<MXQ_E8M0_RCEIL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mx3d::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(k_jagged_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 di.smem_optin - (int)sizeof(jag::Misc) - 64) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        di.ready = true;
+    }
+    *out = &di;
+    return MXQ_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+template <typename... K, typename... A>
+int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool coop, A &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (coop) {
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MXQ_ERR_LAUNCH;
+    }
+    return MXQ_OK;
+}
+
+// ------------------------------------------------------------ jagged plan
+struct JaggedPlan {
+    bool fused = false;
+    int chunk = 0, stages = 0, ncta = 0, rounds = 0, nseg_cap = 0;
+    size_t smem = 0;
+    size_t ws_amax = 0, ws_total = 0;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// host-checkable part of the single-pass conditions (no device queries)
+bool fused_layout_ok(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, int G, const void *out)
+{
+    return s_line == 1 && s_pos % 8 == 0 && s_pos >= L && L > 0 && P > 0 && P % 16 == 0 && G >= 1 &&
+           G <= jag::MAX_SEG && (in == nullptr || aligned(in, 16)) && (out == nullptr || aligned(out, 16)) &&
+           P < (int64_t(1) << 31) && L < (int64_t(1) << 31);
+}
+
+size_t fused_workspace(int64_t L, int G)
+{
+    const int64_t rounds = (L + jag::W - 1) / jag::W;
+    return round_up((size_t)G * (size_t)L * 4, 256) + round_up((size_t)rounds * 4, 256);
+}
+
+int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, int G, const void *out,
+                JaggedPlan *pl)
+{
+    *pl = JaggedPlan();
+    const int force = g_force_path.load();
+    if (force == 2 || !fused_layout_ok(in, L, P, s_line, s_pos, G, out))
+        return MXQ_OK;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    if (!di->coop)
+        return MXQ_OK;
+    const int64_t per = (P + di->sms - 1) / di->sms;
+    const int chunk = (int)((per + jag::OBOX - 1) / jag::OBOX * jag::OBOX);
+    const int ncta = (int)((P + chunk - 1) / chunk);
+    const int nseg_cap = G;
+    const int budget = di->smem_optin - (int)sizeof(jag::Misc) - 64 - 1024;
+    int stages = 0;
+    for (int s = 4; s >= 2; --s)
+        if (jag::layout(chunk, s, nseg_cap).total <= budget) {
+            stages = s;
+            break;
+        }
+    if (stages == 0)
+        return MXQ_OK;
+    const size_t smem = (size_t)jag::layout(chunk, stages, nseg_cap).total + 1024;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_jagged_fused, jag::THREADS, smem) != cudaSuccess ||
+        per_sm < 1 || ncta > per_sm * di->sms)
+        return MXQ_OK;
+    pl->fused = true;
+    pl->chunk = chunk;
+    pl->stages = stages;
+    pl->ncta = ncta;
+    pl->rounds = (int)((L + jag::W - 1) / jag::W);
+    pl->nseg_cap = nseg_cap;
+    pl->smem = smem;
+    pl->ws_amax = round_up((size_t)G * (size_t)L * 4, 256);
+    pl->ws_total = fused_workspace(L, G);
+    return MXQ_OK;
+}
+
+int jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, const int32_t *offs, int G,
+           void *out, float *inv, void *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    if (L < 0 || P < 0 || G < 1)
+        return MXQ_ERR_SHAPE;
+    if (L == 0)
+        return MXQ_OK;
+    if (!offs || !inv || (P > 0 && (!in || !out)))
+        return MXQ_ERR_NULL;
+    JaggedPlan pl;
+    int rc = plan_jagged(in, L, P, s_line, s_pos, G, out, &pl);
+    if (rc != MXQ_OK)
+        return rc;
+    if (g_force_path.load() == 1 && !pl.fused)
+        return MXQ_ERR_UNSUPPORTED;
+    if (pl.fused) {
+        if (!ws || ws_bytes < pl.ws_total)
+            return MXQ_ERR_WORKSPACE;
+        if (!aligned(ws, 256))
+            return MXQ_ERR_ALIGN;
+        CUtensorMap tin, tout;
+        const uint64_t din[2] = {(uint64_t)L, (uint64_t)P};
+        const uint64_t sin[1] = {(uint64_t)s_pos * 2};
+        const uint32_t bin[2] = {jag::W, jag::BOXP};
+        rc = make_map(&tin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, din, sin, bin, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc != MXQ_OK)
+            return rc;
+        const uint64_t dout[2] = {(uint64_t)P, (uint64_t)L};
+        const uint64_t sout[1] = {(uint64_t)P};
+        const uint32_t bout[2] = {jag::OBOX, jag::W};
+        rc = make_map(&tout, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_64B);
+        if (rc != MXQ_OK)
+            return rc;
+        if (cudaMemsetAsync(ws, 0, pl.ws_total, stream) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        jag::Params p;
+        p.L = L;
+        p.P = P;
+        p.G = G;
+        p.chunk = pl.chunk;
+        p.stages = pl.stages;
+        p.rounds = pl.rounds;
+        p.nseg_cap = pl.nseg_cap;
+        p.offs = offs;
+        p.out = static_cast<uint8_t *>(out);
+        p.inv = inv;
+        p.amax = static_cast<unsigned *>(ws);
+        p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + pl.ws_amax);
+        p.wait_ns = wait_ns();
+        p.skip_arrival = g_skip_arrival.load();
+        return launch(k_jagged_fused, dim3(pl.ncta), dim3(jag::THREADS), pl.smem, stream, true, tin, tout, p);
+    }
+    const DevInfo *di = nullptr;
+    rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t warps = L * G;
+    const int64_t grid = std::min<int64_t>((warps + 7) / 8, (int64_t)di->sms * 16);
+    return launch(k_jagged_generic, dim3((unsigned)std::max<int64_t>(grid, 1)), dim3(256), 0, stream, false,
+                  static_cast<const uint16_t *>(in), L, P, s_line, s_pos, offs, G, static_cast<uint8_t *>(out), inv);
+}
+
+} // namespace
+
+// ======================================================================= ABI
+extern "C" {
+
+int fp8_quant_jagged_rowwise(const void *in, int64_t rows, int64_t cols, int64_t stride_row, int64_t stride_col,
+                             const int32_t *offs, int32_t num_groups, void *out, float *inv_scales,
+                             void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    // line = row, position = column
+    return jagged(in, rows, cols, stride_row, stride_col, offs, num_groups, out, inv_scales, workspace,
+                  workspace_bytes, stream);
+}
+
+int fp8_quant_jagged_colwise(const void *in, int64_t rows, int64_t cols, int64_t stride_row, int64_t stride_col,
+                             const int32_t *offs, int32_t num_groups, void *out, float *inv_scales,
+                             void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    // line = column, position = row
+    return jagged(in, cols, rows, stride_col, stride_row, offs, num_groups, out, inv_scales, workspace,
+                  workspace_bytes, stream);
+}
+
+size_t fp8_quant_jagged_workspace_bytes(int64_t rows, int64_t cols, int64_t stride_row, int64_t stride_col,
+                                        int32_t num_groups, int32_t is_colwise)
+{
+    const int64_t L = is_colwise ? cols : rows, P = is_colwise ? rows : cols;
+    const int64_t sl = is_colwise ? stride_col : stride_row, sp = is_colwise ? stride_row : stride_col;
+    if (!fused_layout_ok(nullptr, L, P, sl, sp, num_groups, nullptr))
+        return 0;
+    return fused_workspace(L, num_groups);
+}
+
+int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols, int32_t block_rows, int32_t block_cols,
+                        void *out, float *inv_scales, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0)
+        return MXQ_ERR_SHAPE;
+    if (block_cols != 128 || (block_rows != 1 && block_rows != 128))
+        return MXQ_ERR_UNSUPPORTED;
+    if (cols % 128 || rows % block_rows)
+        return MXQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0)
+        return MXQ_OK;
+    if (!in || !out || !inv_scales)
+        return MXQ_ERR_NULL;
+    if (!aligned(in, 16) || !aligned(out, 16) || !aligned(inv_scales, 4))
+        return MXQ_ERR_ALIGN;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    if (block_rows == 1) {
+        const int64_t nblk = rows * (cols / 128);
+        const int64_t per_cta = (RB_THREADS / 32) * 2 * RB_UNROLL;
+        const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, (int64_t)di->sms * 8);
+        return launch(k_fp8_1x128, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
+                      static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), inv_scales);
+    }
+    if (rows / 128 > 65535)
+        return MXQ_ERR_UNSUPPORTED;
+    return launch(k_fp8_128x128, dim3((unsigned)(cols / 128), (unsigned)(rows / 128)), dim3(256), 0, stream, false,
+                  static_cast<const uint4 *>(in), cols, static_cast<uint2 *>(out), inv_scales);
+}
+
+int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t mode, void *out, uint8_t *scales,
+                        cudaStream_t stream)
+{
+    if (E < 0 || N < 0 || K < 0 || N % 32)
+        return MXQ_ERR_SHAPE;
+    if (mode != MXQ_E8M0_FLOOR && mode != MXQ_E8M0_RCEIL)
+        return MXQ_ERR_UNSUPPORTED;
+    if (E == 0 || N == 0 || K == 0)
+        return MXQ_OK;
+    if (!in || !out || !scales)
+        return MXQ_ERR_NULL;
+    if (K % 8 || !aligned(in, 16) || !aligned(out, 16))
+        return MXQ_ERR_ALIGN;
+    if (E >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    CUtensorMap tin, tout;
+    const uint64_t din[3] = {(uint64_t)K, (uint64_t)N, (uint64_t)E};
+    const uint64_t sin[2] = {(uint64_t)K * 2, (uint64_t)N * K * 2};
+    const uint32_t bin[3] = {mx3d::TK, mx3d::TN, 1};
+    rc = make_map(&tin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, in, din, sin, bin, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t dout[3] = {(uint64_t)N, (uint64_t)K, (uint64_t)E};
+    const uint64_t sout[2] = {(uint64_t)N, (uint64_t)N * K};
+    const uint32_t bout[3] = {mx3d::TN, mx3d::TK, 1};
+    rc = make_map(&tout, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, out, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const int tiles_n = (int)((N + mx3d::TN - 1) / mx3d::TN), tiles_k = (int)((K + mx3d::TK - 1) / mx3d::TK);
+    const int64_t total = E * tiles_n * tiles_k;
+    const int64_t grid = std::min<int64_t>(total, (int64_t)di->sms * mx3d::CTAS_PER_SM);
+    if (mode == MXQ_E8M0_FLOOR)
+        return launch(mx3d::k_mx_3d_colwise<MXQ_E8M0_FLOOR>, dim3((unsigned)grid), dim3(mx3d::THREADS),
+                      mx3d::SMEM_BYTES, stream, false, tin, tout, scales, (int)E, (int)N, (int)K, tiles_n, tiles_k,
+                      wait_ns());
+    return launch(mx3d::k_mx_3d_colwise<MXQ_E8M0_RCEIL>, dim3((unsigned)grid), dim3(mx3d::THREADS), mx3d::SMEM_BYTES,
+                  stream, false, tin, tout, scales, (int)E, (int)N, (int)K, tiles_n, tiles_k, wait_ns());
+}
+
+int mx_quant_rowwise(const void *in, int64_t rows, int64_t cols, int32_t mode, void *out, uint8_t *scales,
+                     cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0 || cols % 32)
+        return MXQ_ERR_SHAPE;
+    if (mode != MXQ_E8M0_FLOOR && mode != MXQ_E8M0_RCEIL)
+        return MXQ_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0)
+        return MXQ_OK;
+    if (!in || !out || !scales)
+        return MXQ_ERR_NULL;
+    if (!aligned(in, 16) || !aligned(out, 16))
+        return MXQ_ERR_ALIGN;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t nblk = rows * (cols / 32);
+    const int64_t per_cta = (RB_THREADS / 32) * 8 * RB_UNROLL;
+    const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, (int64_t)di->sms * 8);
+    const int wa = aligned(scales, 4) ? 1 : 0;
+    if (mode == MXQ_E8M0_FLOOR)
+        return launch(k_mx_1x32<MXQ_E8M0_FLOOR>, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
+                      static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), scales, wa);
+    return launch(k_mx_1x32<MXQ_E8M0_RCEIL>, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
+                  static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), scales, wa);
+}
+
+int64_t mx_blocked_grouped_rows_bound(int64_t rows, int32_t num_groups)
+{
+    if (rows < 0 || num_groups < 0)
+        return -1;
+    return 128 * ((rows + 127 * (int64_t)num_groups) / 128);
+}
+
+int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t cols, const int32_t *offs,
+                                 int32_t num_groups, uint8_t *out, int64_t out_rows_capacity,
+                                 int32_t *out_group_row_starts, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0 || num_groups < 1 || out_rows_capacity < 0 || out_rows_capacity % 128)
+        return MXQ_ERR_SHAPE;
+    if (!offs || (rows * cols > 0 && !scales) || (out_rows_capacity * cols > 0 && !out))
+        return MXQ_ERR_NULL;
+    if (out_rows_capacity < mx_blocked_grouped_rows_bound(rows, num_groups))
+        return MXQ_ERR_SHAPE;
+    if (num_groups > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if (out && !aligned(out, 16))
+        return MXQ_ERR_ALIGN;
+    const int64_t cols4 = (cols + 3) / 4 * 4;
+    if ((cols4 == 0 || out_rows_capacity == 0) && !out_group_row_starts)
+        return MXQ_OK;
+    const int64_t tiles_c = cols4 / 4;
+    const int64_t gx = std::max<int64_t>((tiles_c + blk::TILES - 1) / blk::TILES, 1);
+    const int64_t gy = std::max<int64_t>(out_rows_capacity / 128, 1);
+    if (gy > 65535)
+        return MXQ_ERR_UNSUPPORTED;
+    const int words_ok = (aligned(scales, 4) && cols % 4 == 0) ? 1 : 0;
+    return launch(k_blocked_grouped, dim3((unsigned)gx, (unsigned)gy), dim3(blk::THREADS), 0, stream, false, scales,
+                  rows, cols, offs, (int)num_groups, out, out_group_row_starts, words_ok,
+                  out_rows_capacity / 128);
+}
+
+int mxq_device_status(cudaStream_t stream, int32_t *host_status)
+{
+    if (!host_status)
+        return MXQ_ERR_NULL;
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return MXQ_ERR_CUDA;
+    *host_status = v;
+    return MXQ_OK;
+}
+
+const char *mxq_status_string(int status)
+{
+    switch (status) {
+    case MXQ_OK: return "ok";
+    case MXQ_ERR_NULL: return "null pointer";
+    case MXQ_ERR_SHAPE: return "invalid shape";
+    case MXQ_ERR_ALIGN: return "misaligned pointer or stride";
+    case MXQ_ERR_UNSUPPORTED: return "unsupported parameters";
+    case MXQ_ERR_LAUNCH: return "kernel launch failed";
+    case MXQ_ERR_BAD_OFFSETS: return "malformed group offsets";
+    case MXQ_ERR_TIMEOUT: return "device wait timed out";
+    case MXQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case MXQ_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+    }
+}
+
+int mxq_version(void) { return 10000; }
+
+int mxq_testing_set(int32_t what, int64_t value)
+{
+    switch (what) {
+    case MXQ_TESTING_WAIT_LIMIT_NS: g_wait_ns.store(value > 0 ? value : 1000000000LL); return MXQ_OK;
+    case MXQ_TESTING_SKIP_ARRIVAL: g_skip_arrival.store(value ? 1 : 0); return MXQ_OK;
+    case MXQ_TESTING_FORCE_PATH:
+        if (value < 0 || value > 2)
+            return MXQ_ERR_UNSUPPORTED;
+        g_force_path.store((int)value);
+        return MXQ_OK;
+    default: return MXQ_ERR_UNSUPPORTED;
+    }
+}
+
+} // extern "C"

@@ -1,0 +1,95 @@
+"""The C-ABI library: it loads without a GPU, exports every function declared
+in include/mxq.h, and its host-side checks reject bad arguments before any
+CUDA call. No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mxfp8_quantization_moe_device_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?\**\s*\**([A-Za-z_][A-Za-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_six_ops():
+    names = declared_functions()
+    for op in ["fp8_quant_jagged_rowwise", "fp8_quant_jagged_colwise", "fp8_quant_blockwise",
+               "mx_quant_3d_colwise", "mx_quant_rowwise", "mx_scales_to_blocked_grouped"]:
+        assert op in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in binding.SIGNATURES, n
+
+
+def test_library_is_built_for_sm100a_only():
+    # nvcc flags of the build: one real-architecture target, sm_100a
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_pure_host_functions(lib):
+    assert lib.mxq_version() >= 10000
+    assert lib.mxq_status_string(0) == b"ok"
+    assert lib.mxq_status_string(6) == b"malformed group offsets"
+    assert lib.mx_blocked_grouped_rows_bound(135, 2) == 384
+    assert lib.mx_blocked_grouped_rows_bound(5, 5) == 640
+    # jagged workspace: only the contiguous-line layout needs one
+    ws = lib.fp8_quant_jagged_workspace_bytes(65536, 4096, 4096, 1, 16, 1)
+    assert ws >= 16 * 4096 * 4 + 64 * 4
+    assert lib.fp8_quant_jagged_workspace_bytes(4096, 65536, 1, 4096, 16, 0) == ws
+    assert lib.fp8_quant_jagged_workspace_bytes(100, 96, 1, 100, 2, 0) == 0  # cols % 16 != 0
+    assert lib.fp8_quant_jagged_workspace_bytes(64, 64, 1, 64, 65, 0) == 0   # too many groups
+
+
+def test_host_checks_return_before_any_cuda_call(lib):
+    null = None
+    fake = ctypes.c_void_p(256)  # never dereferenced: every call below fails a host check first
+    # null pointers
+    assert lib.fp8_quant_blockwise(null, 128, 128, 1, 128, fake, fake, null) == binding.ERR_NULL
+    assert lib.mx_quant_rowwise(fake, 4, 64, 0, null, fake, null) == binding.ERR_NULL
+    assert lib.mx_quant_3d_colwise(fake, 1, 64, 64, 0, fake, null, null) == binding.ERR_NULL
+    assert lib.fp8_quant_jagged_colwise(fake, 4, 4, 4, 1, null, 1, fake, fake, null, 0, null) == binding.ERR_NULL
+    assert lib.mx_scales_to_blocked_grouped(fake, 4, 4, null, 1, fake, 128, null, null) == binding.ERR_NULL
+    # shapes
+    assert lib.fp8_quant_blockwise(fake, 128, 100, 1, 128, fake, fake, null) == binding.ERR_SHAPE
+    assert lib.fp8_quant_blockwise(fake, 100, 128, 128, 128, fake, fake, null) == binding.ERR_SHAPE
+    assert lib.fp8_quant_blockwise(fake, 128, 128, 2, 128, fake, fake, null) == binding.ERR_UNSUPPORTED
+    assert lib.mx_quant_rowwise(fake, 4, 48, 0, fake, fake, null) == binding.ERR_SHAPE
+    assert lib.mx_quant_3d_colwise(fake, 1, 48, 64, 0, fake, fake, null) == binding.ERR_SHAPE
+    assert lib.mx_quant_3d_colwise(fake, 1, 64, 64, 7, fake, fake, null) == binding.ERR_UNSUPPORTED
+    assert lib.fp8_quant_jagged_rowwise(fake, 4, 4, 4, 1, fake, 0, fake, fake, null, 0, null) == binding.ERR_SHAPE
+    assert lib.mx_scales_to_blocked_grouped(fake, 300, 4, fake, 2, fake, 128, null, null) == binding.ERR_SHAPE
+    assert lib.mx_scales_to_blocked_grouped(fake, 4, 4, fake, 1, fake, 100, null, null) == binding.ERR_SHAPE
+    # alignment
+    odd = ctypes.c_void_p(258)
+    assert lib.fp8_quant_blockwise(odd, 128, 128, 1, 128, fake, fake, null) == binding.ERR_ALIGN
+    assert lib.mx_quant_3d_colwise(fake, 1, 64, 60, 0, fake, fake, null) == binding.ERR_ALIGN
+    assert lib.mx_scales_to_blocked_grouped(fake, 4, 4, fake, 1, odd, 128, null, null) == binding.ERR_ALIGN
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros((4, 128), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        binding.fp8_quant_blockwise(x)
+    with pytest.raises(TypeError):
+        binding.mx_quant_rowwise(x)

@@ -1,0 +1,488 @@
+"""GPU parity: every CUDA op, called through the C ABI, against the CPU oracle
+on the same seeded inputs. The bar is bit-exactness: every e4m3 byte, every
+E8M0 byte and every fp32 inverse scale (0 ulp). Small cases are compared in
+full (several tiles plus ragged tails); full-size cases are compared on
+oracle-computed samples plus properties checked over every output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp8_quantization_moe_device_b200 import binding as mxq
+from mxfp8_quantization_moe_device_b200 import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+SENT = 0xA5
+PAD = 256  # guard band bytes around outputs (keeps 16-byte alignment)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    mxq.lib()
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+    yield
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+
+
+def words(t):
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def u8(t):
+    return t.detach().cpu().contiguous().view(torch.uint8).numpy()
+
+
+def f32bits(a):
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+
+
+def guarded(n, dtype=torch.uint8):
+    """A buffer with sentinel margins; returns (whole, inner view)."""
+    esz = torch.tensor([], dtype=dtype).element_size()
+    pad = PAD // esz
+    big = torch.empty(n + 2 * pad, dtype=dtype, device=DEV)
+    big.view(torch.uint8).fill_(SENT)
+    return big, big[pad:pad + n]
+
+
+def margins_intact(big, dtype=torch.uint8):
+    esz = torch.tensor([], dtype=dtype).element_size()
+    pad = PAD // esz
+    b = big.view(torch.uint8).cpu().numpy()
+    return bool(np.all(b[:PAD] == SENT) and np.all(b[-PAD:] == SENT)) and pad > 0
+
+
+def status_ok():
+    return mxq.device_status() == 0
+
+
+# ============================================================ jagged
+
+def _offsets(M, spec, seed=0):
+    if isinstance(spec, str):
+        return synth.multinomial_offsets(M, 4, 16, seed)
+    return torch.tensor(spec, dtype=torch.int32)
+
+
+JAGGED = [
+    (256, 512, "multinomial"),
+    (256, 512, [64, 64, 192, 256]),     # forced-empty group
+    (1040, 200, [0, 5, 5, 700, 1000]),  # ragged sizes, empty groups, rows past the last group
+    (4160, 136, [3000, 3001, 4160]),
+    (64, 64, [64]),
+    (32, 8, [0, 0, 32]),
+    (9600, 72, [17, 4000, 4001, 9583]),  # several position chunks per CTA range
+]
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["single_pass", "generic"])
+@pytest.mark.parametrize("M,D,spec", JAGGED)
+def test_jagged_colwise_and_rowwise_vs_oracle(M, D, spec, path):
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
+    try:
+        x = synth.row_scaled_normal_bf16(M, D, seed=M + D, device=DEV)
+        offs = _offsets(M, spec)
+        end = int(offs[-1])
+        w = words(x).reshape(-1)
+        ref_q, ref_inv = oracle.fp8_quant_jagged_colwise(w, M, D, D, 1, offs.numpy())
+        offs_d = offs.to(DEV)
+
+        # colwise on x: column-major output (D, M)
+        big, out = guarded(D * M)
+        bigi, inv = guarded(offs.numel() * D, torch.float32)
+        q, inv_c = mxq.fp8_quant_jagged_colwise(x, offs_d, out=out.view(D, M), inv_scales=inv.view(-1, D))
+        assert status_ok()
+        got = u8(out).reshape(D, M)
+        assert np.array_equal(got[:, :end], ref_q[:, :end])
+        assert np.all(got[:, end:] == SENT)  # rows past the last group untouched
+        assert np.array_equal(f32bits(inv_c.cpu().numpy()), f32bits(ref_inv))
+        assert margins_intact(big) and margins_intact(bigi, torch.float32)
+
+        # rowwise on the transposed view: byte-identical to colwise (cross-op identity)
+        xt = x.t()
+        ref_qr, ref_invr = oracle.fp8_quant_jagged_rowwise(w, D, M, 1, D, offs.numpy())
+        assert np.array_equal(ref_qr, ref_q)
+        big2, out2 = guarded(D * M)
+        qr, inv_r = mxq.fp8_quant_jagged_rowwise(xt, offs_d, out=out2.view(D, M))
+        assert status_ok()
+        got2 = u8(out2).reshape(D, M)
+        assert np.array_equal(got2[:, :end], ref_qr[:, :end])
+        assert np.all(got2[:, end:] == SENT)
+        assert np.array_equal(f32bits(inv_r.cpu().numpy()), f32bits(ref_invr))
+        assert margins_intact(big2)
+    finally:
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+
+
+@pytest.mark.parametrize("R,C,offs", [(24, 160, [7, 7, 100, 150]), (5, 33, [33]), (130, 64, [1, 2, 64])])
+def test_jagged_rowwise_contiguous_rows_generic(R, C, offs):
+    """Groups along the contiguous dimension (not the transposed view): generic path."""
+    x = synth.row_scaled_normal_bf16(R, C, seed=R * C, device=DEV)
+    o = torch.tensor(offs, dtype=torch.int32)
+    ref_q, ref_inv = oracle.fp8_quant_jagged_rowwise(words(x).reshape(-1), R, C, C, 1, o.numpy())
+    out = torch.full((R, C), SENT, dtype=torch.uint8, device=DEV)
+    q, inv = mxq.fp8_quant_jagged_rowwise(x, o.to(DEV), out=out)
+    assert status_ok()
+    end = offs[-1]
+    got = u8(out)
+    assert np.array_equal(got[:, :end], ref_q[:, :end])
+    assert np.all(got[:, end:] == SENT)
+    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
+
+
+def test_jagged_colwise_strided_view_generic():
+    """colwise on a transposed (non-contiguous) view falls back to the generic kernel."""
+    base = synth.row_scaled_normal_bf16(48, 40, seed=3, device=DEV)
+    x = base.t()  # (40, 48), strides (1, 40)
+    o = torch.tensor([10, 10, 33], dtype=torch.int32)
+    ref_q, ref_inv = oracle.fp8_quant_jagged_colwise(words(base).reshape(-1), 40, 48, 1, 40, o.numpy())
+    q, inv = mxq.fp8_quant_jagged_colwise(x, o.to(DEV))
+    assert status_ok()
+    got = u8(q.t())  # (48 cols, 40 rows) buffer
+    assert np.array_equal(got[:, :33], ref_q[:, :33])
+    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
+
+
+def test_jagged_tiny_config_both_outputs():
+    """The tiny jagged workload: A (256, 512), G=4 multinomial groups of 16-row units;
+    colwise on A and rowwise on A^T."""
+    a, offs = synth.tiny_jagged(device=DEV)
+    w = words(a).reshape(-1)
+    rq, rinv = oracle.fp8_quant_jagged_colwise(w, 256, 512, 512, 1, offs.numpy())
+    q, inv = mxq.fp8_quant_jagged_colwise(a, offs.to(DEV))
+    qr, invr = mxq.fp8_quant_jagged_rowwise(a.t(), offs.to(DEV))
+    assert status_ok()
+    end = int(offs[-1])
+    assert np.array_equal(u8(q.t())[:, :end], rq[:, :end])
+    assert np.array_equal(u8(qr)[:, :end], rq[:, :end])
+    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(rinv))
+    assert np.array_equal(f32bits(invr.cpu().numpy()), f32bits(rinv))
+
+
+def _dequant_error_ok(xg, qg, invg):
+    """Property at any size: |q*inv - x| within half an e4m3 spacing of x*s
+    (scaled back), with s recovered as 1/inv up to one fp32 rounding."""
+    x = xg.float()
+    q = qg.float()
+    s = 1.0 / invg.double()
+    xs = (x.double() * s)
+    mag = xs.abs()
+    e = torch.floor(torch.log2(torch.clamp(mag, min=2.0 ** -6)))
+    spacing = torch.where(mag < 2.0 ** -6, torch.full_like(mag, 2.0 ** -9), torch.exp2(e - 3))
+    return bool(torch.all((q.double() - xs).abs() <= spacing / 2 + mag * 2.0 ** -21)) and bool(torch.all(q.abs() <= 448))
+
+
+@pytest.mark.slow
+def test_jagged_full_size_backward_operands():
+    """grad_out^T rowwise and input colwise at (65536, 4096), G=16 Dirichlet(0.5)
+    groups: oracle on sampled (group, line) units, error bound everywhere."""
+    grad_out, inp, offs = synth.jagged_bwd(device=DEV)
+    offs_d = offs.to(DEV)
+    qc, invc = mxq.fp8_quant_jagged_colwise(inp, offs_d)
+    qr, invr = mxq.fp8_quant_jagged_rowwise(grad_out.t(), offs_d)
+    assert status_ok()
+    rng = np.random.default_rng(0)
+    o = offs.numpy()
+    starts = np.concatenate([[0], o[:-1]])
+    nonempty = [g for g in range(len(o)) if o[g] > starts[g]]
+    for src, q, inv in ((inp, qc.t(), invc), (grad_out, qr, invr)):
+        for _ in range(48):
+            g = int(rng.choice(nonempty))
+            c = int(rng.integers(0, 4096))
+            a, b = int(starts[g]), int(o[g])
+            col = words(src[a:b, c])
+            rq, rinv = oracle.fp8_quant_jagged_colwise(col, b - a, 1, 1, 1, [b - a])
+            assert np.array_equal(u8(q[c, a:b]), rq[0]), (g, c)
+            assert f32bits(inv[g, c].item()) == f32bits(rinv[0, 0])
+        for g in nonempty:
+            a, b = int(starts[g]), int(o[g])
+            assert _dequant_error_ok(src[a:b].t(), q[:, a:b], inv[g][:, None]), g
+
+
+# ============================================================ blockwise
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (37, 384), (256, 512), (1000, 1280)])
+def test_blockwise_1x128_vs_oracle(rows, cols):
+    x = synth.outlier_normal_bf16(rows, cols, seed=rows, device=DEV)
+    rq, rinv = oracle.fp8_quant_blockwise(words(x), 1, 128)
+    big, out = guarded(rows * cols)
+    q, inv = mxq.fp8_quant_blockwise(x, 1, 128, out=out.view(rows, cols))
+    assert status_ok()
+    assert np.array_equal(u8(out).reshape(rows, cols), rq)
+    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(rinv))
+    assert margins_intact(big)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (384, 256), (256, 1280)])
+def test_blockwise_128x128_vs_oracle(rows, cols):
+    x = synth.normal_bf16((rows, cols), 0.02, seed=rows + cols, device=DEV)
+    x[5, 7] = 3.0  # one outlier block
+    rq, rinv = oracle.fp8_quant_blockwise(words(x), 128, 128)
+    big, out = guarded(rows * cols)
+    q, inv = mxq.fp8_quant_blockwise(x, 128, 128, out=out.view(rows, cols))
+    assert status_ok()
+    assert np.array_equal(u8(out).reshape(rows, cols), rq)
+    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(rinv))
+    assert margins_intact(big)
+
+
+@pytest.mark.slow
+def test_blockwise_full_size_llama3_8b_shapes():
+    act = synth.blockwise_act(device=DEV)
+    wt = synth.blockwise_weight(device=DEV)
+    qa, ia = mxq.fp8_quant_blockwise(act, 1, 128)
+    qw, iw = mxq.fp8_quant_blockwise(wt, 128, 128)
+    assert status_ok()
+    rng = np.random.default_rng(1)
+    for _ in range(64):
+        r, b = int(rng.integers(0, 16384)), int(rng.integers(0, 32))
+        rq, ri = oracle.fp8_quant_blockwise(words(act[r:r + 1, b * 128:(b + 1) * 128]), 1, 128)
+        assert np.array_equal(u8(qa[r:r + 1, b * 128:(b + 1) * 128]), rq)
+        assert f32bits(ia[r, b].item()) == f32bits(ri[0, 0])
+    for _ in range(12):
+        bi, bj = int(rng.integers(0, 112)), int(rng.integers(0, 32))
+        blk = wt[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128]
+        rq, ri = oracle.fp8_quant_blockwise(words(blk), 128, 128)
+        assert np.array_equal(u8(qw[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128]), rq)
+        assert f32bits(iw[bi, bj].item()) == f32bits(ri[0, 0])
+    assert _dequant_error_ok(act.view(-1, 128), qa.view(-1, 128), ia.view(-1, 1))
+
+
+# ============================================================ MX
+
+@pytest.mark.parametrize("mode", ["floor", "rceil"])
+@pytest.mark.parametrize("E,N,K", [(1, 64, 64), (3, 96, 200), (2, 256, 128), (1, 160, 8), (4, 128, 320)])
+def test_mx_3d_colwise_vs_oracle(E, N, K, mode):
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=E * N * K, device=DEV, lo=-30, hi=30).view(E, N, K)
+    m = oracle.FLOOR if mode == "floor" else oracle.RCEIL
+    rq, rs = oracle.mx_quant_3d_colwise(w.cpu(), m)
+    big, out = guarded(E * K * N)
+    bigs, sc = guarded(E * K * (N // 32))
+    q, s = mxq.mx_quant_3d_colwise(w, mode, out=out.view(E, K, N), scales=sc.view(E, K, N // 32))
+    assert status_ok()
+    assert q.stride() == (N * K, 1, N)
+    assert np.array_equal(u8(out).reshape(E, K, N), rq)
+    assert np.array_equal(u8(sc).reshape(E, K, N // 32), rs)
+    assert margins_intact(big) and margins_intact(bigs)
+
+
+@pytest.mark.parametrize("mode", ["floor", "rceil"])
+@pytest.mark.parametrize("rows,cols", [(1, 32), (7, 96), (256, 7168 // 8), (300, 4096)])
+def test_mx_rowwise_vs_oracle(rows, cols, mode):
+    x = synth.row_scaled_normal_bf16(rows, cols, seed=rows * 3 + cols, device=DEV, lo=-20, hi=20)
+    m = oracle.FLOOR if mode == "floor" else oracle.RCEIL
+    rq, rs = oracle.mx_quant_rowwise(x.cpu(), m)
+    big, out = guarded(rows * cols)
+    q, s = mxq.mx_quant_rowwise(x, mode, out=out.view(rows, cols))
+    assert status_ok()
+    assert np.array_equal(u8(out).reshape(rows, cols), rq)
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert margins_intact(big)
+
+
+@pytest.mark.parametrize("mode", ["floor", "rceil"])
+def test_mx_scale_rule_exhaustive_over_bf16_amax(mode):
+    """Every non-negative finite bf16 value as a block amax (and its block
+    mates at a few fractions of it): scale bytes and codes match the oracle."""
+    wds = np.arange(0, 0x7F80, dtype=np.uint32)  # +0 .. largest finite
+    amax = (wds << 16).view(np.float32)
+    n = amax.size
+    blk = np.zeros((n, 32), dtype=np.float32)
+    fr = np.array([1.0, -0.5, 0.3, -0.77, 0.01, 0.125, -1e-3, 0.999], dtype=np.float32)
+    blk[:, :8] = amax[:, None] * fr[None, :]
+    x = torch.from_numpy(blk).to(torch.bfloat16)  # fractions rounded to bf16 (<= amax in magnitude)
+    x[:, 0] = torch.from_numpy(amax).to(torch.bfloat16)
+    m = oracle.FLOOR if mode == "floor" else oracle.RCEIL
+    rq, rs = oracle.mx_quant_rowwise(x, m)
+    q, s = mxq.mx_quant_rowwise(x.to(DEV), mode)
+    assert status_ok()
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert np.array_equal(u8(q), rq)
+
+
+def test_e4m3_cast_exhaustive_over_bf16():
+    """At scale byte 127 (factor 1) MX elements are the plain saturating cast:
+    every bf16 pattern with |x| < 512, negative zero and subnormals included."""
+    wds = np.arange(0, 1 << 16, dtype=np.uint32)
+    v = (wds << 16).view(np.float32)
+    v = v[np.isfinite(v) & (np.abs(v) < 448.0)]
+    per = 31
+    nb = (v.size + per - 1) // per
+    blk = np.zeros((nb, 32), dtype=np.float32)
+    blk[:, 0] = 300.0  # floor byte 127 -> factor 1
+    flat = np.zeros(nb * per, dtype=np.float32)
+    flat[: v.size] = v
+    blk[:, 1:] = flat.reshape(nb, per)
+    x = torch.from_numpy(blk).to(torch.bfloat16)
+    rq, rs = oracle.mx_quant_rowwise(x, oracle.FLOOR)
+    assert np.all(rs == 127)
+    q, s = mxq.mx_quant_rowwise(x.to(DEV), "floor")
+    assert status_ok()
+    assert np.array_equal(u8(q), rq)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", ["floor", "rceil"])
+def test_mx_3d_full_size_expert_weights(mode):
+    """(E, 8192, 5120) for E = 1 (every byte vs the oracle) and E = 64
+    (oracle on sampled blocks, scale rule checked on every block)."""
+    m = oracle.FLOOR if mode == "floor" else oracle.RCEIL
+    w1 = synth.mx3d_weight(1, device=DEV)
+    q, s = mxq.mx_quant_3d_colwise(w1, mode)
+    assert status_ok()
+    rq, rs = oracle.mx_quant_3d_colwise(w1.cpu(), m)
+    assert np.array_equal(u8(q.transpose(1, 2)), rq)
+    assert np.array_equal(s.cpu().numpy(), rs)
+    del w1, q, s
+    w = synth.mx3d_weight(64, device=DEV)
+    q, s = mxq.mx_quant_3d_colwise(w, mode)
+    assert status_ok()
+    rng = np.random.default_rng(2)
+    for _ in range(64):
+        e, k, b = int(rng.integers(0, 64)), int(rng.integers(0, 5120)), int(rng.integers(0, 256))
+        col = w[e, b * 32:(b + 1) * 32, k:k + 1].contiguous()
+        rq, rs = oracle.mx_quant_3d_colwise(col.view(1, 32, 1).cpu(), m)
+        assert np.array_equal(u8(q[e, b * 32:(b + 1) * 32, k]), rq.reshape(-1))
+        assert int(s[e, k, b]) == int(rs.reshape(-1)[0])
+    # scale rule on every block: amax / 2^(byte-127) in [256, 512) (floor) or
+    # the smallest power of two putting it <= 448 (rceil)
+    amax = w.float().abs().view(64, 256, 32, 5120).amax(dim=2).transpose(1, 2)  # (E, K, N/32)
+    r = amax.double() * torch.exp2(127.0 - s.double())
+    if mode == "floor":
+        assert bool(torch.all((r < 512) & ((r >= 256) | (s == 0))))
+    else:
+        assert bool(torch.all((r <= 448) & ((r * 2 > 448) | (s == 0))))
+
+
+@pytest.mark.slow
+def test_mx_rowwise_full_size_tokens():
+    x, offs = synth.mx_act(device=DEV)
+    for mode, m in (("floor", oracle.FLOOR), ("rceil", oracle.RCEIL)):
+        q, s = mxq.mx_quant_rowwise(x, mode)
+        assert status_ok()
+        rng = np.random.default_rng(3)
+        rows = np.sort(rng.choice(65536, size=64, replace=False))
+        sub = x[torch.from_numpy(rows).to(DEV)]
+        rq, rs = oracle.mx_quant_rowwise(sub.cpu(), m)
+        assert np.array_equal(u8(q[torch.from_numpy(rows).to(DEV)]), rq)
+        assert np.array_equal(s[torch.from_numpy(rows).to(DEV)].cpu().numpy(), rs)
+
+
+# ============================================================ blocked layout
+
+BLOCKED = [
+    (135, 8, [5, 130]),
+    (129, 7, [0, 128, 1]),        # byte-load path (cols % 4 != 0), empty group
+    (300, 12, [128, 0, 0, 129]),   # rows past the last group
+    (1000, 33, [1, 2, 3, 500, 0, 494]),
+    (64, 224, [64]),
+    (4096, 300, [4000, 96]),
+]
+
+
+@pytest.mark.parametrize("rows,cols,sizes", BLOCKED)
+def test_blocked_grouped_vs_oracle(rows, cols, sizes):
+    s = synth.uniform_u8((rows, cols), 0, 254, seed=rows + cols)
+    offs = torch.tensor(np.cumsum(sizes), dtype=torch.int32)
+    ref, ref_starts = oracle.mx_scales_to_blocked_grouped(s.numpy(), offs.numpy())
+    cap = mxq.blocked_grouped_rows_bound(rows, len(sizes))
+    big, out = guarded(ref.size)
+    o, starts = mxq.mx_scales_to_blocked_grouped(s.to(DEV), offs.to(DEV), capacity_rows=cap, out=out)
+    assert status_ok()
+    assert np.array_equal(u8(out), ref)
+    assert np.array_equal(starts.cpu().numpy(), ref_starts)
+    assert margins_intact(big)
+
+
+@pytest.mark.parametrize("R,C", [(65536, 224), (8192, 512), (5120, 1024), (7168, 2048), (2048, 32768),
+                                 (8192, 4096)])
+def test_blocked_grouped_config_shapes(R, C):
+    """The MX activation scales (65536, 224) with G=64 Dirichlet(0.3) groups and
+    the scale-sweep shapes with G=8 Dirichlet(1.0) groups."""
+    if (R, C) == (65536, 224):
+        offs = synth.dirichlet_offsets(R, 64, 0.3, 8)
+        s = synth.uniform_u8((R, C), 0, 254, seed=9)
+    else:
+        s, offs = synth.scale_sweep(R, C)
+    ref, ref_starts = oracle.mx_scales_to_blocked_grouped(s.numpy(), offs.numpy())
+    o, starts = mxq.mx_scales_to_blocked_grouped(s.to(DEV), offs.to(DEV))
+    assert status_ok()
+    assert np.array_equal(o.cpu().numpy(), ref)
+    assert np.array_equal(starts.cpu().numpy(), ref_starts)
+
+
+# ============================================================ errors and edges
+
+def test_bad_offsets_are_reported_and_nothing_is_written():
+    x = synth.row_scaled_normal_bf16(256, 64, seed=1, device=DEV)
+    for path in (1, 2):
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
+        for bad in ([64, 32, 256], [-16, 256], [64, 272]):
+            out = torch.full((64, 256), SENT, dtype=torch.uint8, device=DEV)
+            mxq.fp8_quant_jagged_colwise(x, torch.tensor(bad, dtype=torch.int32, device=DEV), out=out)
+            assert mxq.device_status() == mxq.ERR_BAD_OFFSETS
+            assert bool(torch.all(out == SENT))
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+    s = torch.zeros((256, 8), dtype=torch.uint8, device=DEV)
+    out = torch.full((mxq.blocked_grouped_rows_bound(256, 2) * 8,), SENT, dtype=torch.uint8, device=DEV)
+    mxq.mx_scales_to_blocked_grouped(s, torch.tensor([200, 100], dtype=torch.int32, device=DEV), out=out)
+    assert mxq.device_status() == mxq.ERR_BAD_OFFSETS
+    assert bool(torch.all(out == SENT))
+    assert mxq.device_status() == 0  # cleared by the read
+
+
+def test_barrier_timeout_is_reported_and_context_survives():
+    """One CTA skips its arrival on the amax barrier: the others' bounded waits
+    expire, the kernel returns, the status reads TIMEOUT and the next call
+    on the same context is correct."""
+    x = synth.row_scaled_normal_bf16(4096, 128, seed=2, device=DEV)
+    offs = torch.tensor([1000, 4096], dtype=torch.int32)
+    try:
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, 1)
+        mxq.testing_set(mxq.TESTING_WAIT_LIMIT_NS, 20_000_000)
+        mxq.testing_set(mxq.TESTING_SKIP_ARRIVAL, 1)
+        mxq.fp8_quant_jagged_colwise(x, offs.to(DEV))
+        assert mxq.device_status() == mxq.ERR_TIMEOUT
+    finally:
+        mxq.testing_set(mxq.TESTING_SKIP_ARRIVAL, 0)
+        mxq.testing_set(mxq.TESTING_WAIT_LIMIT_NS, 0)
+    q, inv = mxq.fp8_quant_jagged_colwise(x, offs.to(DEV))
+    assert status_ok()
+    rq, rinv = oracle.fp8_quant_jagged_colwise(words(x).reshape(-1), 4096, 128, 128, 1, offs.numpy())
+    assert np.array_equal(u8(q.t()), rq)
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+
+
+def test_empty_and_degenerate_inputs():
+    # zero rows: nothing launched, success
+    x0 = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    q, inv = mxq.fp8_quant_blockwise(x0, 1, 128)
+    q, s = mxq.mx_quant_rowwise(torch.empty((0, 64), dtype=torch.bfloat16, device=DEV))
+    assert status_ok()
+    # all groups empty: every inverse scale is the 1e-12 floor's
+    x = torch.randn((16, 32), device=DEV).to(torch.bfloat16)
+    q, inv = mxq.fp8_quant_jagged_colwise(x, torch.zeros(3, dtype=torch.int32, device=DEV))
+    assert status_ok()
+    want = oracle.fp8_inv_scale(0.0)
+    assert np.all(f32bits(inv.cpu().numpy()) == f32bits(np.float32(want)))
+    # all-zero input: codes 0, floor scales
+    z = torch.zeros((256, 128), dtype=torch.bfloat16, device=DEV)
+    q, inv = mxq.fp8_quant_blockwise(z, 128, 128)
+    assert bool(torch.all(q.view(torch.uint8) == 0))
+    q, s = mxq.mx_quant_3d_colwise(z.view(2, 128, 128), "rceil")
+    assert bool(torch.all(s == 0)) and bool(torch.all(q.contiguous().view(torch.uint8) == 0))
+
+
+def test_misaligned_pointers_are_rejected():
+    buf = torch.zeros(4096 + 8, dtype=torch.bfloat16, device=DEV)
+    x = buf[1:1 + 4096].view(32, 128)  # 2-byte offset
+    with pytest.raises(mxq.MXQError) as ei:
+        mxq.fp8_quant_blockwise(x, 1, 128)
+    assert ei.value.code == mxq.ERR_ALIGN
+    with pytest.raises(mxq.MXQError) as ei:
+        mxq.mx_quant_rowwise(x)
+    assert ei.value.code == mxq.ERR_ALIGN
