@@ -189,6 +189,33 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
 int64_t mx_blocked_grouped_rows_bound(int64_t rows, int32_t num_groups);
 
 /* ------------------------------------------------------------------------ *
+ * fp8_quant_jagged_colwise_noalloc - the source pages have no counterpart to
+ * this entry point; it exists for callers that cannot allocate device memory
+ * (a plugin inside a framework that owns all device memory and passes no
+ * workspace, or a path where cudaMalloc's device-wide synchronization is not
+ * acceptable). Same arguments, layout and results as
+ * fp8_quant_jagged_colwise, without the workspace: the scratch is a fixed
+ * array of fp8_quant_jagged_colwise_noalloc_max_scratch_bytes() bytes
+ * (1 MiB) inside the library, held by every GPU that loads it until exit.
+ *   - A problem whose single-pass scratch would exceed that size (see
+ *     fp8_quant_jagged_workspace_bytes with is_colwise = 1) returns
+ *     MXQ_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make it before any stream capture.
+ *   - The call allocates nothing. All calls on a device share the array
+ *     (each clears what it uses first), so calls that overlap on the GPU
+ *     race; serialize them.
+ * ------------------------------------------------------------------------ */
+int fp8_quant_jagged_colwise_noalloc(const void *in, int64_t rows, int64_t cols,
+                                     int64_t stride_row, int64_t stride_col,
+                                     const int32_t *offs, int32_t num_groups,
+                                     void *out, float *inv_scales,
+                                     cudaStream_t stream);
+
+/* Size in bytes of the fixed scratch array of the allocation-free entry point. */
+size_t fp8_quant_jagged_colwise_noalloc_max_scratch_bytes(void);
+
+/* ------------------------------------------------------------------------ *
  * Status and housekeeping
  * ------------------------------------------------------------------------ */
 

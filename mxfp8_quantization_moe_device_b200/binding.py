@@ -32,6 +32,8 @@ SIGNATURES = {
     "fp8_quant_jagged_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "fp8_quant_jagged_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     "fp8_quant_jagged_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64, _i32, _i32]),
+    "fp8_quant_jagged_colwise_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp]),
+    "fp8_quant_jagged_colwise_noalloc_max_scratch_bytes": (_sz, []),
     "fp8_quant_blockwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
@@ -142,6 +144,25 @@ def fp8_quant_jagged_colwise(x, offs, *, out=None, inv_scales=None, workspace=No
     """e4m3 quantization of x (rows, cols), one scale per (column, group),
     groups along rows. Returns (q column-major (rows, cols) view, inv (G, cols))."""
     return _jagged("fp8_quant_jagged_colwise", x, offs, True, out, inv_scales, workspace)
+
+
+def fp8_quant_jagged_colwise_noalloc(x, offs, *, out, inv_scales):
+    """fp8_quant_jagged_colwise through the allocation-free entry point: the
+    library uses its own fixed scratch array, so the caller passes only the
+    preallocated outputs (out: (cols, rows) uint8 buffer, inv_scales: (G, cols)
+    fp32) and nothing is allocated, here or in the library. Calls that
+    overlap on the GPU share that scratch and must be serialized."""
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    dev = x.device
+    _offsets(offs, dev)
+    rows, cols = x.shape
+    sr, sc = x.stride()
+    rc = lib().fp8_quant_jagged_colwise_noalloc(_ptr(x), rows, cols, sr, sc, _ptr(offs), offs.numel(), _ptr(out),
+                                                _ptr(inv_scales), _stream(dev))
+    _check("fp8_quant_jagged_colwise_noalloc", rc)
+    return out.view(torch.float8_e4m3fn).t(), inv_scales
 
 
 # ---------------------------------------------------------------- blockwise

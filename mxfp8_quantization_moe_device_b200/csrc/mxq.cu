@@ -425,6 +425,75 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
                   out_rows_capacity / 128);
 }
 
+} // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of fp8_quant_jagged_colwise.
+//
+// Some callers cannot call cudaMalloc: a plugin running inside a framework
+// that owns all of the device memory and hands it no workspace argument, or
+// a latency-critical path where cudaMalloc's implicit device-wide
+// synchronization is not acceptable. This entry point needs no workspace from
+// them: its scratch (the per-(group, column) amax table and the round
+// counters) lives in the fixed-size array below, which every GPU that loads
+// this library keeps for the life of the process.
+//
+// The array's host-side name is only a stand-in for the device symbol, so its
+// device address is looked up once per device with cudaGetSymbolAddress, with
+// that device current, on the first call made on that device. Make that first
+// call before any stream capture. All calls on a device share the one array
+// and each call clears the part it uses before its kernel runs; calls that
+// overlap on the GPU (on different streams, or from several host threads)
+// race on it and must be serialized by the caller.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20; // 1 MiB per device
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+void *g_noalloc_ptr[128];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(void **out)
+{
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 128)
+        return MXQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[d]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return MXQ_ERR_CUDA;
+        g_noalloc_ptr[d] = p;
+    }
+    *out = g_noalloc_ptr[d];
+    return MXQ_OK;
+}
+
+} // namespace
+
+extern "C" int fp8_quant_jagged_colwise_noalloc(const void *in, int64_t rows, int64_t cols, int64_t stride_row,
+                                                int64_t stride_col, const int32_t *offs, int32_t num_groups,
+                                                void *out, float *inv_scales, cudaStream_t stream)
+{
+    const size_t need = fp8_quant_jagged_workspace_bytes(rows, cols, stride_row, stride_col, num_groups, 1);
+    if (need > kNoAllocScratchBytes)
+        return MXQ_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (need > 0) {
+        const int rc = noalloc_scratch(&scratch);
+        if (rc != MXQ_OK)
+            return rc;
+    }
+    return fp8_quant_jagged_colwise(in, rows, cols, stride_row, stride_col, offs, num_groups, out, inv_scales,
+                                    scratch, need > 0 ? kNoAllocScratchBytes : 0, stream);
+}
+
+extern "C" size_t fp8_quant_jagged_colwise_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" {
+
 int mxq_device_status(cudaStream_t stream, int32_t *host_status)
 {
     if (!host_status)
