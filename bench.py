@@ -49,7 +49,7 @@ KERNEL_NAMES = {
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
     p.add_argument("--experts", type=int, default=64, help="E of the MX 3-D expert-weight op")
@@ -59,6 +59,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--reps", type=int, default=20, help="reps per shape in the per-shape sweep")
+    p.add_argument("--profile-op", default=None, choices=list(Workload.OPS),
+                   help="run only this op (for single-kernel profiler captures)")
+    p.add_argument("--iters", type=int, default=3, help="calls of --profile-op after one warm-up")
     return p.parse_args()
 
 
@@ -98,67 +101,65 @@ def load_traffic(kernel):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons sampled every ~5 ms through NVML
+    during the timed region (nvidia-smi's period is too coarse for it)."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.rows = []
+        self.stop_flag = threading.Event()
+        self.t = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self.nv = None
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+    def _run(self):
+        nv, h = self.nv, self.h
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self.stop_flag.is_set():
+            try:
+                self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), nv.nvmlDeviceGetPowerUsage(h) / 1e3,
+                                  int(get_reasons(h))))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def stop(self):
-        if self.proc is None:
+        if self.t is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
-                                 hw=f[5] == "Active", hwt=f[6] == "Active", swt=f[7] == "Active",
-                                 pcap=f[8] == "Active"))
-            except ValueError:
-                continue
-        if not rows:
+        self.stop_flag.set()
+        self.t.join(timeout=2)
+        if not self.rows:
             return None
-        loaded = [r for r in rows if r["power"] > 300] or rows
-        reasons = []
-        for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                          ("pcap", "sw_power_cap")):
-            if any(r[key] for r in loaded):
-                reasons.append(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
-                "reasons": reasons, "samples": len(loaded)}
+        reasons = [name for name, bit in self.REASONS if any(r[2] & bit for r in self.rows)]
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.smax,
+                "reasons": reasons, "samples": len(self.rows),
+                "power_w_median": round(statistics.median(r[1] for r in self.rows), 1)}
 
 
 # ----------------------------------------------------------------- workload
 
 class Workload:
-    """Device tensors, outputs and the per-op launch closures of one step."""
+    """Device tensors, outputs and the per-op launch closures of one step.
+    `only` restricts construction to the tensors of one op (profiling)."""
 
-    def __init__(self, dev, experts, mx3d_mode, with_outputs=True):
+    OPS = ("blockwise_1x128", "blockwise_128x128", "jagged_rowwise", "jagged_colwise", "mx_3d_colwise",
+           "mx_rowwise", "blocked_grouped")
+
+    def __init__(self, dev, experts, mx3d_mode, only=None):
         import torch
         from mxfp8_quantization_moe_device_b200 import binding as mxq
         from mxfp8_quantization_moe_device_b200 import synth
@@ -167,65 +168,90 @@ class Workload:
         self.experts = experts
         self.mx3d_mode = mx3d_mode
         t = torch
-        self.act = synth.blockwise_act(device=dev)
-        self.wt = synth.blockwise_weight(device=dev)
-        self.grad_out, self.inp, offs16 = synth.jagged_bwd(device=dev)
-        self.offs16 = offs16.to(dev)
-        self.w3 = synth.mx3d_weight(experts, device=dev)
-        self.tok, offs64 = synth.mx_act(device=dev)
-        self.offs64 = offs64.to(dev)
-        M, D = self.inp.shape
-        E, N, K = self.w3.shape
-        T, KT = self.tok.shape
+        want = set(self.OPS if only is None else [only])
         u8 = dict(dtype=t.uint8, device=dev)
         f32 = dict(dtype=t.float32, device=dev)
-        self.o = dict(
-            act_q=t.empty(self.act.shape, **u8), act_s=t.empty((16384, 32), **f32),
-            wt_q=t.empty(self.wt.shape, **u8), wt_s=t.empty((112, 32), **f32),
-            go_q=t.empty((D, M), **u8), go_s=t.empty((16, D), **f32),
-            in_q=t.empty((D, M), **u8), in_s=t.empty((16, D), **f32),
-            w3_q=t.empty((E, K, N), **u8), w3_s=t.empty((E, K, N // 32), **u8),
-            tok_q=t.empty((T, KT), **u8), tok_s=t.empty((T, KT // 32), **u8),
-        )
-        cap = mxq.blocked_grouped_rows_bound(T, 64)
-        self.cap = cap
-        self.o["blk"] = t.empty(cap * ((KT // 32 + 3) // 4 * 4), **u8)
-        self.o["blk_starts"] = t.empty(64, dtype=t.int32, device=dev)
-        ws_r = mxq.jagged_workspace_bytes(D, M, 1, D, 16, False)
-        ws_c = mxq.jagged_workspace_bytes(M, D, D, 1, 16, True)
-        self.ws_r = t.empty(max(ws_r, 1), **u8)
-        self.ws_c = t.empty(max(ws_c, 1), **u8)
-        self.ops = self._ops()
-
-    def _ops(self):
-        mxq, o = self.mxq, self.o
-        E, N, K = self.w3.shape
-        T, KT = self.tok.shape
-        M, D = self.inp.shape
-        G16 = 16
-        ops = [
-            ("blockwise_1x128", lambda: mxq.fp8_quant_blockwise(self.act, 1, 128, out=o["act_q"], inv_scales=o["act_s"]),
-             16384 * 4096 * 3 + 16384 * 32 * 4),
-            ("blockwise_128x128", lambda: mxq.fp8_quant_blockwise(self.wt, 128, 128, out=o["wt_q"], inv_scales=o["wt_s"]),
-             14336 * 4096 * 3 + 112 * 32 * 4),
-            ("jagged_rowwise", lambda: mxq.fp8_quant_jagged_rowwise(self.grad_out.t(), self.offs16, out=o["go_q"],
-                                                                   inv_scales=o["go_s"], workspace=self.ws_r),
-             M * D * 3 + G16 * D * 4),
-            ("jagged_colwise", lambda: mxq.fp8_quant_jagged_colwise(self.inp, self.offs16, out=o["in_q"],
-                                                                   inv_scales=o["in_s"], workspace=self.ws_c),
-             M * D * 3 + G16 * D * 4),
-            ("mx_3d_colwise", lambda: mxq.mx_quant_3d_colwise(self.w3, self.mx3d_mode, out=o["w3_q"], scales=o["w3_s"]),
-             E * N * K * 3 + E * K * N // 32),
-            ("mx_rowwise", lambda: mxq.mx_quant_rowwise(self.tok, "floor", out=o["tok_q"], scales=o["tok_s"]),
-             T * KT * 3 + T * KT // 32),
-            ("blocked_grouped", lambda: mxq.mx_scales_to_blocked_grouped(o["tok_s"], self.offs64, capacity_rows=self.cap,
-                                                                        out=o["blk"], group_row_starts=o["blk_starts"]),
-             T * (KT // 32) + self.cap * ((KT // 32 + 3) // 4 * 4)),
-        ]
-        return ops
+        self.o = {}
+        self.ops = []
+        if "blockwise_1x128" in want:
+            self.act = synth.blockwise_act(device=dev)
+            self.o.update(act_q=t.empty(self.act.shape, **u8), act_s=t.empty((16384, 32), **f32))
+            self.ops.append(("blockwise_1x128", lambda: mxq.fp8_quant_blockwise(
+                self.act, 1, 128, out=self.o["act_q"], inv_scales=self.o["act_s"]), 16384 * 4096 * 3 + 16384 * 32 * 4))
+        if "blockwise_128x128" in want:
+            self.wt = synth.blockwise_weight(device=dev)
+            self.o.update(wt_q=t.empty(self.wt.shape, **u8), wt_s=t.empty((112, 32), **f32))
+            self.ops.append(("blockwise_128x128", lambda: mxq.fp8_quant_blockwise(
+                self.wt, 128, 128, out=self.o["wt_q"], inv_scales=self.o["wt_s"]), 14336 * 4096 * 3 + 112 * 32 * 4))
+        if want & {"jagged_rowwise", "jagged_colwise"}:
+            self.grad_out, self.inp, offs16 = synth.jagged_bwd(device=dev)
+            self.offs16 = offs16.to(dev)
+            M, D = self.inp.shape
+            jb = M * D * 3 + 16 * D * 4
+            if "jagged_rowwise" in want:
+                self.o.update(go_q=t.empty((D, M), **u8), go_s=t.empty((16, D), **f32))
+                self.ws_r = t.empty(max(mxq.jagged_workspace_bytes(D, M, 1, D, 16, False), 1), **u8)
+                self.ops.append(("jagged_rowwise", lambda: mxq.fp8_quant_jagged_rowwise(
+                    self.grad_out.t(), self.offs16, out=self.o["go_q"], inv_scales=self.o["go_s"],
+                    workspace=self.ws_r), jb))
+            if "jagged_colwise" in want:
+                self.o.update(in_q=t.empty((D, M), **u8), in_s=t.empty((16, D), **f32))
+                self.ws_c = t.empty(max(mxq.jagged_workspace_bytes(M, D, D, 1, 16, True), 1), **u8)
+                self.ops.append(("jagged_colwise", lambda: mxq.fp8_quant_jagged_colwise(
+                    self.inp, self.offs16, out=self.o["in_q"], inv_scales=self.o["in_s"], workspace=self.ws_c), jb))
+        if "mx_3d_colwise" in want:
+            self.w3 = synth.mx3d_weight(experts, device=dev)
+            E, N, K = self.w3.shape
+            self.o.update(w3_q=t.empty((E, K, N), **u8), w3_s=t.empty((E, K, N // 32), **u8))
+            self.ops.append(("mx_3d_colwise", lambda: mxq.mx_quant_3d_colwise(
+                self.w3, self.mx3d_mode, out=self.o["w3_q"], scales=self.o["w3_s"]), E * N * K * 3 + E * K * N // 32))
+        if want & {"mx_rowwise", "blocked_grouped"}:
+            self.tok, offs64 = synth.mx_act(device=dev)
+            self.offs64 = offs64.to(dev)
+            T, KT = self.tok.shape
+            self.o.update(tok_q=t.empty((T, KT), **u8), tok_s=t.empty((T, KT // 32), **u8))
+            if "mx_rowwise" in want:
+                self.ops.append(("mx_rowwise", lambda: mxq.mx_quant_rowwise(
+                    self.tok, "floor", out=self.o["tok_q"], scales=self.o["tok_s"]), T * KT * 3 + T * KT // 32))
+            if "blocked_grouped" in want:
+                if "mx_rowwise" not in want:
+                    mxq.mx_quant_rowwise(self.tok, "floor", out=self.o["tok_q"], scales=self.o["tok_s"])
+                self.cap = mxq.blocked_grouped_rows_bound(T, 64)
+                c4 = (KT // 32 + 3) // 4 * 4
+                self.o.update(blk=t.empty(self.cap * c4, **u8), blk_starts=t.empty(64, dtype=t.int32, device=dev))
+                self.ops.append(("blocked_grouped", lambda: mxq.mx_scales_to_blocked_grouped(
+                    self.o["tok_s"], self.offs64, capacity_rows=self.cap, out=self.o["blk"],
+                    group_row_starts=self.o["blk_starts"]), T * (KT // 32) + self.cap * c4))
 
     def step_bytes(self):
         return sum(b for _, _, b in self.ops)
+
+
+def profile_op(args):
+    """Run one op of the workload `iters` times after one warm-up call (for
+    ncu captures of a single kernel) and print its event-timed durations."""
+    import torch
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = Workload(dev, args.experts, args.mx3d_mode, only=args.profile_op)
+    name, fn, nbytes = wl.ops[0]
+    fn()
+    torch.cuda.synchronize()
+    res = []
+    for _ in range(args.iters):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        us = a.elapsed_time(b) * 1e3
+        res.append({"us": round(us, 2), "GB/s": round(nbytes / (us * 1e-6) / 1e9, 1)})
+    status = wl.mxq.device_status()
+    print(json.dumps({"op": name, "experts": args.experts, "mode": args.mx3d_mode, "bytes": nbytes,
+                      "runs": res, "status": status}))
+    if status != 0:
+        raise SystemExit(f"device status {status}")
 
 
 def time_steps(wl, steps, warmup, per_op=True):
@@ -434,6 +460,8 @@ def main():
         os.environ["CUDA_VISIBLE_DEVICES"] = str(local)
     import torch
 
+    if args.profile_op:
+        return profile_op(args)
     if args.impl == "reference":
         return main_reference(args, world, rank)
 

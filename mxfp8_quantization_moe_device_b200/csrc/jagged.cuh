@@ -17,22 +17,33 @@
 // Two kernels:
 //   k_jagged_generic  any strides: one warp per (line, group), two passes
 //                     over the group's elements (amax, then cast).
-//   k_jagged_fused    contiguous lines: a single pass in one cooperative
-//                     launch. Each CTA owns a fixed range of positions and
-//                     walks the lines in rounds of 64. Per round it TMA-loads
-//                     its (positions x 64 lines) slab into shared memory
-//                     (a 3-stage ring), reduces the per-(group, line) amax of
-//                     its rows and merges it into a global amax table with
-//                     atomicMax on the fp32 bit pattern (exact and order-free
-//                     for non-negative values), then arrives on the round's
-//                     counter. One round later (so the wait overlaps the next
-//                     round's loads and reduction) it waits for all CTAs,
-//                     reads the final amax of its groups, casts the slab it
-//                     still holds in shared memory and writes the transpose
-//                     through a 64B-swizzled staging buffer with TMA stores.
-//                     HBM traffic is the algorithmic 2 B read + 1 B written
-//                     per element; skewed or empty groups only change how
-//                     many rows of a CTA's range fall in each group.
+//   k_jagged_fused    contiguous lines: one cooperative launch that keeps
+//                     the HBM traffic near the algorithmic 2 B read + 1 B
+//                     written per element by reading every strip twice, once
+//                     from HBM and once from L2. Each CTA owns a fixed range of
+//                     positions; the lines are walked in strips of 256 (512
+//                     contiguous bytes per position row, 32 MB per strip at
+//                     65536 positions). Warp roles per CTA:
+//                       - producer A streams strip r of the CTA's rows from HBM
+//                         through a 12-deep TMA ring (evict-last L2 policy);
+//                       - four amax warps reduce the per-(group, line) amax of
+//                         each box (tree max over 16 rows when the box lies in
+//                         one group), merge it in shared memory and then into
+//                         a global table with atomicMax on the fp32 bit
+//                         pattern (exact and order-free for non-negative
+//                         values), and arrive on the strip's counter;
+//                       - producer B re-streams the same rows out of L2 through
+//                         a second ring (evict-first); its data never depends
+//                         on the barrier, so it simply runs ahead;
+//                       - eight cast warps wait until every CTA has arrived for
+//                         the strip, read their groups' final amax from L2,
+//                         cast, and write the transpose through a 64B-swizzled
+//                         staging tile with TMA stores.
+//                     The amax warps start strip r+2 only after the cast of
+//                     strip r is done, so at most two strips are live in L2
+//                     while HBM reads and writes overlap. Skewed or empty
+//                     groups only change how many rows of a range fall in
+//                     each group.
 #pragma once
 
 #include "common.cuh"
@@ -91,24 +102,31 @@ __global__ void __launch_bounds__(256) k_jagged_generic(const uint16_t *__restri
 }
 
 // ---------------------------------------------------------------------------
-// Single-pass cooperative path (contiguous lines).
+// Single-pass-over-HBM cooperative path (contiguous lines).
 // ---------------------------------------------------------------------------
 namespace jag {
 
-constexpr int W = 64;                 // lines per round (128 B of bf16 per position)
-constexpr int CWARPS = 8;             // consumer warps
-constexpr int THREADS = (CWARPS + 1) * 32;
-constexpr int BOXP = 32;              // positions per TMA load box
-constexpr int OBOX = 64;              // positions per TMA store box (64 B, 64B swizzle)
-constexpr int MAX_SEG = 64;           // groups a CTA's range may intersect (host checks G)
+constexpr int W = 256;                    // lines per strip (512 B of bf16 per position)
+constexpr int BWARPS = 8;                 // cast warps (pass B)
+constexpr int AWARPS = 4;                 // amax warps (pass A)
+constexpr int NB = BWARPS * 32;           // cast threads: 0 .. NB-1
+constexpr int NA = AWARPS * 32;           // amax threads: NB .. NB+NA-1
+constexpr int THREADS = NB + NA + 64;     // + two producer warps (HBM ring, L2 ring)
+constexpr int BOXR = 16;                  // positions per TMA load box
+constexpr int BOX_BYTES = W * 2 * BOXR;   // 8 KB
+constexpr int OPOS = 64;                  // positions per TMA store box (64 B rows, 64B swizzle)
+constexpr int OBOX_BYTES = OPOS * W;      // 16 KB
+constexpr int GROUP_BOXES = OPOS / BOXR;  // load boxes per store box
+constexpr int SA = 12;                    // HBM ring (pass A): 96 KB in flight
+constexpr int SB = 8;                     // L2 ring (pass B): two store boxes ahead
+constexpr int ASEG = 8;                   // segments reduced in shared memory (more go to global)
+constexpr int MAX_SEG = 64;               // groups a CTA's range may intersect (host checks G)
 
 struct Params {
     int64_t L, P;          // lines, positions
     int G;
-    int chunk;             // positions per CTA (multiple of OBOX)
-    int stages;            // TMA ring depth
-    int rounds;            // ceil(L / W)
-    int nseg_cap;          // segment-table capacity (>= min(G, ...))
+    int chunk;             // positions per CTA (multiple of OPOS)
+    int rounds;            // strips: ceil(L / W)
     const int32_t *offs;
     uint8_t *out;          // out[l * P + p]
     float *inv;
@@ -119,37 +137,78 @@ struct Params {
 };
 
 // shared memory carve-up (byte offsets from a 1024-aligned base)
-struct Layout {
-    int in_off, in_stage_bytes;
-    int stg_off;           // output staging: chunk/64 boxes of 64 x 64 bytes
-    int stab_off;          // scale table: nseg_cap x W floats
-    int red_off;           // CWARPS x 32 words
-    int bar_off;           // full[stages], empty[stages]
-    int misc_off;          // small ints
-    int total;
-};
-
-__host__ __device__ inline Layout layout(int chunk, int stages, int nseg_cap)
-{
-    Layout y;
-    y.in_off = 0;
-    y.in_stage_bytes = chunk * W * 2;
-    y.stg_off = stages * y.in_stage_bytes;               // multiple of 1024 (chunk % 64 == 0)
-    y.stab_off = y.stg_off + chunk * W;
-    y.red_off = y.stab_off + nseg_cap * W * 4;
-    y.bar_off = y.red_off + CWARPS * 32 * 4;
-    y.misc_off = y.bar_off + 2 * stages * 8;
-    y.total = y.misc_off + 64;
-    return y;
-}
+constexpr int RA_OFF = 0;
+constexpr int RB_OFF = RA_OFF + SA * BOX_BYTES;
+constexpr int STG_OFF = RB_OFF + SB * BOX_BYTES;
+constexpr int ATAB_OFF = STG_OFF + 2 * OBOX_BYTES;
+constexpr int BAR_OFF = ATAB_OFF + ASEG * W * 4;
+constexpr int SMEM_TOTAL = BAR_OFF + 2 * (SA + SB) * 8;
+constexpr size_t SMEM_BYTES = SMEM_TOTAL + 1024; // + manual 1 KB alignment
 
 struct Misc {
     int nseg;              // non-empty group segments of this CTA's range
     int abort_flag;
+    int b_done;            // strips whose cast (pass B) this CTA has finished
     int seg_g[MAX_SEG];    // group of each segment
     int seg_lo[MAX_SEG];   // segment rows, relative to the range start
     int seg_hi[MAX_SEG];
 };
+
+MXQ_DEV uint64_t policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+MXQ_DEV uint64_t policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+MXQ_DEV void tma_load_2d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+
+MXQ_DEV void tma_store_2d_hint(const CUtensorMap *map, const void *src, int x, int y, uint64_t pol)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint"
+                 " [%0, {%2, %3}], [%1], %4;" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "l"(pol)
+                 : "memory");
+}
+
+// max of |a|, |b| over packed bf16 pairs
+MXQ_DEV uint32_t absmax2(uint32_t a, uint32_t b) { return absmax_bf16x2(a & 0x7FFF7FFFu, b); }
+
+// fill `n` boxes of TMA ring (stages S, barriers full/empty) with the boxes
+// `first..first+n-1` of a pass; `seq` counts boxes through the ring
+MXQ_DEV bool ring_fill(uint8_t *ring, uint64_t *full, uint64_t *empty, int S, int &seq, const CUtensorMap *map,
+                       int x, int64_t y0, int n, uint64_t pol, uint64_t wait_ns)
+{
+    for (int b = 0; b < n; ++b, ++seq) {
+        const int s = seq % S;
+        if (seq >= S && !mbar_wait(&empty[s], ((uint32_t)(seq / S) & 1u) ^ 1u, wait_ns))
+            return false;
+        mbar_arrive_expect_tx(&full[s], BOX_BYTES);
+        tma_load_2d_hint(ring + s * BOX_BYTES, map, &full[s], x, (int)(y0 + b * BOXR), pol);
+    }
+    return true;
+}
+
+MXQ_DEV void ring_drain(uint64_t *full, int S, int seq, uint64_t wait_ns)
+{
+    for (int j = seq - S; j < seq; ++j)
+        if (j >= 0)
+            mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, wait_ns);
+}
 
 } // namespace jag
 
@@ -160,145 +219,102 @@ __global__ void __launch_bounds__(jag::THREADS, 1)
     using namespace jag;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const Layout y = layout(p.chunk, p.stages, p.nseg_cap);
-    uint8_t *in_s = base + y.in_off;
-    uint8_t *stg = base + y.stg_off;
-    float *stab = reinterpret_cast<float *>(base + y.stab_off);
-    uint32_t *red = reinterpret_cast<uint32_t *>(base + y.red_off);
-    uint64_t *full = reinterpret_cast<uint64_t *>(base + y.bar_off);
-    uint64_t *empty = full + p.stages;
+    uint8_t *ring_a = base + RA_OFF;
+    uint8_t *ring_b = base + RB_OFF;
+    uint8_t *stg = base + STG_OFF;
+    uint32_t *atab = reinterpret_cast<uint32_t *>(base + ATAB_OFF); // amax bits of segments < ASEG
+    uint64_t *full_a = reinterpret_cast<uint64_t *>(base + BAR_OFF);
+    uint64_t *empty_a = full_a + SA;
+    uint64_t *full_b = empty_a + SA;
+    uint64_t *empty_b = full_b + SB;
     __shared__ Misc mi;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ncta = gridDim.x;
     const int64_t lo = (int64_t)blockIdx.x * p.chunk;
-    // offsets are validated by every CTA identically, so all of them return
-    // together on bad offsets and no barrier is left waiting
+    // every CTA validates the same offsets, so on bad offsets all return
+    // together and no barrier is left waiting
     if (!offsets_ok(p.offs, p.G, p.P))
         return;
     const int64_t end_all = p.offs[p.G - 1];
-    const int64_t hi = min(lo + (int64_t)p.chunk, end_all); // rows this CTA quantizes
+    const int64_t hi = min(lo + (int64_t)p.chunk, end_all);
+    const int rows_here = hi > lo ? (int)(hi - lo) : 0;
+    const int nbox = (rows_here + BOXR - 1) / BOXR;
+    const int ngroups = (nbox + GROUP_BOXES - 1) / GROUP_BOXES;
 
     if (threadIdx.x == 0) {
-        // segments: the non-empty groups intersecting [lo, hi), in order,
-        // each clipped to the range; together they tile [lo, hi)
+        // non-empty groups intersecting [lo, hi), clipped: they tile [0, rows_here)
         int n = 0;
-        if (hi > lo) {
+        if (rows_here > 0) {
             int a = 0, b = p.G - 1; // first group with end > lo
             while (a < b) {
                 const int m = (a + b) >> 1;
                 if (p.offs[m] > lo) b = m; else a = m + 1;
             }
-            for (int g = a; g < p.G; ++g) {
+            for (int g = a; g < p.G && n < MAX_SEG; ++g) {
                 const int64_t gs = g ? p.offs[g - 1] : 0, ge = p.offs[g];
                 if (gs >= hi)
                     break;
                 if (ge == gs)
                     continue;
-                if (n < MAX_SEG) {
-                    mi.seg_g[n] = g;
-                    mi.seg_lo[n] = (int)(max(gs, lo) - lo);
-                    mi.seg_hi[n] = (int)(min(ge, hi) - lo);
-                }
+                mi.seg_g[n] = g;
+                mi.seg_lo[n] = (int)(max(gs, lo) - lo);
+                mi.seg_hi[n] = (int)(min(ge, hi) - lo);
                 ++n;
             }
         }
         mi.nseg = n;
         mi.abort_flag = 0;
-        for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], CWARPS);
+        mi.b_done = 0;
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&empty_a[s], AWARPS);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty_b[s], BWARPS);
         }
         fence_mbar_init();
     }
     __syncthreads();
-    // nseg <= G <= nseg_cap <= MAX_SEG: the host only takes this path then
-    
     const int nseg = mi.nseg;
     const int R = p.rounds;
-    const int nbox = p.chunk / BOXP;
-    const uint32_t stage_bytes = (uint32_t)y.in_stage_bytes;
+    const int64_t L = p.L;
+    constexpr int PRODUCER_A = (NB + NA) / 32, PRODUCER_B = PRODUCER_A + 1;
 
-    if (warp == CWARPS) {
-        // ------------------------------------------------ producer warp
+    if (warp >= PRODUCER_A) {
+        // ------------------------------------------------ producer warps
+        // PRODUCER_A streams the strips from HBM for pass A, keeping them in
+        // L2; PRODUCER_B streams them again out of L2 for pass B. B's data
+        // does not depend on the amax barrier (only its scales do), so its
+        // producer just runs ahead within its ring.
         if (lane == 0) {
-            int r = 0;
-            for (; r < R; ++r) {
-                const int s = r % p.stages;
-                const uint32_t ph = (uint32_t)(r / p.stages) & 1u;
-                if (r >= p.stages && !mbar_wait(&empty[s], ph ^ 1u, p.wait_ns))
+            const bool is_a = warp == PRODUCER_A;
+            const uint64_t pol = is_a ? policy_evict_last() : policy_evict_first();
+            uint8_t *ring = is_a ? ring_a : ring_b;
+            uint64_t *full = is_a ? full_a : full_b, *empty = is_a ? empty_a : empty_b;
+            const int S = is_a ? SA : SB;
+            int seq = 0;
+            for (int r = 0; r < R; ++r)
+                if (!ring_fill(ring, full, empty, S, seq, &tm_in, r * W, lo, nbox, pol, p.wait_ns))
                     break;
-                mbar_arrive_expect_tx(&full[s], stage_bytes);
-                uint8_t *dst = in_s + (size_t)s * stage_bytes;
-                for (int b = 0; b < nbox; ++b)
-                    tma_load_2d(dst + b * BOXP * W * 2, &tm_in, &full[s], r * W, (int)(lo + b * BOXP));
-            }
-            for (int j = r - p.stages; j < r; ++j)
-                if (j >= 0)
-                    mbar_wait(&full[j % p.stages], (uint32_t)(j / p.stages) & 1u, p.wait_ns);
+            ring_drain(full, S, seq, p.wait_ns);
         }
         return;
     }
 
-    // ---------------------------------------------------- consumer warps
-    const int ctid = threadIdx.x;              // 0 .. CWARPS*32-1
-    const int NC = CWARPS * 32;
-    const int64_t L = p.L;
-    for (int r = 0; r <= R; ++r) {
-        // ---- phase 1 of round r: per-(group, line) amax of this CTA's rows
-        if (r < R) {
-            const int s = r % p.stages;
-            const uint32_t ph = (uint32_t)(r / p.stages) & 1u;
-            bool ok = mbar_wait(&full[s], ph, p.wait_ns);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok)
-                mi.abort_flag = 1;
-            const uint32_t *slab = reinterpret_cast<const uint32_t *>(in_s + (size_t)s * stage_bytes);
-            const int64_t l0 = (int64_t)r * W + 2 * lane; // this lane's line pair
-            for (int sg = 0; sg < nseg; ++sg) {
-                const int a = mi.seg_lo[sg], b = mi.seg_hi[sg];
-                uint32_t acc = 0;
-                int i = a + warp;
-                for (; i + 3 * CWARPS < b; i += 4 * CWARPS) {
-                    const uint32_t x0 = slab[(i + 0 * CWARPS) * 32 + lane];
-                    const uint32_t x1 = slab[(i + 1 * CWARPS) * 32 + lane];
-                    const uint32_t x2 = slab[(i + 2 * CWARPS) * 32 + lane];
-                    const uint32_t x3 = slab[(i + 3 * CWARPS) * 32 + lane];
-                    acc = absmax_bf16x2(absmax_bf16x2(acc, x0), x1);
-                    acc = absmax_bf16x2(absmax_bf16x2(acc, x2), x3);
-                }
-                for (; i < b; i += CWARPS)
-                    acc = absmax_bf16x2(acc, slab[i * 32 + lane]);
-                red[warp * 32 + lane] = acc;
-                named_barrier(1, NC);
-                if (ctid < 32) {
-                    uint32_t m = red[ctid];
-                    for (int k = 1; k < CWARPS; ++k)
-                        m = absmax_bf16x2(m, red[k * 32 + ctid]);
-                    const int g = mi.seg_g[sg];
-                    unsigned *dst = p.amax + (int64_t)g * L;
-                    // skip lines past L; an amax of 0 never changes the table
-                    const float a0 = bf16_lo(m), a1 = bf16_hi(m);
-                    if (l0 < L && a0 > 0.0f)
-                        atomicMax(dst + l0, __float_as_uint(a0));
-                    if (l0 + 1 < L && a1 > 0.0f)
-                        atomicMax(dst + l0 + 1, __float_as_uint(a1));
-                }
-                named_barrier(1, NC);
-            }
-            if (ctid == 0 && !(p.skip_arrival && blockIdx.x == 0)) {
-                __threadfence();
-                red_release_gpu_add(p.counters + r, 1);
-            }
-        }
-        // ---- phase 2 of round r-1: wait for every CTA, cast, store
-        if (r >= 1) {
-            const int rr = r - 1;
-            const int s = rr % p.stages;
-            if (ctid == 0) {
-                bulk_wait_read<0>(); // staging free again
+    if (warp >= BWARPS) {
+        // ------------------------------------------------ amax warps (pass A)
+        // thread = one line pair, all 16 rows of each box
+        const int ta = threadIdx.x - NB;
+        const int lp = ta;
+        int seq = 0;
+        for (int r = 0; r < R; ++r) {
+            // keep at most two strips live in L2: strip r may start once this
+            // CTA's cast of strip r-2 is done
+            if (r >= 2 && ta == 0) {
                 const uint64_t t0 = globaltimer();
-                while (ld_acquire_gpu(p.counters + rr) < ncta) {
+                while (*(volatile int *)&mi.b_done < r - 1 && !*(volatile int *)&mi.abort_flag) {
                     if (globaltimer() - t0 > p.wait_ns) {
                         set_status(MXQ_ERR_TIMEOUT);
                         mi.abort_flag = 1;
@@ -306,123 +322,235 @@ __global__ void __launch_bounds__(jag::THREADS, 1)
                     }
                 }
             }
-            named_barrier(1, NC);
-            if (mi.abort_flag)
+            for (int i = ta; i < ASEG * W; i += NA)
+                atab[i] = 0u;
+            named_barrier(2, NA);
+            if (*(volatile int *)&mi.abort_flag)
                 break;
-            // scale table for this round's lines
-            for (int t = ctid; t < nseg * W; t += NC) {
-                const int sg = t / W, li = t % W;
-                const int64_t l = (int64_t)rr * W + li;
-                float s = 0.0f;
-                if (l < L)
-                    s = fp8_scale(__uint_as_float(__ldcg(p.amax + (int64_t)mi.seg_g[sg] * L + l)));
-                stab[sg * W + li] = s;
-            }
-            // inverse scales of the groups this CTA is responsible for
-            for (int g = blockIdx.x; g < p.G; g += ncta) {
-                for (int li = ctid; li < W; li += NC) {
-                    const int64_t l = (int64_t)rr * W + li;
-                    if (l < L)
-                        p.inv[(int64_t)g * L + l] = fp8_inv(fp8_scale(__uint_as_float(__ldcg(p.amax + (int64_t)g * L + l))));
+            const int64_t la = (int64_t)r * W + 2 * lp;
+            int cs = 0;
+            int next = nseg ? mi.seg_hi[0] : 0;
+            uint32_t acc = 0;
+            auto flush = [&](int seg, uint32_t v) {
+                if (!v)
+                    return;
+                if (seg < ASEG) {
+                    atomicMax(&atab[seg * W + 2 * lp], v << 16);
+                    atomicMax(&atab[seg * W + 2 * lp + 1], v & 0xFFFF0000u);
+                } else {
+                    unsigned *dst = p.amax + (int64_t)mi.seg_g[seg] * L + la;
+                    if (la < L)
+                        atomicMax(dst, v << 16);
+                    if (la + 1 < L)
+                        atomicMax(dst + 1, v & 0xFFFF0000u);
+                }
+            };
+            for (int b = 0; b < nbox; ++b, ++seq) {
+                const int s = seq % SA;
+                bool ok = mbar_wait(&full_a[s], (uint32_t)(seq / SA) & 1u, p.wait_ns);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok)
+                    mi.abort_flag = 1;
+                const uint32_t *bp = reinterpret_cast<const uint32_t *>(ring_a + s * BOX_BYTES) + lp;
+                uint32_t v[BOXR];
+#pragma unroll
+                for (int k = 0; k < BOXR; ++k)
+                    v[k] = bp[k * (W / 2)];
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty_a[s]);
+                const int row0 = b * BOXR;
+                const int rlast = row0 + BOXR - 1;
+                if (rlast < next && rlast < rows_here) {
+                    // all 16 rows valid and in the current segment
+                    uint32_t m0 = absmax2(absmax2(absmax2(v[0], v[1]), absmax2(v[2], v[3])),
+                                          absmax2(absmax2(v[4], v[5]), absmax2(v[6], v[7])));
+                    uint32_t m1 = absmax2(absmax2(absmax2(v[8], v[9]), absmax2(v[10], v[11])),
+                                          absmax2(absmax2(v[12], v[13]), absmax2(v[14], v[15])));
+                    acc = absmax_bf16x2(absmax_bf16x2(acc, m0), m1);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < BOXR; ++k) {
+                        const int row = row0 + k;
+                        if (row < rows_here) {
+                            if (row >= next) {
+                                flush(cs, acc);
+                                acc = 0;
+                                do {
+                                    ++cs;
+                                } while (row >= mi.seg_hi[cs]);
+                                next = mi.seg_hi[cs];
+                            }
+                            acc = absmax_bf16x2(acc, v[k]);
+                        }
+                    }
                 }
             }
-            named_barrier(1, NC);
+            if (rows_here > 0)
+                flush(cs, acc);
+            named_barrier(2, NA);
+            for (int i = ta; i < min(nseg, ASEG) * W; i += NA) {
+                const uint32_t v = atab[i];
+                const int64_t l = (int64_t)r * W + (i % W);
+                if (v && l < L)
+                    atomicMax(p.amax + (int64_t)mi.seg_g[i / W] * L + l, v);
+            }
+            named_barrier(2, NA);
+            if (ta == 0 && !(p.skip_arrival && blockIdx.x == 0))
+                red_release_gpu_add(p.counters + r, 1); // bar.sync + release order the warps' atomics
+        }
+        return;
+    }
 
-            // cast: a task is 16 positions x this lane's 2 lines
-            const uint32_t *slab = reinterpret_cast<const uint32_t *>(in_s + (size_t)s * stage_bytes);
-            const int64_t rows_here = hi - lo; // may be <= 0
-            const int ntask16 = rows_here > 0 ? (int)((rows_here + 15) / 16) : 0;
-            const int64_t l0 = (int64_t)rr * W + 2 * lane;
-            const uint32_t stg_base = smem_u32(stg);
-            const int bsel = (lane >> 2) & 1;
-            // boxes that end at or before end_all use TMA; the one that
-            // straddles end_all is written directly
-            const int full_boxes = (int)((hi - lo) / OBOX);
-            for (int t16 = warp; t16 < ntask16; t16 += CWARPS) {
-                const int i0 = t16 * 16;
-                // group segment of each row: find the segment of row i0
-                int sg = 0;
-                while (sg + 1 < nseg && mi.seg_hi[sg] <= i0)
-                    ++sg;
-                const bool one_seg = mi.seg_hi[sg] >= min((int64_t)i0 + 16, rows_here);
+    // ---------------------------------------------------- cast warps (pass B)
+    const int tb = threadIdx.x;
+    const int lp = tb & 127;       // line pair within the strip: lines 2lp, 2lp+1
+    const int half = tb >> 7;      // slices half, half + 2 of each store box
+    const int bsel = (lp >> 2) & 1;
+    const int full_groups = rows_here / OPOS;
+    const uint64_t out_pol = policy_evict_first();
+    int seq = 0;
+    for (int r = 0; r < R; ++r) {
+        // wait for every CTA's amax of strip r
+        if (tb == 0) {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire_gpu(p.counters + r) < ncta && !*(volatile int *)&mi.abort_flag) {
+                if (globaltimer() - t0 > p.wait_ns) {
+                    set_status(MXQ_ERR_TIMEOUT);
+                    mi.abort_flag = 1;
+                    break;
+                }
+            }
+        }
+        named_barrier(1, NB);
+        if (*(volatile int *)&mi.abort_flag)
+            break;
+        for (int g = blockIdx.x; g < p.G; g += ncta)
+            for (int li = tb; li < W; li += NB) {
+                const int64_t l = (int64_t)r * W + li;
+                if (l < L)
+                    p.inv[(int64_t)g * L + l] = fp8_inv(fp8_scale(__uint_as_float(__ldcg(p.amax + (int64_t)g * L + l))));
+            }
+        const int64_t lb = (int64_t)r * W + 2 * lp;
+        int cs = 0;
+        int sc_seg = -1; // segment whose scales s0b, s1b hold
+        float s0b = 0.0f, s1b = 0.0f;
+        auto scales = [&](int seg, float &s0, float &s1) {
+            const unsigned *src = p.amax + (int64_t)mi.seg_g[seg] * L + lb;
+            s0 = lb < L ? fp8_scale(__uint_as_float(__ldcg(src))) : 0.0f;
+            s1 = lb + 1 < L ? fp8_scale(__uint_as_float(__ldcg(src + 1))) : 0.0f;
+        };
+        for (int og = 0; og < ngroups; ++og) {
+            const int nb = min(GROUP_BOXES, nbox - og * GROUP_BOXES);
+            bool ok = true;
+            for (int j = 0; j < nb; ++j)
+                ok &= mbar_wait(&full_b[(seq + j) % SB], (uint32_t)((seq + j) / SB) & 1u, p.wait_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                mi.abort_flag = 1;
+            const int ob = og & 1;
+            if (tb == 0)
+                bulk_wait_read<1>(); // staging buffer ob was read by the store of group og-2
+            named_barrier(1, NB);
+            const uint32_t stg_addr = smem_u32(stg + ob * OBOX_BYTES);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int sl = half + 2 * t; // 16-row slice of the store box
+                const int i0 = og * OPOS + sl * BOXR; // first row (relative to lo)
+                if (sl >= nb || i0 >= rows_here)
+                    continue;
+                const uint32_t *box = reinterpret_cast<const uint32_t *>(ring_b + ((seq + sl) % SB) * BOX_BYTES) + lp;
+                uint32_t x[BOXR];
+#pragma unroll
+                for (int k = 0; k < BOXR; ++k)
+                    x[k] = box[k * (W / 2)];
+                while (cs + 1 < nseg && mi.seg_hi[cs] <= i0)
+                    ++cs;
                 uint32_t o0[4], o1[4];
-                if (one_seg) {
-                    const float s0 = stab[sg * W + 2 * lane], s1 = stab[sg * W + 2 * lane + 1];
+                if (mi.seg_hi[cs] >= min(i0 + BOXR, rows_here)) {
+                    if (sc_seg != cs) {
+                        scales(cs, s0b, s1b);
+                        sc_seg = cs;
+                    }
+                    const float s0 = s0b, s1 = s1b;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint32_t x0 = slab[(i0 + 4 * k + 0) * 32 + lane];
-                        const uint32_t x1 = slab[(i0 + 4 * k + 1) * 32 + lane];
-                        const uint32_t x2 = slab[(i0 + 4 * k + 2) * 32 + lane];
-                        const uint32_t x3 = slab[(i0 + 4 * k + 3) * 32 + lane];
+                        const uint32_t x0 = x[4 * k + 0], x1 = x[4 * k + 1];
+                        const uint32_t x2 = x[4 * k + 2], x3 = x[4 * k + 3];
                         o0[k] = e4m3x2(__fmul_rn(bf16_lo(x0), s0), __fmul_rn(bf16_lo(x1), s0)) |
                                 (e4m3x2(__fmul_rn(bf16_lo(x2), s0), __fmul_rn(bf16_lo(x3), s0)) << 16);
                         o1[k] = e4m3x2(__fmul_rn(bf16_hi(x0), s1), __fmul_rn(bf16_hi(x1), s1)) |
                                 (e4m3x2(__fmul_rn(bf16_hi(x2), s1), __fmul_rn(bf16_hi(x3), s1)) << 16);
                     }
                 } else {
+                    // the slice crosses group boundaries: per-row scale
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         uint32_t a0 = 0, a1 = 0;
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const int i = i0 + 4 * k + j;
-                            int sj = sg;
-                            while (sj + 1 < nseg && mi.seg_hi[sj] <= i)
+                            const int row = i0 + 4 * k + j;
+                            int sj = cs;
+                            while (sj + 1 < nseg && mi.seg_hi[sj] <= row)
                                 ++sj;
-                            const float s0 = stab[sj * W + 2 * lane], s1 = stab[sj * W + 2 * lane + 1];
-                            const uint32_t x = slab[i * 32 + lane];
-                            a0 |= e4m3x2(__fmul_rn(bf16_lo(x), s0), 0.0f) << (8 * j);
-                            a1 |= e4m3x2(__fmul_rn(bf16_hi(x), s1), 0.0f) << (8 * j);
+                            float s0, s1;
+                            scales(sj, s0, s1);
+                            const uint32_t xv = x[4 * k + j];
+                            a0 |= e4m3x2(__fmul_rn(bf16_lo(xv), s0), 0.0f) << (8 * j);
+                            a1 |= e4m3x2(__fmul_rn(bf16_hi(xv), s1), 0.0f) << (8 * j);
                         }
                         o0[k] = a0;
                         o1[k] = a1;
                     }
                 }
-                const int box = i0 / OBOX;
-                if (box < full_boxes) {
-                    // staging box: 64 lines x 64 bytes, 16-byte chunk c of
-                    // line l stored at chunk c ^ ((l >> 1) & 3) (64B swizzle)
-                    const uint32_t bbase = stg_base + box * (OBOX * W);
-                    const int c = (i0 % OBOX) / 16;
+                if (og < full_groups) {
+                    // staging: 256 lines x 64 bytes; 16-byte chunk c of line l
+                    // at chunk c ^ ((l >> 1) & 3) (64B swizzle). Alternating
+                    // the lane's two lines keeps each 16-byte store
+                    // instruction on 8 distinct bank groups.
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const int b = bsel ^ j;
-                        const int line = 2 * lane + b;
-                        const int pc = c ^ ((line >> 1) & 3);
-                        const uint4 val = b ? make_uint4(o1[0], o1[1], o1[2], o1[3])
-                                            : make_uint4(o0[0], o0[1], o0[2], o0[3]);
-                        sts_v4(bbase + line * OBOX + pc * 16, val);
+                        const int bb = bsel ^ j;
+                        const int line = 2 * lp + bb;
+                        const int pc = sl ^ (lp & 3);
+                        const uint4 val = bb ? make_uint4(o1[0], o1[1], o1[2], o1[3])
+                                             : make_uint4(o0[0], o0[1], o0[2], o0[3]);
+                        sts_v4(stg_addr + line * OPOS + pc * 16, val);
                     }
                 } else {
-                    // the box holding end_all: direct byte stores of rows below hi
+                    // the store box that holds end_all: direct byte stores
 #pragma unroll
-                    for (int b = 0; b < 2; ++b) {
-                        const int64_t l = l0 + b;
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const int64_t l = lb + bb;
                         if (l >= L)
                             continue;
                         uint8_t *dst = p.out + l * p.P + lo + i0;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const uint32_t word = b ? o1[j >> 2] : o0[j >> 2];
-                            if (lo + i0 + j < hi)
+                            const uint32_t word = bb ? o1[j >> 2] : o0[j >> 2];
+                            if (i0 + j < rows_here)
                                 dst[j] = (uint8_t)(word >> (8 * (j & 3)));
                         }
                     }
                 }
             }
-            fence_proxy_async_smem();
-            named_barrier(1, NC);
-            // release the input stage and store the full boxes
+            __syncwarp();
             if (lane == 0)
-                mbar_arrive(&empty[s]);
-            if (ctid == 0) {
-                for (int bx = 0; bx < full_boxes; ++bx)
-                    tma_store_2d(&tm_out, stg + bx * (OBOX * W), (int)(lo + bx * OBOX), rr * W);
+                for (int j = 0; j < nb; ++j)
+                    mbar_arrive(&empty_b[(seq + j) % SB]);
+            seq += nb;
+            fence_proxy_async_smem();
+            named_barrier(1, NB);
+            if (tb == 0 && og < full_groups) {
+                tma_store_2d_hint(&tm_out, stg + ob * OBOX_BYTES, (int)(lo + og * OPOS), r * W, out_pol);
                 bulk_commit();
             }
         }
+        named_barrier(1, NB);
+        if (tb == 0)
+            *(volatile int *)&mi.b_done = r + 1;
     }
-    if (threadIdx.x == 0)
+    if (tb == 0)
         bulk_wait<0>();
 }
 

@@ -128,7 +128,7 @@ int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_
 // ------------------------------------------------------------ jagged plan
 struct JaggedPlan {
     bool fused = false;
-    int chunk = 0, stages = 0, ncta = 0, rounds = 0, nseg_cap = 0;
+    int chunk = 0, ncta = 0, rounds = 0;
     size_t smem = 0;
     size_t ws_amax = 0, ws_total = 0;
 };
@@ -163,29 +163,19 @@ int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_
     if (!di->coop)
         return MXQ_OK;
     const int64_t per = (P + di->sms - 1) / di->sms;
-    const int chunk = (int)((per + jag::OBOX - 1) / jag::OBOX * jag::OBOX);
+    const int chunk = (int)((per + jag::OPOS - 1) / jag::OPOS * jag::OPOS);
     const int ncta = (int)((P + chunk - 1) / chunk);
-    const int nseg_cap = G;
-    const int budget = di->smem_optin - (int)sizeof(jag::Misc) - 64 - 1024;
-    int stages = 0;
-    for (int s = 4; s >= 2; --s)
-        if (jag::layout(chunk, s, nseg_cap).total <= budget) {
-            stages = s;
-            break;
-        }
-    if (stages == 0)
+    const size_t smem = jag::SMEM_BYTES;
+    if ((int)smem > di->smem_optin - (int)sizeof(jag::Misc) - 64)
         return MXQ_OK;
-    const size_t smem = (size_t)jag::layout(chunk, stages, nseg_cap).total + 1024;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_jagged_fused, jag::THREADS, smem) != cudaSuccess ||
         per_sm < 1 || ncta > per_sm * di->sms)
         return MXQ_OK;
     pl->fused = true;
     pl->chunk = chunk;
-    pl->stages = stages;
     pl->ncta = ncta;
     pl->rounds = (int)((L + jag::W - 1) / jag::W);
-    pl->nseg_cap = nseg_cap;
     pl->smem = smem;
     pl->ws_amax = round_up((size_t)G * (size_t)L * 4, 256);
     pl->ws_total = fused_workspace(L, G);
@@ -215,13 +205,13 @@ int jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, 
         CUtensorMap tin, tout;
         const uint64_t din[2] = {(uint64_t)L, (uint64_t)P};
         const uint64_t sin[1] = {(uint64_t)s_pos * 2};
-        const uint32_t bin[2] = {jag::W, jag::BOXP};
+        const uint32_t bin[2] = {jag::W, jag::BOXR};
         rc = make_map(&tin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, din, sin, bin, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc != MXQ_OK)
             return rc;
         const uint64_t dout[2] = {(uint64_t)P, (uint64_t)L};
         const uint64_t sout[1] = {(uint64_t)P};
-        const uint32_t bout[2] = {jag::OBOX, jag::W};
+        const uint32_t bout[2] = {jag::OPOS, jag::W};
         rc = make_map(&tout, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_64B);
         if (rc != MXQ_OK)
             return rc;
@@ -232,9 +222,7 @@ int jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, 
         p.P = P;
         p.G = G;
         p.chunk = pl.chunk;
-        p.stages = pl.stages;
         p.rounds = pl.rounds;
-        p.nseg_cap = pl.nseg_cap;
         p.offs = offs;
         p.out = static_cast<uint8_t *>(out);
         p.inv = inv;
