@@ -216,27 +216,24 @@ MXQ_DEV uint32_t e8m0_floor(float amax)
     return (uint32_t)(k + 127);
 }
 
-// E8M0 scale byte, rceil mode: ceil(log2(amax / 448)) from the exponent and
-// mantissa fields of the fp32 quotient. For bf16 amax the fp32 rounding of
-// the quotient never crosses a power of two, so this equals the exact value.
+// E8M0 scale byte, rceil mode: ceil(log2(amax / 448)), clamped to
+// [-127, 127], biased by 127. For a normal amax = M * 2^E with M in [1, 2),
+// amax / 448 = (M / 1.75) * 2^(E - 8) and log2(M / 1.75) lies in (-1, 0] for
+// M <= 1.75 and in (0, 1) above, so the exponent is E - 8 plus one exactly
+// when the mantissa exceeds 1.75 (fraction bits > 0x600000). Zero and
+// subnormal amax lie below 448 * 2^-127 and give the smallest scale.
 MXQ_DEV uint32_t e8m0_rceil(float amax)
 {
-    const uint32_t b = __float_as_uint(__fdiv_rn(amax, 448.0f));
-    const int e = (int)(b >> 23);
-    const uint32_t m = b & 0x7FFFFFu;
-    int k;
+    const uint32_t bits = __float_as_uint(amax); // amax >= 0
+    const int e = (int)(bits >> 23);
     if (e == 0)
-        k = m > 0x400000u ? -126 : -127; // subnormal quotient: (2^-127, 2^-126) -> -126
-    else
-        k = e - 127 + (m != 0u ? 1 : 0);
+        return 0u;
+    int k = e - 127 - 8 + ((bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
     k = k < -127 ? -127 : (k > 127 ? 127 : k);
     return (uint32_t)(k + 127);
 }
 
-template <int MODE> MXQ_DEV uint32_t e8m0(float amax)
-{
-    return MODE == MXQ_E8M0_RCEIL ? e8m0_rceil(amax) : e8m0_floor(amax);
-}
+MXQ_DEV uint32_t e8m0_mode(float amax, int mode) { return mode == MXQ_E8M0_RCEIL ? e8m0_rceil(amax) : e8m0_floor(amax); }
 
 // 2^(127 - byte) as an exact fp32 power of two (byte <= 253).
 MXQ_DEV float mx_factor(uint32_t byte) { return __uint_as_float((254u - byte) << 23); }

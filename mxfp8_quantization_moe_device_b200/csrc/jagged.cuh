@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(jag::THREADS, 1)
     const int nseg = mi.nseg;
     const int R = p.rounds;
     const int64_t L = p.L;
-    constexpr int PRODUCER_A = (NB + NA) / 32, PRODUCER_B = PRODUCER_A + 1;
+    constexpr int PRODUCER_A = (NB + NA) / 32;
 
     if (warp >= PRODUCER_A) {
         // ------------------------------------------------ producer warps

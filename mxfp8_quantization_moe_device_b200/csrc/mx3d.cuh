@@ -45,10 +45,9 @@ struct __align__(1024) Smem {
 
 constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024; // + manual 1 KB alignment
 
-template <int MODE>
 __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
     k_mx_3d_colwise(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
-                    uint8_t *__restrict__ scales, int E, int N, int K, int tiles_n, int tiles_k,
+                    uint8_t *__restrict__ scales, int E, int N, int K, int tiles_n, int tiles_k, int mode,
                     uint64_t wait_ns)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -123,7 +122,8 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
         if (lane == 0)
             mbar_arrive(&sm.empty[s]);
 
-        const uint32_t b0 = e8m0<MODE>(bf16_lo(acc)), b1 = e8m0<MODE>(bf16_hi(acc));
+        const float a0 = bf16_lo(acc), a1 = bf16_hi(acc);
+        const uint32_t b0 = e8m0_mode(a0, mode), b1 = e8m0_mode(a1, mode);
         const float f0 = mx_factor(b0), f1 = mx_factor(b1);
         uint32_t q0[8], q1[8]; // column 2*lane and 2*lane+1, 32 bytes each
 #pragma unroll

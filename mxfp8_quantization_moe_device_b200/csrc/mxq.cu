@@ -87,9 +87,7 @@ int device_info(const DevInfo **out)
             cudaDeviceGetAttribute(&di.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess ||
             cudaDeviceGetAttribute(&di.coop, cudaDevAttrCooperativeLaunch, d) != cudaSuccess)
             return MXQ_ERR_CUDA;
-        if (cudaFuncSetAttribute(mx3d::k_mx_3d_colwise<MXQ_E8M0_FLOOR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)mx3d::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(mx3d::k_mx_3d_colwise<MXQ_E8M0_RCEIL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(mx3d::k_mx_3d_colwise, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mx3d::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(k_jagged_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  di.smem_optin - (int)sizeof(jag::Misc) - 64) != cudaSuccess)
@@ -101,6 +99,15 @@ int device_info(const DevInfo **out)
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// CTAs of `kernel` that fit on the GPU at once (one full wave)
+template <typename K> int64_t resident_ctas(K kernel, int threads, const DevInfo *di)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return (int64_t)per_sm * di->sms;
+}
 
 template <typename... K, typename... A>
 int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool coop, A &&...args)
@@ -297,7 +304,7 @@ int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols, int32_t bloc
     if (block_rows == 1) {
         const int64_t nblk = rows * (cols / 128);
         const int64_t per_cta = (RB_THREADS / 32) * 2 * RB_UNROLL;
-        const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, (int64_t)di->sms * 8);
+        const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, resident_ctas(k_fp8_1x128, RB_THREADS, di));
         return launch(k_fp8_1x128, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
                       static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), inv_scales);
     }
@@ -342,12 +349,8 @@ int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t
     const int tiles_n = (int)((N + mx3d::TN - 1) / mx3d::TN), tiles_k = (int)((K + mx3d::TK - 1) / mx3d::TK);
     const int64_t total = E * tiles_n * tiles_k;
     const int64_t grid = std::min<int64_t>(total, (int64_t)di->sms * mx3d::CTAS_PER_SM);
-    if (mode == MXQ_E8M0_FLOOR)
-        return launch(mx3d::k_mx_3d_colwise<MXQ_E8M0_FLOOR>, dim3((unsigned)grid), dim3(mx3d::THREADS),
-                      mx3d::SMEM_BYTES, stream, false, tin, tout, scales, (int)E, (int)N, (int)K, tiles_n, tiles_k,
-                      wait_ns());
-    return launch(mx3d::k_mx_3d_colwise<MXQ_E8M0_RCEIL>, dim3((unsigned)grid), dim3(mx3d::THREADS), mx3d::SMEM_BYTES,
-                  stream, false, tin, tout, scales, (int)E, (int)N, (int)K, tiles_n, tiles_k, wait_ns());
+    return launch(mx3d::k_mx_3d_colwise, dim3((unsigned)grid), dim3(mx3d::THREADS), mx3d::SMEM_BYTES, stream, false,
+                  tin, tout, scales, (int)E, (int)N, (int)K, tiles_n, tiles_k, (int)mode, wait_ns());
 }
 
 int mx_quant_rowwise(const void *in, int64_t rows, int64_t cols, int32_t mode, void *out, uint8_t *scales,
@@ -369,13 +372,10 @@ int mx_quant_rowwise(const void *in, int64_t rows, int64_t cols, int32_t mode, v
         return rc;
     const int64_t nblk = rows * (cols / 32);
     const int64_t per_cta = (RB_THREADS / 32) * 8 * RB_UNROLL;
-    const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, (int64_t)di->sms * 8);
+    const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, resident_ctas(k_mx_1x32, RB_THREADS, di));
     const int wa = aligned(scales, 4) ? 1 : 0;
-    if (mode == MXQ_E8M0_FLOOR)
-        return launch(k_mx_1x32<MXQ_E8M0_FLOOR>, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
-                      static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), scales, wa);
-    return launch(k_mx_1x32<MXQ_E8M0_RCEIL>, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
-                  static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), scales, wa);
+    return launch(k_mx_1x32, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false, static_cast<const uint4 *>(in),
+                  nblk, static_cast<uint2 *>(out), scales, wa, (int)mode);
 }
 
 int64_t mx_blocked_grouped_rows_bound(int64_t rows, int32_t num_groups)
@@ -403,10 +403,15 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
     if ((cols4 == 0 || out_rows_capacity == 0) && !out_group_row_starts)
         return MXQ_OK;
     const int64_t tiles_c = cols4 / 4;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
     const int64_t gx = std::max<int64_t>((tiles_c + blk::TILES - 1) / blk::TILES, 1);
-    const int64_t gy = std::max<int64_t>(out_rows_capacity / 128, 1);
-    if (gy > 65535)
-        return MXQ_ERR_UNSUPPORTED;
+    // enough CTAs to fill the GPU; each walks tile rows with stride gy
+    const int64_t tile_rows = std::max<int64_t>(out_rows_capacity / 128, 1);
+    const int64_t want = std::max<int64_t>((int64_t)di->sms * 4 / gx, 1);
+    const int64_t gy = std::min<int64_t>(tile_rows, std::min<int64_t>(want, 65535));
     const int words_ok = (aligned(scales, 4) && cols % 4 == 0) ? 1 : 0;
     return launch(k_blocked_grouped, dim3((unsigned)gx, (unsigned)gy), dim3(blk::THREADS), 0, stream, false, scales,
                   rows, cols, offs, (int)num_groups, out, out_group_row_starts, words_ok,

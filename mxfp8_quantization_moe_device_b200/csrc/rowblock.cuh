@@ -110,10 +110,9 @@ __global__ void __launch_bounds__(256) k_fp8_128x128(const uint4 *__restrict__ i
 // gives the E8M0 byte; lanes 0 and 16 gather four bytes each by shuffle and
 // store them as one word.
 // ---------------------------------------------------------------------------
-template <int MODE>
 __global__ void __launch_bounds__(RB_THREADS) k_mx_1x32(const uint4 *__restrict__ in, int64_t nblk,
                                                        uint2 *__restrict__ out, uint8_t *__restrict__ scales,
-                                                       int scales_word_aligned)
+                                                       int scales_word_aligned, int mode)
 {
     const int lane = threadIdx.x & 31;
     const int q = lane >> 2, l4 = lane & 3;
@@ -135,7 +134,7 @@ __global__ void __launch_bounds__(RB_THREADS) k_mx_1x32(const uint4 *__restrict_
             float amax = absmax_of_pair(acc);
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            const uint32_t byte = e8m0<MODE>(amax);
+            const uint32_t byte = e8m0_mode(amax, mode);
             const float f = mx_factor(byte);
             // gather the four scale bytes of blocks (lane & 16)/4 .. +3
             const int src = lane & 16;
