@@ -448,6 +448,25 @@ def run_e2e(wl, steps):
     return ms, bi, bo
 
 
+# ----------------------------------------------------------------- ranks
+
+def max_over_ranks(x, device, world):
+    """Max of a per-rank float over all ranks (the timing rule: the slowest
+    replica sets the step time). Every rank must call it."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(step_bytes, steps, total_ms_max, world):
+    """Whole-job GB/s: every replica moves step_bytes per step."""
+    return world * step_bytes * steps / (total_ms_max * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------- main
 
 def main():
@@ -491,12 +510,9 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
     ms_per_step = total_ms / args.steps
-    value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    value = aggregate_value(step_bytes, args.steps, total_ms, world)
 
     per_op = {}
     for (name, _, nbytes), ts in zip(wl.ops, per):
@@ -537,10 +553,7 @@ def main():
                                "sample": SAMPLE_DESC, "seconds": round(spent, 2), "per_op_GB/s": per_o}
     if not args.no_e2e:
         ms, bi, bo = run_e2e(wl, max(1, args.e2e_steps))
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev, world)
         out["e2e"] = {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                       "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 3),
                       "steps": max(1, args.e2e_steps)}
