@@ -119,7 +119,9 @@ int fp8_quant_jagged_colwise(const void *in, int64_t rows, int64_t cols,
 
 /* Workspace size for the jagged ops with these arguments (rowwise: pass the
  * rowwise shape and strides; colwise: the colwise ones, with is_colwise = 1).
- * Returns 0 when the call needs none. */
+ * Returns 0 when the call needs none. Depends only on the layout, so it may
+ * be larger than a particular call uses (small problems run a kernel that
+ * needs no workspace). */
 size_t fp8_quant_jagged_workspace_bytes(int64_t rows, int64_t cols,
                                         int64_t stride_row, int64_t stride_col,
                                         int32_t num_groups, int32_t is_colwise);

@@ -50,6 +50,21 @@ MXQ_DEV void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Release a TMA ring slot this warp has read with ordinary loads: every lane
+// orders its reads (generic proxy) before the next fill of the slot (a TMA
+// write, async proxy) with a proxy fence, issued once `dep` - a value
+// computed from every word the lane loaded - is available, so no load is
+// still in flight; then lane 0 arrives on the slot's empty barrier. Without
+// the fence the refill can overwrite words the loads have not read.
+MXQ_DEV void release_slot_after(uint64_t *empty, uint32_t dep)
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::"r"(dep) : "memory");
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(empty)) : "memory");
+    __syncwarp();
+}
+
 MXQ_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;

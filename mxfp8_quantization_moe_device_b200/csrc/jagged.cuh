@@ -68,8 +68,13 @@ MXQ_DEV bool offsets_ok(const int32_t *__restrict__ offs, int G, int64_t extent)
 }
 
 // ---------------------------------------------------------------------------
-// Generic path: any strides. One warp per (line, group).
+// Generic path: any strides. One warp per (line, group). A group of up to
+// 32 * GB positions is read once, all loads issued together, and kept in
+// registers for the cast; longer groups take two batched passes. Latency,
+// not bandwidth, bounds the small problems this path serves.
 // ---------------------------------------------------------------------------
+constexpr int GB = 8; // positions per lane per batch
+
 __global__ void __launch_bounds__(256) k_jagged_generic(const uint16_t *__restrict__ in, int64_t L, int64_t P,
                                                         int64_t s_line, int64_t s_pos,
                                                         const int32_t *__restrict__ offs, int G,
@@ -86,18 +91,48 @@ __global__ void __launch_bounds__(256) k_jagged_generic(const uint16_t *__restri
         const int g = (int)(task - l * G);
         const int64_t p0 = g ? offs[g - 1] : 0, p1 = offs[g];
         const uint16_t *src = in + l * s_line;
+        uint8_t *dst = out + l * P;
+        float v[GB];
         float amax = 0.0f;
-        for (int64_t p = p0 + lane; p < p1; p += 32)
-            amax = fmaxf(amax, fabsf(bf16_lo(src[p * s_pos])));
+        const bool one_batch = p1 - p0 <= 32 * GB;
+        for (int64_t b0 = p0; b0 < p1; b0 += 32 * GB) {
+#pragma unroll
+            for (int i = 0; i < GB; ++i) {
+                const int64_t p = b0 + lane + 32 * i;
+                v[i] = p < p1 ? bf16_lo(__ldg(src + p * s_pos)) : 0.0f;
+            }
+#pragma unroll
+            for (int i = 0; i < GB; ++i)
+                amax = fmaxf(amax, fabsf(v[i]));
+        }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1)
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float s = fp8_scale(amax);
         if (lane == 0)
             inv[(int64_t)g * L + l] = fp8_inv(s);
-        uint8_t *dst = out + l * P;
-        for (int64_t p = p0 + lane; p < p1; p += 32)
-            dst[p] = (uint8_t)e4m3x2(__fmul_rn(bf16_lo(src[p * s_pos]), s), 0.0f);
+        if (one_batch) {
+#pragma unroll
+            for (int i = 0; i < GB; ++i) {
+                const int64_t p = p0 + lane + 32 * i;
+                if (p < p1)
+                    dst[p] = (uint8_t)e4m3x2(__fmul_rn(v[i], s), 0.0f);
+            }
+        } else {
+            for (int64_t b0 = p0; b0 < p1; b0 += 32 * GB) {
+#pragma unroll
+                for (int i = 0; i < GB; ++i) {
+                    const int64_t p = b0 + lane + 32 * i;
+                    v[i] = p < p1 ? bf16_lo(__ldg(src + p * s_pos)) : 0.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < GB; ++i) {
+                    const int64_t p = b0 + lane + 32 * i;
+                    if (p < p1)
+                        dst[p] = (uint8_t)e4m3x2(__fmul_rn(v[i], s), 0.0f);
+                }
+            }
+        }
     }
 }
 
@@ -356,9 +391,12 @@ __global__ void __launch_bounds__(jag::THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < BOXR; ++k)
                     v[k] = bp[k * (W / 2)];
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&empty_a[s]);
+                // release the slot once every word has landed in a register
+                uint32_t dep = 0;
+#pragma unroll
+                for (int k = 0; k < BOXR; ++k)
+                    dep ^= v[k];
+                release_slot_after(&empty_a[s], dep);
                 const int row0 = b * BOXR;
                 const int rlast = row0 + BOXR - 1;
                 if (rlast < next && rlast < rows_here) {
@@ -395,9 +433,13 @@ __global__ void __launch_bounds__(jag::THREADS, 1)
                 if (v && l < L)
                     atomicMax(p.amax + (int64_t)mi.seg_g[i / W] * L + l, v);
             }
+            // each thread's global atomics (here and in flush) must be
+            // performed at GPU scope before the arrival: bar.sync orders
+            // memory only within the CTA
+            __threadfence();
             named_barrier(2, NA);
             if (ta == 0 && !(p.skip_arrival && blockIdx.x == 0))
-                red_release_gpu_add(p.counters + r, 1); // bar.sync + release order the warps' atomics
+                red_release_gpu_add(p.counters + r, 1);
         }
         return;
     }
@@ -534,12 +576,14 @@ __global__ void __launch_bounds__(jag::THREADS, 1)
                     }
                 }
             }
+            // the ring reads above (generic proxy) and the staging writes are
+            // ordered before the boxes' next TMA fill and the TMA store
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
                 for (int j = 0; j < nb; ++j)
                     mbar_arrive(&empty_b[(seq + j) % SB]);
             seq += nb;
-            fence_proxy_async_smem();
             named_barrier(1, NB);
             if (tb == 0 && og < full_groups) {
                 tma_store_2d_hint(&tm_out, stg + ob * OBOX_BYTES, (int)(lo + og * OPOS), r * W, out_pol);

@@ -118,9 +118,9 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
             v[i] = tile[(w * 32 + i) * (TK / 2) + lane];
             acc = absmax_bf16x2(acc, v[i]);
         }
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.empty[s]);
+        // release the input stage once every loaded word has been consumed
+        // (acc depends on all 32 of them)
+        release_slot_after(&sm.empty[s], acc);
 
         const float a0 = bf16_lo(acc), a1 = bf16_hi(acc);
         const uint32_t b0 = e8m0_mode(a0, mode), b1 = e8m0_mode(a1, mode);

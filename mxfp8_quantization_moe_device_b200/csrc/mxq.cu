@@ -70,6 +70,9 @@ struct DevInfo {
     int sms = 0;
     int smem_optin = 0;
     int coop = 0;
+    int jag_per_sm = 0;   // resident CTAs of the single-pass jagged kernel
+    int rb_per_sm = 0;    // resident CTAs of the 1x128 kernel
+    int mx32_per_sm = 0;  // resident CTAs of the 1x32 kernel
 };
 
 DevInfo g_dev[128];
@@ -92,6 +95,11 @@ int device_info(const DevInfo **out)
             cudaFuncSetAttribute(k_jagged_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  di.smem_optin - (int)sizeof(jag::Misc) - 64) != cudaSuccess)
             return MXQ_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.jag_per_sm, k_jagged_fused, jag::THREADS,
+                                                          jag::SMEM_BYTES) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.rb_per_sm, k_fp8_1x128, RB_THREADS, 0) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mx32_per_sm, k_mx_1x32, RB_THREADS, 0) != cudaSuccess)
+            return MXQ_ERR_CUDA;
         di.ready = true;
     }
     *out = &di;
@@ -100,14 +108,6 @@ int device_info(const DevInfo **out)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// CTAs of `kernel` that fit on the GPU at once (one full wave)
-template <typename K> int64_t resident_ctas(K kernel, int threads, const DevInfo *di)
-{
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    return (int64_t)per_sm * di->sms;
-}
 
 template <typename... K, typename... A>
 int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool coop, A &&...args)
@@ -163,6 +163,10 @@ int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_
     const int force = g_force_path.load();
     if (force == 2 || !fused_layout_ok(in, L, P, s_line, s_pos, G, out))
         return MXQ_OK;
+    // small problems are launch- and latency-bound: the generic kernel (no
+    // workspace clear, no cooperative launch, no strip barriers) is faster
+    if (force == 0 && L * P <= (int64_t(1) << 21))
+        return MXQ_OK;
     const DevInfo *di = nullptr;
     int rc = device_info(&di);
     if (rc != MXQ_OK)
@@ -175,9 +179,7 @@ int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_
     const size_t smem = jag::SMEM_BYTES;
     if ((int)smem > di->smem_optin - (int)sizeof(jag::Misc) - 64)
         return MXQ_OK;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_jagged_fused, jag::THREADS, smem) != cudaSuccess ||
-        per_sm < 1 || ncta > per_sm * di->sms)
+    if (di->jag_per_sm < 1 || ncta > di->jag_per_sm * di->sms)
         return MXQ_OK;
     pl->fused = true;
     pl->chunk = chunk;
@@ -304,7 +306,7 @@ int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols, int32_t bloc
     if (block_rows == 1) {
         const int64_t nblk = rows * (cols / 128);
         const int64_t per_cta = (RB_THREADS / 32) * 2 * RB_UNROLL;
-        const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, resident_ctas(k_fp8_1x128, RB_THREADS, di));
+        const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, (int64_t)std::max(di->rb_per_sm, 1) * di->sms);
         return launch(k_fp8_1x128, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false,
                       static_cast<const uint4 *>(in), nblk, static_cast<uint2 *>(out), inv_scales);
     }
@@ -372,7 +374,7 @@ int mx_quant_rowwise(const void *in, int64_t rows, int64_t cols, int32_t mode, v
         return rc;
     const int64_t nblk = rows * (cols / 32);
     const int64_t per_cta = (RB_THREADS / 32) * 8 * RB_UNROLL;
-    const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, resident_ctas(k_mx_1x32, RB_THREADS, di));
+    const int64_t grid = std::min<int64_t>((nblk + per_cta - 1) / per_cta, (int64_t)std::max(di->mx32_per_sm, 1) * di->sms);
     const int wa = aligned(scales, 4) ? 1 : 0;
     return launch(k_mx_1x32, dim3((unsigned)grid), dim3(RB_THREADS), 0, stream, false, static_cast<const uint4 *>(in),
                   nblk, static_cast<uint2 *>(out), scales, wa, (int)mode);

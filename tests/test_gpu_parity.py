@@ -203,6 +203,29 @@ def test_jagged_full_size_backward_operands():
             assert _dequant_error_ok(src[a:b].t(), q[:, a:b], inv[g][:, None]), g
 
 
+@pytest.mark.slow
+def test_jagged_full_size_scales_every_unit_repeated():
+    """Every (group, column) inverse scale of the full-size colwise op equals
+    the fp32 reciprocal of 448 / max(amax, 1e-12) of its unit, over several
+    calls: the single-pass kernel's cross-CTA amax reduction and its TMA ring
+    reuse must never race. amax here is a max over bf16 values (exact); the
+    scale arithmetic is cross-checked against the oracle on a sample."""
+    _, inp, offs = synth.jagged_bwd(device=DEV)
+    o = offs.tolist()
+    starts = [0] + o[:-1]
+    amax = torch.stack([inp[a:b].float().abs().amax(dim=0) if b > a else torch.zeros(4096, device=DEV)
+                        for a, b in zip(starts, o)])
+    s = torch.tensor(448.0, device=DEV) / torch.clamp(amax, min=float(np.float32(1e-12)))
+    want = (1.0 / s).view(torch.int32)  # fp32 IEEE division on the GPU, as R1 states
+    for probe in [(0, 0), (3, 100), (15, 4095)]:
+        g, c = probe
+        assert f32bits(want.view(torch.float32)[g, c].item()) == f32bits(oracle.fp8_inv_scale(float(amax[g, c])))
+    for _ in range(4):
+        q, inv = mxq.fp8_quant_jagged_colwise(inp, offs.to(DEV))
+        assert status_ok()
+        assert torch.equal(inv.view(torch.int32), want)
+
+
 # ============================================================ blockwise
 
 @pytest.mark.parametrize("rows,cols", [(1, 128), (37, 384), (256, 512), (1000, 1280)])
