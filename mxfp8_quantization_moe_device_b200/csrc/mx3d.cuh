@@ -9,7 +9,7 @@
 //     stores (N, K, E), so host work is O(1) in E;
 //   * a persistent grid (2 CTAs per SM) walks (expert, n-tile, k-tile) work
 //     items with k fastest, so E = 1 fills the GPU as well as E = 64;
-//   * per CTA: one producer warp drives a 5-stage TMA ring of 128 x 64 bf16
+//   * per CTA: one producer warp drives a 4-stage TMA ring of 128 x 64 bf16
 //     tiles (16 KB); four consumer warps each own one 32-row MX block of a
 //     tile, a lane owning two adjacent columns. Each lane keeps its 32 x 2
 //     values in registers, takes the block amax with packed bf16 max,
@@ -27,7 +27,7 @@ namespace mx3d {
 
 constexpr int TN = 128;              // n rows per tile (four 32-row MX blocks)
 constexpr int TK = 64;               // k columns per tile
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int CWARPS = 4;            // consumer warps (one per MX block)
 constexpr int THREADS = (CWARPS + 1) * 32;
 constexpr int IN_BYTES = TN * TK * 2;  // 16384
