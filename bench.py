@@ -38,8 +38,8 @@ WORKLOAD = "moe_quant_path"
 KERNEL_NAMES = {
     "blockwise_1x128": "k_fp8_1x128",
     "blockwise_128x128": "k_fp8_128x128",
-    "jagged_rowwise": "k_jagged_fused",
-    "jagged_colwise": "k_jagged_fused",
+    "jagged_rowwise": "k_jagged_amax+k_jagged_cast",
+    "jagged_colwise": "k_jagged_amax+k_jagged_cast",
     "mx_3d_colwise": "k_mx_3d_colwise",
     "mx_rowwise": "k_mx_1x32",
     "blocked_grouped": "k_blocked_grouped",

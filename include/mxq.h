@@ -199,7 +199,7 @@ int64_t mx_blocked_grouped_rows_bound(int64_t rows, int32_t num_groups);
  * fp8_quant_jagged_colwise, without the workspace: the scratch is a fixed
  * array of fp8_quant_jagged_colwise_noalloc_max_scratch_bytes() bytes
  * (1 MiB) inside the library, held by every GPU that loads it until exit.
- *   - A problem whose single-pass scratch would exceed that size (see
+ *   - A problem whose workspace would exceed that size (see
  *     fp8_quant_jagged_workspace_bytes with is_colwise = 1) returns
  *     MXQ_ERR_WORKSPACE and launches nothing.
  *   - The first call on a device looks up the array's device address with
@@ -234,12 +234,13 @@ int mxq_version(void);
 /* Test hooks (host-side settings read at launch time):
  *   MXQ_TESTING_WAIT_LIMIT_NS  bound of every device-side wait, nanoseconds
  *                              (default 1e9; 0 restores the default).
- *   MXQ_TESTING_SKIP_ARRIVAL   when 1, one CTA of the single-pass jagged
- *                              kernels skips its arrival on the amax barrier,
- *                              so the others' bounded waits expire and report
+ *   MXQ_TESTING_SKIP_ARRIVAL   when 1, CTA 0 of the jagged cast pass never
+ *                              issues its first TMA load, so the transaction
+ *                              arrival on that ring slot never comes, the
+ *                              bounded waits on it expire and report
  *                              MXQ_ERR_TIMEOUT; 0 turns it off.
- *   MXQ_TESTING_FORCE_PATH     jagged ops: 0 automatic, 1 single-pass
- *                              barrier kernel, 2 generic kernel. */
+ *   MXQ_TESTING_FORCE_PATH     jagged ops: 0 automatic, 1 two-pass TMA
+ *                              kernels (amax, then cast), 2 generic kernel. */
 #define MXQ_TESTING_WAIT_LIMIT_NS 1
 #define MXQ_TESTING_SKIP_ARRIVAL 2
 #define MXQ_TESTING_FORCE_PATH 3

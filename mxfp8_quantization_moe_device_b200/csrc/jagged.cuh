@@ -14,36 +14,21 @@
 // rowwise, a row-major input for colwise) the op reads position-major rows
 // and writes their transpose.
 //
-// Two kernels:
-//   k_jagged_generic  any strides: one warp per (line, group), two passes
-//                     over the group's elements (amax, then cast).
-//   k_jagged_fused    contiguous lines: one cooperative launch that keeps
-//                     the HBM traffic near the algorithmic 2 B read + 1 B
-//                     written per element by reading every strip twice, once
-//                     from HBM and once from L2. Each CTA owns a fixed range of
-//                     positions; the lines are walked in strips of 256 (512
-//                     contiguous bytes per position row, 32 MB per strip at
-//                     65536 positions). Warp roles per CTA:
-//                       - producer A streams strip r of the CTA's rows from HBM
-//                         through a 12-deep TMA ring (evict-last L2 policy);
-//                       - four amax warps reduce the per-(group, line) amax of
-//                         each box (tree max over 16 rows when the box lies in
-//                         one group), merge it in shared memory and then into
-//                         a global table with atomicMax on the fp32 bit
-//                         pattern (exact and order-free for non-negative
-//                         values), and arrive on the strip's counter;
-//                       - producer B re-streams the same rows out of L2 through
-//                         a second ring (evict-first); its data never depends
-//                         on the barrier, so it simply runs ahead;
-//                       - eight cast warps wait until every CTA has arrived for
-//                         the strip, read their groups' final amax from L2,
-//                         cast, and write the transpose through a 64B-swizzled
-//                         staging tile with TMA stores.
-//                     The amax warps start strip r+2 only after the cast of
-//                     strip r is done, so at most two strips are live in L2
-//                     while HBM reads and writes overlap. Skewed or empty
-//                     groups only change how many rows of a range fall in
-//                     each group.
+// Kernels:
+//   k_jagged_generic  any strides, small problems: one warp per (line, group),
+//                     the group read into registers, reduced, then cast.
+//   k_jagged_amax +   contiguous lines, two streaming passes. The amax pass
+//   k_jagged_cast     runs warp workers, each owning 256 lines (16 bytes per
+//                     lane per row) and an equal run of positions, keeping 16
+//                     rows of loads in flight and merging its maxima into a
+//                     global (G, L) fp32 table by atomicMax only at group ends.
+//                     The cast pass has the MX 3-D kernel's structure: a TMA
+//                     ring of 128 x 64 tiles, one consumer warp per 32-row
+//                     block, scales from the finished table (prefetched a tile
+//                     ahead), and the transpose leaving through a
+//                     128B-swizzled staging tile and TMA stores. The input is
+//                     read twice (5 B of HBM traffic per element instead of
+//                     3); in exchange neither kernel synchronizes across CTAs.
 #pragma once
 
 #include "common.cuh"
@@ -136,465 +121,365 @@ __global__ void __launch_bounds__(256) k_jagged_generic(const uint16_t *__restri
     }
 }
 
+
 // ---------------------------------------------------------------------------
-// Single-pass-over-HBM cooperative path (contiguous lines).
+// Two-pass path (contiguous lines): amax pass
 // ---------------------------------------------------------------------------
 namespace jag {
 
-constexpr int W = 256;                    // lines per strip (512 B of bf16 per position)
-constexpr int BWARPS = 8;                 // cast warps (pass B)
-constexpr int AWARPS = 4;                 // amax warps (pass A)
-constexpr int NB = BWARPS * 32;           // cast threads: 0 .. NB-1
-constexpr int NA = AWARPS * 32;           // amax threads: NB .. NB+NA-1
-constexpr int THREADS = NB + NA + 64;     // + two producer warps (HBM ring, L2 ring)
-constexpr int BOXR = 16;                  // positions per TMA load box
-constexpr int BOX_BYTES = W * 2 * BOXR;   // 8 KB
-constexpr int OPOS = 64;                  // positions per TMA store box (64 B rows, 64B swizzle)
-constexpr int OBOX_BYTES = OPOS * W;      // 16 KB
-constexpr int GROUP_BOXES = OPOS / BOXR;  // load boxes per store box
-constexpr int SA = 12;                    // HBM ring (pass A): 96 KB in flight
-constexpr int SB = 8;                     // L2 ring (pass B): two store boxes ahead
-constexpr int ASEG = 8;                   // segments reduced in shared memory (more go to global)
-constexpr int MAX_SEG = 64;               // groups a CTA's range may intersect (host checks G)
+constexpr int MAX_SEG = 64; // groups the two-pass kernels accept (host checks G)
 
-struct Params {
-    int64_t L, P;          // lines, positions
-    int G;
-    int chunk;             // positions per CTA (multiple of OPOS)
-    int rounds;            // strips: ceil(L / W)
-    const int32_t *offs;
-    uint8_t *out;          // out[l * P + p]
-    float *inv;
-    unsigned *amax;        // workspace: G * L fp32 bit patterns, zeroed
-    int *counters;         // workspace: rounds ints, zeroed
-    uint64_t wait_ns;
-    int skip_arrival;      // test hook
-};
+namespace amx {
+constexpr int W = 256;       // lines per chunk: 16 bytes (8 lines) per lane
+constexpr int BR = 16;       // rows per batch of loads in flight per lane
+constexpr int THREADS = 256;
+constexpr int CTAS_PER_SM = 2;
+} // namespace amx
 
-// shared memory carve-up (byte offsets from a 1024-aligned base)
-constexpr int RA_OFF = 0;
-constexpr int RB_OFF = RA_OFF + SA * BOX_BYTES;
-constexpr int STG_OFF = RB_OFF + SB * BOX_BYTES;
-constexpr int ATAB_OFF = STG_OFF + 2 * OBOX_BYTES;
-constexpr int BAR_OFF = ATAB_OFF + ASEG * W * 4;
-constexpr int SMEM_TOTAL = BAR_OFF + 2 * (SA + SB) * 8;
-constexpr size_t SMEM_BYTES = SMEM_TOTAL + 1024; // + manual 1 KB alignment
-
-struct Misc {
-    int nseg;              // non-empty group segments of this CTA's range
-    int abort_flag;
-    int b_done;            // strips whose cast (pass B) this CTA has finished
-    int seg_g[MAX_SEG];    // group of each segment
-    int seg_lo[MAX_SEG];   // segment rows, relative to the range start
-    int seg_hi[MAX_SEG];
-};
-
-MXQ_DEV uint64_t policy_evict_last()
+// first group whose end is > p (p < offs[G-1])
+MXQ_DEV int group_of(const int *soffs, int G, int64_t p)
 {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-MXQ_DEV uint64_t policy_evict_first()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-MXQ_DEV void tma_load_2d_hint(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y, uint64_t pol)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
-}
-
-MXQ_DEV void tma_store_2d_hint(const CUtensorMap *map, const void *src, int x, int y, uint64_t pol)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint"
-                 " [%0, {%2, %3}], [%1], %4;" ::"l"(map),
-                 "r"(smem_u32(src)), "r"(x), "r"(y), "l"(pol)
-                 : "memory");
-}
-
-// max of |a|, |b| over packed bf16 pairs
-MXQ_DEV uint32_t absmax2(uint32_t a, uint32_t b) { return absmax_bf16x2(a & 0x7FFF7FFFu, b); }
-
-// fill `n` boxes of TMA ring (stages S, barriers full/empty) with the boxes
-// `first..first+n-1` of a pass; `seq` counts boxes through the ring
-MXQ_DEV bool ring_fill(uint8_t *ring, uint64_t *full, uint64_t *empty, int S, int &seq, const CUtensorMap *map,
-                       int x, int64_t y0, int n, uint64_t pol, uint64_t wait_ns)
-{
-    for (int b = 0; b < n; ++b, ++seq) {
-        const int s = seq % S;
-        if (seq >= S && !mbar_wait(&empty[s], ((uint32_t)(seq / S) & 1u) ^ 1u, wait_ns))
-            return false;
-        mbar_arrive_expect_tx(&full[s], BOX_BYTES);
-        tma_load_2d_hint(ring + s * BOX_BYTES, map, &full[s], x, (int)(y0 + b * BOXR), pol);
+    int a = 0, b = G - 1;
+    while (a < b) {
+        const int m = (a + b) >> 1;
+        if (soffs[m] > p) b = m; else a = m + 1;
     }
-    return true;
-}
-
-MXQ_DEV void ring_drain(uint64_t *full, int S, int seq, uint64_t wait_ns)
-{
-    for (int j = seq - S; j < seq; ++j)
-        if (j >= 0)
-            mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, wait_ns);
+    return a;
 }
 
 } // namespace jag
 
-__global__ void __launch_bounds__(jag::THREADS, 1)
-    k_jagged_fused(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
-                   const jag::Params p)
+// amax[g * L + l] = max |x| over group g's positions of line l, as fp32 bits
+// (the table must be zero on entry).
+//
+// Workers are warps. Worker (c, j) owns lines [256c, 256c + 256), a lane
+// owning eight adjacent lines (one 16-byte load per row), and the j-th of
+// `wpc` equal runs of positions [0, offs[G-1]). It keeps 16 rows of loads in
+// flight, reduces them with packed bf16 max while the batch lies in one
+// group, and merges its running maxima into the table with atomicMax on the
+// fp32 bit pattern (exact and order-free for non-negative values) only when
+// its run crosses a group end and when it finishes.
+__global__ void __launch_bounds__(jag::amx::THREADS, jag::amx::CTAS_PER_SM)
+    k_jagged_amax(const uint16_t *__restrict__ in, int64_t L, int64_t P, int64_t s_pos,
+                  const int32_t *__restrict__ offs, int G, int wpc, unsigned *__restrict__ amax)
 {
     using namespace jag;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *ring_a = base + RA_OFF;
-    uint8_t *ring_b = base + RB_OFF;
-    uint8_t *stg = base + STG_OFF;
-    uint32_t *atab = reinterpret_cast<uint32_t *>(base + ATAB_OFF); // amax bits of segments < ASEG
-    uint64_t *full_a = reinterpret_cast<uint64_t *>(base + BAR_OFF);
-    uint64_t *empty_a = full_a + SA;
-    uint64_t *full_b = empty_a + SA;
-    uint64_t *empty_b = full_b + SB;
-    __shared__ Misc mi;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ncta = gridDim.x;
-    const int64_t lo = (int64_t)blockIdx.x * p.chunk;
-    // every CTA validates the same offsets, so on bad offsets all return
-    // together and no barrier is left waiting
-    if (!offsets_ok(p.offs, p.G, p.P))
+    using namespace jag::amx;
+    __shared__ int soffs[MAX_SEG];
+    if (!offsets_ok(offs, G, P))
         return;
-    const int64_t end_all = p.offs[p.G - 1];
-    const int64_t hi = min(lo + (int64_t)p.chunk, end_all);
-    const int rows_here = hi > lo ? (int)(hi - lo) : 0;
-    const int nbox = (rows_here + BOXR - 1) / BOXR;
-    const int ngroups = (nbox + GROUP_BOXES - 1) / GROUP_BOXES;
+    for (int g = threadIdx.x; g < G; g += blockDim.x)
+        soffs[g] = offs[g];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t end_all = soffs[G - 1];
+    const int64_t chunks = (L + W - 1) / W;
+    const int64_t wid = ((int64_t)blockIdx.x * THREADS + threadIdx.x) >> 5;
+    if (wid >= chunks * wpc)
+        return;
+    const int64_t c = wid % chunks, j = wid / chunks;
+    const int64_t run = ((end_all + wpc - 1) / wpc + BR - 1) / BR * BR;
+    int64_t r = j * run;
+    const int64_t rend = min(end_all, r + run);
+    if (r >= rend)
+        return;
+    const int64_t line0 = c * W + 8 * lane;
+    const int nvalid = (int)max((int64_t)0, min((int64_t)8, L - line0)); // lines of this lane
+    const uint16_t *src = in + line0;
 
+    int g = group_of(soffs, G, r);
+    int64_t gend = soffs[g];
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};
+    auto flush = [&]() {
+        unsigned *dst = amax + (int64_t)g * L + line0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (2 * q < nvalid && (acc[q] & 0xFFFFu))
+                atomicMax(dst + 2 * q, acc[q] << 16);
+            if (2 * q + 1 < nvalid && (acc[q] >> 16))
+                atomicMax(dst + 2 * q + 1, acc[q] & 0xFFFF0000u);
+            acc[q] = 0u;
+        }
+    };
+    for (; r < rend; r += BR) {
+        uint4 v[BR];
+#pragma unroll
+        for (int k = 0; k < BR; ++k) {
+            const int64_t row = r + k;
+            v[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (row < rend) {
+                const uint16_t *p = src + row * s_pos;
+                if (nvalid == 8) {
+                    v[k] = ld_stream_v4(reinterpret_cast<const uint4 *>(p));
+                } else if (nvalid > 0) {
+                    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+                    for (int i = 0; i < nvalid; ++i)
+                        w4[i >> 1] |= (uint32_t)__ldg(p + i) << (16 * (i & 1));
+                    v[k] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+        }
+        if (min(r + BR, rend) <= gend) {
+            // the whole batch lies in group g (rows past rend read as zero)
+#pragma unroll
+            for (int k = 0; k < BR; ++k) {
+                acc[0] = absmax_bf16x2(acc[0], v[k].x);
+                acc[1] = absmax_bf16x2(acc[1], v[k].y);
+                acc[2] = absmax_bf16x2(acc[2], v[k].z);
+                acc[3] = absmax_bf16x2(acc[3], v[k].w);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < BR; ++k) {
+                const int64_t row = r + k;
+                if (row < rend) {
+                    if (row >= gend) {
+                        flush();
+                        do {
+                            ++g;
+                        } while (row >= soffs[g]);
+                        gend = soffs[g];
+                    }
+                    acc[0] = absmax_bf16x2(acc[0], v[k].x);
+                    acc[1] = absmax_bf16x2(acc[1], v[k].y);
+                    acc[2] = absmax_bf16x2(acc[2], v[k].z);
+                    acc[3] = absmax_bf16x2(acc[3], v[k].w);
+                }
+            }
+        }
+    }
+    flush();
+}
+
+// ---------------------------------------------------------------------------
+// Two-pass path (contiguous lines): cast pass, the MX 3-D tile structure
+// ---------------------------------------------------------------------------
+namespace jag {
+namespace cst {
+constexpr int TP = 128;                 // positions per tile (four 32-row blocks)
+constexpr int TL = 64;                  // lines per tile
+constexpr int STAGES = 4;
+constexpr int CWARPS = 4;               // one 32-row block each
+constexpr int THREADS = (CWARPS + 1) * 32;
+constexpr int IN_BYTES = TP * TL * 2;   // 16 KB
+constexpr int OUT_BYTES = TP * TL;      // 8 KB
+constexpr int CTAS_PER_SM = 2;
+
+struct __align__(1024) Smem {
+    uint8_t in[STAGES][IN_BYTES];
+    uint8_t out[2][OUT_BYTES];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    int offs[MAX_SEG];
+    int abort_flag;
+};
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+} // namespace cst
+} // namespace jag
+
+// out[l * P + p] = e4m3(x(l, p) * s(group(p), l)), s = 448 / max(amax, 1e-12)
+// from the finished amax table; inv[g * L + l] = 1 / s (written by the first
+// tiles_l CTAs). Rows past offs[G-1] are not written. A consumer warp owns a
+// 32-row block of each tile; the group and the two amax words of its next
+// tile are loaded while it works on the current one, so the table's L2
+// latency stays off the per-tile path. `drop_load`: test hook, CTA 0 never
+// issues its first tile, so the bounded waits on it expire.
+__global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
+    k_jagged_cast(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out, int64_t L,
+                  int64_t P, const int32_t *__restrict__ offs, int G, const unsigned *__restrict__ amax,
+                  uint8_t *__restrict__ out, float *__restrict__ inv, uint64_t wait_ns, int drop_load)
+{
+    using namespace jag;
+    using namespace jag::cst;
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (!offsets_ok(offs, G, P))
+        return;
+    const int64_t end_all = offs[G - 1];
+    const int64_t tiles_p = (end_all + TP - 1) / TP, tiles_l = (L + TL - 1) / TL;
+    const int64_t total = tiles_p * tiles_l;
     if (threadIdx.x == 0) {
-        // non-empty groups intersecting [lo, hi), clipped: they tile [0, rows_here)
-        int n = 0;
-        if (rows_here > 0) {
-            int a = 0, b = p.G - 1; // first group with end > lo
-            while (a < b) {
-                const int m = (a + b) >> 1;
-                if (p.offs[m] > lo) b = m; else a = m + 1;
-            }
-            for (int g = a; g < p.G && n < MAX_SEG; ++g) {
-                const int64_t gs = g ? p.offs[g - 1] : 0, ge = p.offs[g];
-                if (gs >= hi)
-                    break;
-                if (ge == gs)
-                    continue;
-                mi.seg_g[n] = g;
-                mi.seg_lo[n] = (int)(max(gs, lo) - lo);
-                mi.seg_hi[n] = (int)(min(ge, hi) - lo);
-                ++n;
-            }
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], CWARPS);
         }
-        mi.nseg = n;
-        mi.abort_flag = 0;
-        mi.b_done = 0;
-        for (int s = 0; s < SA; ++s) {
-            mbar_init(&full_a[s], 1);
-            mbar_init(&empty_a[s], AWARPS);
-        }
-        for (int s = 0; s < SB; ++s) {
-            mbar_init(&full_b[s], 1);
-            mbar_init(&empty_b[s], BWARPS);
-        }
+        sm.abort_flag = 0;
         fence_mbar_init();
     }
+    for (int g = threadIdx.x; g < G; g += blockDim.x)
+        sm.offs[g] = offs[g];
     __syncthreads();
-    const int nseg = mi.nseg;
-    const int R = p.rounds;
-    const int64_t L = p.L;
-    constexpr int PRODUCER_A = (NB + NA) / 32;
 
-    if (warp >= PRODUCER_A) {
-        // ------------------------------------------------ producer warps
-        // PRODUCER_A streams the strips from HBM for pass A, keeping them in
-        // L2; PRODUCER_B streams them again out of L2 for pass B. B's data
-        // does not depend on the amax barrier (only its scales do), so its
-        // producer just runs ahead within its ring.
+    // inverse scales of every (group, line), empty groups included
+    for (int64_t lt = blockIdx.x; lt < tiles_l; lt += gridDim.x)
+        for (int i = threadIdx.x; i < G * TL; i += blockDim.x) {
+            const int g = i / TL;
+            const int64_t l = lt * TL + (i % TL);
+            if (l < L)
+                inv[(int64_t)g * L + l] = fp8_inv(fp8_scale(__uint_as_float(__ldg(amax + (int64_t)g * L + l))));
+        }
+
+    if (warp == CWARPS) {
+        // ------------------------------------------------ producer warp
         if (lane == 0) {
-            const bool is_a = warp == PRODUCER_A;
-            const uint64_t pol = is_a ? policy_evict_last() : policy_evict_first();
-            uint8_t *ring = is_a ? ring_a : ring_b;
-            uint64_t *full = is_a ? full_a : full_b, *empty = is_a ? empty_a : empty_b;
-            const int S = is_a ? SA : SB;
-            int seq = 0;
-            for (int r = 0; r < R; ++r)
-                if (!ring_fill(ring, full, empty, S, seq, &tm_in, r * W, lo, nbox, pol, p.wait_ns))
+            int it = 0;
+            for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+                const int s = it % STAGES;
+                if (it >= STAGES && !mbar_wait(&sm.empty[s], ((uint32_t)(it / STAGES) & 1u) ^ 1u, wait_ns))
                     break;
-            ring_drain(full, S, seq, p.wait_ns);
+                if (drop_load && blockIdx.x == 0 && it == 0)
+                    continue; // test hook: this tile never arrives
+                const int64_t pt = t / tiles_l, lt = t - pt * tiles_l;
+                mbar_arrive_expect_tx(&sm.full[s], IN_BYTES);
+                tma_load_2d(sm.in[s], &tm_in, &sm.full[s], (int)(lt * TL), (int)(pt * TP));
+            }
+            // drain: every issued fill lands before the CTA exits
+            for (int j = it - STAGES; j < it; ++j)
+                if (j >= 0 && !(drop_load && blockIdx.x == 0 && j == 0))
+                    mbar_wait(&sm.full[j % STAGES], (uint32_t)(j / STAGES) & 1u, wait_ns);
         }
         return;
     }
 
-    if (warp >= BWARPS) {
-        // ------------------------------------------------ amax warps (pass A)
-        // thread = one line pair, all 16 rows of each box
-        const int ta = threadIdx.x - NB;
-        const int lp = ta;
-        int seq = 0;
-        for (int r = 0; r < R; ++r) {
-            // keep at most two strips live in L2: strip r may start once this
-            // CTA's cast of strip r-2 is done
-            if (r >= 2 && ta == 0) {
-                const uint64_t t0 = globaltimer();
-                while (*(volatile int *)&mi.b_done < r - 1 && !*(volatile int *)&mi.abort_flag) {
-                    if (globaltimer() - t0 > p.wait_ns) {
-                        set_status(MXQ_ERR_TIMEOUT);
-                        mi.abort_flag = 1;
-                        break;
-                    }
-                }
+    // ---------------------------------------------------- consumer warps
+    const int w = warp; // rows 32w .. 32w+31 of the tile
+    // group of the block's first row and the amax words of the lane's lines
+    struct Pre {
+        int g;
+        uint32_t a0, a1;
+    };
+    auto prefetch = [&](int64_t t) {
+        Pre pr;
+        const int64_t pt = t / tiles_l, lt = t - pt * tiles_l;
+        const int64_t p0 = pt * TP + 32 * w;
+        const int64_t l0 = lt * TL + 2 * lane;
+        pr.g = group_of(sm.offs, G, p0);
+        const unsigned *row = amax + (int64_t)pr.g * L;
+        pr.a0 = l0 < L ? __ldg(row + l0) : 0u;
+        pr.a1 = l0 + 1 < L ? __ldg(row + l0 + 1) : 0u;
+        return pr;
+    };
+    bool prev_stored = true;
+    int it = 0;
+    Pre cur = {0, 0u, 0u};
+    if ((int64_t)blockIdx.x < total)
+        cur = prefetch(blockIdx.x);
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+        const int s = it % STAGES;
+        const int ob = it & 1;
+        const int64_t pt = t / tiles_l, lt = t - pt * tiles_l;
+        const int64_t p0 = pt * TP + 32 * w;          // this warp's first position
+        const int64_t l0 = lt * TL + 2 * lane;        // this lane's lines l0, l0+1
+        Pre nxt = cur;
+        if (t + gridDim.x < total)
+            nxt = prefetch(t + gridDim.x);
+        bool ok = mbar_wait(&sm.full[s], (uint32_t)(it / STAGES) & 1u, wait_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok)
+            sm.abort_flag = 1;
+        const uint32_t *tile = reinterpret_cast<const uint32_t *>(sm.in[s]);
+        uint32_t v[32];
+        uint32_t dep = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            v[i] = tile[(w * 32 + i) * (TL / 2) + lane];
+            dep ^= v[i];
+        }
+        release_slot_after(&sm.empty[s], dep);
+
+        const int g = cur.g;
+        uint32_t q0[8], q1[8]; // lines l0, l0+1: 32 position bytes each
+        if (p0 < end_all && (int64_t)sm.offs[g] >= p0 + 32) {
+            // the block lies in one group
+            const float s0 = fp8_scale(__uint_as_float(cur.a0)), s1 = fp8_scale(__uint_as_float(cur.a1));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t *r = v + 4 * j;
+                q0[j] = e4m3x2(__fmul_rn(bf16_lo(r[0]), s0), __fmul_rn(bf16_lo(r[1]), s0)) |
+                        (e4m3x2(__fmul_rn(bf16_lo(r[2]), s0), __fmul_rn(bf16_lo(r[3]), s0)) << 16);
+                q1[j] = e4m3x2(__fmul_rn(bf16_hi(r[0]), s1), __fmul_rn(bf16_hi(r[1]), s1)) |
+                        (e4m3x2(__fmul_rn(bf16_hi(r[2]), s1), __fmul_rn(bf16_hi(r[3]), s1)) << 16);
             }
-            for (int i = ta; i < ASEG * W; i += NA)
-                atab[i] = 0u;
-            named_barrier(2, NA);
-            if (*(volatile int *)&mi.abort_flag)
-                break;
-            const int64_t la = (int64_t)r * W + 2 * lp;
-            int cs = 0;
-            int next = nseg ? mi.seg_hi[0] : 0;
-            uint32_t acc = 0;
-            auto flush = [&](int seg, uint32_t v) {
-                if (!v)
-                    return;
-                if (seg < ASEG) {
-                    atomicMax(&atab[seg * W + 2 * lp], v << 16);
-                    atomicMax(&atab[seg * W + 2 * lp + 1], v & 0xFFFF0000u);
-                } else {
-                    unsigned *dst = p.amax + (int64_t)mi.seg_g[seg] * L + la;
-                    if (la < L)
-                        atomicMax(dst, v << 16);
-                    if (la + 1 < L)
-                        atomicMax(dst + 1, v & 0xFFFF0000u);
-                }
+        } else {
+            // the block crosses group ends (or offs[G-1]): per-row group
+            auto scale_of = [&](int grp, int64_t l) {
+                return l < L ? fp8_scale(__uint_as_float(__ldg(amax + (int64_t)grp * L + l))) : 0.0f;
             };
-            for (int b = 0; b < nbox; ++b, ++seq) {
-                const int s = seq % SA;
-                bool ok = mbar_wait(&full_a[s], (uint32_t)(seq / SA) & 1u, p.wait_ns);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok)
-                    mi.abort_flag = 1;
-                const uint32_t *bp = reinterpret_cast<const uint32_t *>(ring_a + s * BOX_BYTES) + lp;
-                uint32_t v[BOXR];
+            int gg = g;
 #pragma unroll
-                for (int k = 0; k < BOXR; ++k)
-                    v[k] = bp[k * (W / 2)];
-                // release the slot once every word has landed in a register
-                uint32_t dep = 0;
+            for (int j = 0; j < 8; ++j) {
+                uint32_t a0 = 0, a1 = 0;
 #pragma unroll
-                for (int k = 0; k < BOXR; ++k)
-                    dep ^= v[k];
-                release_slot_after(&empty_a[s], dep);
-                const int row0 = b * BOXR;
-                const int rlast = row0 + BOXR - 1;
-                if (rlast < next && rlast < rows_here) {
-                    // all 16 rows valid and in the current segment
-                    uint32_t m0 = absmax2(absmax2(absmax2(v[0], v[1]), absmax2(v[2], v[3])),
-                                          absmax2(absmax2(v[4], v[5]), absmax2(v[6], v[7])));
-                    uint32_t m1 = absmax2(absmax2(absmax2(v[8], v[9]), absmax2(v[10], v[11])),
-                                          absmax2(absmax2(v[12], v[13]), absmax2(v[14], v[15])));
-                    acc = absmax_bf16x2(absmax_bf16x2(acc, m0), m1);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < BOXR; ++k) {
-                        const int row = row0 + k;
-                        if (row < rows_here) {
-                            if (row >= next) {
-                                flush(cs, acc);
-                                acc = 0;
-                                do {
-                                    ++cs;
-                                } while (row >= mi.seg_hi[cs]);
-                                next = mi.seg_hi[cs];
-                            }
-                            acc = absmax_bf16x2(acc, v[k]);
-                        }
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    const int64_t row = p0 + 4 * j + k;
+                    while (gg + 1 < G && (int64_t)sm.offs[gg] <= row)
+                        ++gg;
+                    const float s0 = scale_of(gg, l0), s1 = scale_of(gg, l0 + 1);
+                    const uint32_t x = v[4 * j + k];
+                    a0 |= e4m3x2(__fmul_rn(bf16_lo(x), s0), 0.0f) << (8 * k);
+                    a1 |= e4m3x2(__fmul_rn(bf16_hi(x), s1), 0.0f) << (8 * k);
                 }
+                q0[j] = a0;
+                q1[j] = a1;
             }
-            if (rows_here > 0)
-                flush(cs, acc);
-            named_barrier(2, NA);
-            for (int i = ta; i < min(nseg, ASEG) * W; i += NA) {
-                const uint32_t v = atab[i];
-                const int64_t l = (int64_t)r * W + (i % W);
-                if (v && l < L)
-                    atomicMax(p.amax + (int64_t)mi.seg_g[i / W] * L + l, v);
-            }
-            // each thread's global atomics (here and in flush) must be
-            // performed at GPU scope before the arrival: bar.sync orders
-            // memory only within the CTA
-            __threadfence();
-            named_barrier(2, NA);
-            if (ta == 0 && !(p.skip_arrival && blockIdx.x == 0))
-                red_release_gpu_add(p.counters + r, 1);
         }
-        return;
-    }
+        cur = nxt;
 
-    // ---------------------------------------------------- cast warps (pass B)
-    const int tb = threadIdx.x;
-    const int lp = tb & 127;       // line pair within the strip: lines 2lp, 2lp+1
-    const int half = tb >> 7;      // slices half, half + 2 of each store box
-    const int bsel = (lp >> 2) & 1;
-    const int full_groups = rows_here / OPOS;
-    const uint64_t out_pol = policy_evict_first();
-    int seq = 0;
-    for (int r = 0; r < R; ++r) {
-        // wait for every CTA's amax of strip r
-        if (tb == 0) {
-            const uint64_t t0 = globaltimer();
-            while (ld_acquire_gpu(p.counters + r) < ncta && !*(volatile int *)&mi.abort_flag) {
-                if (globaltimer() - t0 > p.wait_ns) {
-                    set_status(MXQ_ERR_TIMEOUT);
-                    mi.abort_flag = 1;
-                    break;
-                }
-            }
+        // a tile wholly below offs[G-1] leaves through the staging tile and a
+        // TMA store; the tile holding offs[G-1] is written directly
+        const bool full_tile = pt * TP + TP <= end_all;
+        // staging buffer ob was read by the store of tile it-2; when tile
+        // it-1 issued no store, that one may be the newest group
+        if (threadIdx.x == 0) {
+            if (prev_stored)
+                bulk_wait_read<1>();
+            else
+                bulk_wait_read<0>();
         }
-        named_barrier(1, NB);
-        if (*(volatile int *)&mi.abort_flag)
-            break;
-        for (int g = blockIdx.x; g < p.G; g += ncta)
-            for (int li = tb; li < W; li += NB) {
-                const int64_t l = (int64_t)r * W + li;
-                if (l < L)
-                    p.inv[(int64_t)g * L + l] = fp8_inv(fp8_scale(__uint_as_float(__ldcg(p.amax + (int64_t)g * L + l))));
+        named_barrier(1, CWARPS * 32);
+        if (full_tile) {
+            // staging: 64 rows (lines) x 128 bytes (positions), 16-byte chunk c
+            // of row r at chunk c ^ (r & 7) (128B swizzle); the lane's two
+            // lines alternate so each 16-byte store hits 8 bank groups
+            const uint32_t ob_addr = smem_u32(sm.out[ob]);
+            const int bsel = (lane >> 2) & 1;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int b = bsel ^ (j & 1), h = j >> 1;
+                const int row = 2 * lane + b;
+                const int chunk = (2 * w + h) ^ (row & 7);
+                uint4 val;
+                if (b) val = make_uint4(q1[4 * h], q1[4 * h + 1], q1[4 * h + 2], q1[4 * h + 3]);
+                else   val = make_uint4(q0[4 * h], q0[4 * h + 1], q0[4 * h + 2], q0[4 * h + 3]);
+                sts_v4(ob_addr + row * 128 + chunk * 16, val);
             }
-        const int64_t lb = (int64_t)r * W + 2 * lp;
-        int cs = 0;
-        int sc_seg = -1; // segment whose scales s0b, s1b hold
-        float s0b = 0.0f, s1b = 0.0f;
-        auto scales = [&](int seg, float &s0, float &s1) {
-            const unsigned *src = p.amax + (int64_t)mi.seg_g[seg] * L + lb;
-            s0 = lb < L ? fp8_scale(__uint_as_float(__ldcg(src))) : 0.0f;
-            s1 = lb + 1 < L ? fp8_scale(__uint_as_float(__ldcg(src + 1))) : 0.0f;
-        };
-        for (int og = 0; og < ngroups; ++og) {
-            const int nb = min(GROUP_BOXES, nbox - og * GROUP_BOXES);
-            bool ok = true;
-            for (int j = 0; j < nb; ++j)
-                ok &= mbar_wait(&full_b[(seq + j) % SB], (uint32_t)((seq + j) / SB) & 1u, p.wait_ns);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok)
-                mi.abort_flag = 1;
-            const int ob = og & 1;
-            if (tb == 0)
-                bulk_wait_read<1>(); // staging buffer ob was read by the store of group og-2
-            named_barrier(1, NB);
-            const uint32_t stg_addr = smem_u32(stg + ob * OBOX_BYTES);
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const int sl = half + 2 * t; // 16-row slice of the store box
-                const int i0 = og * OPOS + sl * BOXR; // first row (relative to lo)
-                if (sl >= nb || i0 >= rows_here)
-                    continue;
-                const uint32_t *box = reinterpret_cast<const uint32_t *>(ring_b + ((seq + sl) % SB) * BOX_BYTES) + lp;
-                uint32_t x[BOXR];
-#pragma unroll
-                for (int k = 0; k < BOXR; ++k)
-                    x[k] = box[k * (W / 2)];
-                while (cs + 1 < nseg && mi.seg_hi[cs] <= i0)
-                    ++cs;
-                uint32_t o0[4], o1[4];
-                if (mi.seg_hi[cs] >= min(i0 + BOXR, rows_here)) {
-                    if (sc_seg != cs) {
-                        scales(cs, s0b, s1b);
-                        sc_seg = cs;
-                    }
-                    const float s0 = s0b, s1 = s1b;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t x0 = x[4 * k + 0], x1 = x[4 * k + 1];
-                        const uint32_t x2 = x[4 * k + 2], x3 = x[4 * k + 3];
-                        o0[k] = e4m3x2(__fmul_rn(bf16_lo(x0), s0), __fmul_rn(bf16_lo(x1), s0)) |
-                                (e4m3x2(__fmul_rn(bf16_lo(x2), s0), __fmul_rn(bf16_lo(x3), s0)) << 16);
-                        o1[k] = e4m3x2(__fmul_rn(bf16_hi(x0), s1), __fmul_rn(bf16_hi(x1), s1)) |
-                                (e4m3x2(__fmul_rn(bf16_hi(x2), s1), __fmul_rn(bf16_hi(x3), s1)) << 16);
-                    }
-                } else {
-                    // the slice crosses group boundaries: per-row scale
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        uint32_t a0 = 0, a1 = 0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int row = i0 + 4 * k + j;
-                            int sj = cs;
-                            while (sj + 1 < nseg && mi.seg_hi[sj] <= row)
-                                ++sj;
-                            float s0, s1;
-                            scales(sj, s0, s1);
-                            const uint32_t xv = x[4 * k + j];
-                            a0 |= e4m3x2(__fmul_rn(bf16_lo(xv), s0), 0.0f) << (8 * j);
-                            a1 |= e4m3x2(__fmul_rn(bf16_hi(xv), s1), 0.0f) << (8 * j);
-                        }
-                        o0[k] = a0;
-                        o1[k] = a1;
-                    }
-                }
-                if (og < full_groups) {
-                    // staging: 256 lines x 64 bytes; 16-byte chunk c of line l
-                    // at chunk c ^ ((l >> 1) & 3) (64B swizzle). Alternating
-                    // the lane's two lines keeps each 16-byte store
-                    // instruction on 8 distinct bank groups.
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int bb = bsel ^ j;
-                        const int line = 2 * lp + bb;
-                        const int pc = sl ^ (lp & 3);
-                        const uint4 val = bb ? make_uint4(o1[0], o1[1], o1[2], o1[3])
-                                             : make_uint4(o0[0], o0[1], o0[2], o0[3]);
-                        sts_v4(stg_addr + line * OPOS + pc * 16, val);
-                    }
-                } else {
-                    // the store box that holds end_all: direct byte stores
-#pragma unroll
-                    for (int bb = 0; bb < 2; ++bb) {
-                        const int64_t l = lb + bb;
-                        if (l >= L)
-                            continue;
-                        uint8_t *dst = p.out + l * p.P + lo + i0;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const uint32_t word = bb ? o1[j >> 2] : o0[j >> 2];
-                            if (i0 + j < rows_here)
-                                dst[j] = (uint8_t)(word >> (8 * (j & 3)));
-                        }
-                    }
-                }
-            }
-            // the ring reads above (generic proxy) and the staging writes are
-            // ordered before the boxes' next TMA fill and the TMA store
             fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                for (int j = 0; j < nb; ++j)
-                    mbar_arrive(&empty_b[(seq + j) % SB]);
-            seq += nb;
-            named_barrier(1, NB);
-            if (tb == 0 && og < full_groups) {
-                tma_store_2d_hint(&tm_out, stg + ob * OBOX_BYTES, (int)(lo + og * OPOS), r * W, out_pol);
-                bulk_commit();
+        } else {
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+                const int64_t l = l0 + bb;
+                if (l >= L)
+                    continue;
+                uint8_t *dst = out + l * P + p0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t word = bb ? q1[j >> 2] : q0[j >> 2];
+                    if (p0 + j < end_all)
+                        dst[j] = (uint8_t)(word >> (8 * (j & 3)));
+                }
             }
         }
-        named_barrier(1, NB);
-        if (tb == 0)
-            *(volatile int *)&mi.b_done = r + 1;
+        named_barrier(1, CWARPS * 32);
+        if (sm.abort_flag)
+            break;
+        if (threadIdx.x == 0 && full_tile) {
+            tma_store_2d(&tm_out, sm.out[ob], (int)(pt * TP), (int)(lt * TL));
+            bulk_commit();
+        }
+        prev_stored = full_tile;
     }
-    if (tb == 0)
+    if (threadIdx.x == 0)
         bulk_wait<0>();
 }
 

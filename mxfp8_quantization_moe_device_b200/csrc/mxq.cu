@@ -16,7 +16,7 @@ using namespace mxq;
 namespace {
 
 std::atomic<int64_t> g_wait_ns{1000000000LL};
-std::atomic<int> g_skip_arrival{0};
+std::atomic<int> g_drop_load{0};
 std::atomic<int> g_force_path{0};
 
 uint64_t wait_ns() { return (uint64_t)g_wait_ns.load(); }
@@ -70,7 +70,8 @@ struct DevInfo {
     int sms = 0;
     int smem_optin = 0;
     int coop = 0;
-    int jag_per_sm = 0;   // resident CTAs of the single-pass jagged kernel
+    int amx_per_sm = 0;   // resident CTAs of the jagged amax pass
+    int cst_per_sm = 0;   // resident CTAs of the jagged cast pass
     int rb_per_sm = 0;    // resident CTAs of the 1x128 kernel
     int mx32_per_sm = 0;  // resident CTAs of the 1x32 kernel
 };
@@ -92,11 +93,13 @@ int device_info(const DevInfo **out)
             return MXQ_ERR_CUDA;
         if (cudaFuncSetAttribute(mx3d::k_mx_3d_colwise, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mx3d::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(k_jagged_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 di.smem_optin - (int)sizeof(jag::Misc) - 64) != cudaSuccess)
+            cudaFuncSetAttribute(k_jagged_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)jag::cst::SMEM_BYTES) != cudaSuccess)
             return MXQ_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.jag_per_sm, k_jagged_fused, jag::THREADS,
-                                                          jag::SMEM_BYTES) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.amx_per_sm, k_jagged_amax, jag::amx::THREADS, 0) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.cst_per_sm, k_jagged_cast, jag::cst::THREADS,
+                                                          jag::cst::SMEM_BYTES) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.rb_per_sm, k_fp8_1x128, RB_THREADS, 0) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mx32_per_sm, k_mx_1x32, RB_THREADS, 0) != cudaSuccess)
             return MXQ_ERR_CUDA;
@@ -134,60 +137,54 @@ int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_
 
 // ------------------------------------------------------------ jagged plan
 struct JaggedPlan {
-    bool fused = false;
-    int chunk = 0, ncta = 0, rounds = 0;
-    size_t smem = 0;
-    size_t ws_amax = 0, ws_total = 0;
+    bool twopass = false;
+    int wpc = 0;              // amax pass: warps per 256-line chunk
+    int grid_a = 0, grid_c = 0;
+    size_t ws = 0;
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// host-checkable part of the single-pass conditions (no device queries)
-bool fused_layout_ok(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, int G, const void *out)
+// host-checkable conditions of the two-pass kernels (no device queries):
+// lines contiguous, 16-byte aligned rows for the vector loads and the TMA
+// maps of input and output, at most jag::MAX_SEG groups
+bool twopass_layout_ok(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, int G, const void *out)
 {
     return s_line == 1 && s_pos % 8 == 0 && s_pos >= L && L > 0 && P > 0 && P % 16 == 0 && G >= 1 &&
            G <= jag::MAX_SEG && (in == nullptr || aligned(in, 16)) && (out == nullptr || aligned(out, 16)) &&
            P < (int64_t(1) << 31) && L < (int64_t(1) << 31);
 }
 
-size_t fused_workspace(int64_t L, int G)
-{
-    const int64_t rounds = (L + jag::W - 1) / jag::W;
-    return round_up((size_t)G * (size_t)L * 4, 256) + round_up((size_t)rounds * 4, 256);
-}
+size_t twopass_workspace(int64_t L, int G) { return round_up((size_t)G * (size_t)L * 4, 256); }
 
 int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, int G, const void *out,
                 JaggedPlan *pl)
 {
     *pl = JaggedPlan();
     const int force = g_force_path.load();
-    if (force == 2 || !fused_layout_ok(in, L, P, s_line, s_pos, G, out))
+    if (force == 2 || !twopass_layout_ok(in, L, P, s_line, s_pos, G, out))
         return MXQ_OK;
-    // small problems are launch- and latency-bound: the generic kernel (no
-    // workspace clear, no cooperative launch, no strip barriers) is faster
+    // small problems are launch- and latency-bound: the generic kernel (one
+    // launch, no workspace clear) is faster
     if (force == 0 && L * P <= (int64_t(1) << 21))
         return MXQ_OK;
     const DevInfo *di = nullptr;
     int rc = device_info(&di);
     if (rc != MXQ_OK)
         return rc;
-    if (!di->coop)
+    if (di->amx_per_sm < 1 || di->cst_per_sm < 1)
         return MXQ_OK;
-    const int64_t per = (P + di->sms - 1) / di->sms;
-    const int chunk = (int)((per + jag::OPOS - 1) / jag::OPOS * jag::OPOS);
-    const int ncta = (int)((P + chunk - 1) / chunk);
-    const size_t smem = jag::SMEM_BYTES;
-    if ((int)smem > di->smem_optin - (int)sizeof(jag::Misc) - 64)
-        return MXQ_OK;
-    if (di->jag_per_sm < 1 || ncta > di->jag_per_sm * di->sms)
-        return MXQ_OK;
-    pl->fused = true;
-    pl->chunk = chunk;
-    pl->ncta = ncta;
-    pl->rounds = (int)((L + jag::W - 1) / jag::W);
-    pl->smem = smem;
-    pl->ws_amax = round_up((size_t)G * (size_t)L * 4, 256);
-    pl->ws_total = fused_workspace(L, G);
+    pl->twopass = true;
+    // amax pass: every resident warp is a worker; the warps of a 256-line
+    // chunk split the positions into equal runs of at least 64 rows
+    const int64_t chunks = (L + jag::amx::W - 1) / jag::amx::W;
+    const int64_t warps = (int64_t)di->sms * di->amx_per_sm * (jag::amx::THREADS / 32);
+    const int64_t wpc = std::max<int64_t>(1, std::min<int64_t>(warps / chunks, (P + 63) / 64));
+    pl->wpc = (int)wpc;
+    pl->grid_a = (int)((chunks * wpc * 32 + jag::amx::THREADS - 1) / jag::amx::THREADS);
+    const int64_t tiles = (P + jag::cst::TP - 1) / jag::cst::TP * ((L + jag::cst::TL - 1) / jag::cst::TL);
+    pl->grid_c = (int)std::min<int64_t>(tiles, (int64_t)di->sms * di->cst_per_sm);
+    pl->ws = twopass_workspace(L, G);
     return MXQ_OK;
 }
 
@@ -204,42 +201,37 @@ int jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, 
     int rc = plan_jagged(in, L, P, s_line, s_pos, G, out, &pl);
     if (rc != MXQ_OK)
         return rc;
-    if (g_force_path.load() == 1 && !pl.fused)
+    if (g_force_path.load() == 1 && !pl.twopass)
         return MXQ_ERR_UNSUPPORTED;
-    if (pl.fused) {
-        if (!ws || ws_bytes < pl.ws_total)
+    if (pl.twopass) {
+        if (!ws || ws_bytes < pl.ws)
             return MXQ_ERR_WORKSPACE;
         if (!aligned(ws, 256))
             return MXQ_ERR_ALIGN;
-        CUtensorMap tin, tout;
+        // cast pass: 128 positions x 64 lines in, the 64 x 128 transpose out
+        CUtensorMap tc, to;
         const uint64_t din[2] = {(uint64_t)L, (uint64_t)P};
         const uint64_t sin[1] = {(uint64_t)s_pos * 2};
-        const uint32_t bin[2] = {jag::W, jag::BOXR};
-        rc = make_map(&tin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, din, sin, bin, CU_TENSOR_MAP_SWIZZLE_NONE);
+        const uint32_t bc[2] = {jag::cst::TL, jag::cst::TP};
+        rc = make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, din, sin, bc, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc != MXQ_OK)
             return rc;
         const uint64_t dout[2] = {(uint64_t)P, (uint64_t)L};
         const uint64_t sout[1] = {(uint64_t)P};
-        const uint32_t bout[2] = {jag::OPOS, jag::W};
-        rc = make_map(&tout, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_64B);
+        const uint32_t bo[2] = {jag::cst::TP, jag::cst::TL};
+        rc = make_map(&to, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bo, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc != MXQ_OK)
             return rc;
-        if (cudaMemsetAsync(ws, 0, pl.ws_total, stream) != cudaSuccess)
+        unsigned *amax = static_cast<unsigned *>(ws);
+        if (cudaMemsetAsync(ws, 0, (size_t)G * (size_t)L * 4, stream) != cudaSuccess)
             return MXQ_ERR_CUDA;
-        jag::Params p;
-        p.L = L;
-        p.P = P;
-        p.G = G;
-        p.chunk = pl.chunk;
-        p.rounds = pl.rounds;
-        p.offs = offs;
-        p.out = static_cast<uint8_t *>(out);
-        p.inv = inv;
-        p.amax = static_cast<unsigned *>(ws);
-        p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + pl.ws_amax);
-        p.wait_ns = wait_ns();
-        p.skip_arrival = g_skip_arrival.load();
-        return launch(k_jagged_fused, dim3(pl.ncta), dim3(jag::THREADS), pl.smem, stream, true, tin, tout, p);
+        rc = launch(k_jagged_amax, dim3(pl.grid_a), dim3(jag::amx::THREADS), 0, stream, false,
+                    static_cast<const uint16_t *>(in), L, P, s_pos, offs, G, pl.wpc, amax);
+        if (rc != MXQ_OK)
+            return rc;
+        return launch(k_jagged_cast, dim3(pl.grid_c), dim3(jag::cst::THREADS), jag::cst::SMEM_BYTES, stream, false,
+                      tc, to, L, P, offs, G, static_cast<const unsigned *>(amax), static_cast<uint8_t *>(out), inv,
+                      wait_ns(), g_drop_load.load());
     }
     const DevInfo *di = nullptr;
     rc = device_info(&di);
@@ -279,9 +271,9 @@ size_t fp8_quant_jagged_workspace_bytes(int64_t rows, int64_t cols, int64_t stri
 {
     const int64_t L = is_colwise ? cols : rows, P = is_colwise ? rows : cols;
     const int64_t sl = is_colwise ? stride_col : stride_row, sp = is_colwise ? stride_row : stride_col;
-    if (!fused_layout_ok(nullptr, L, P, sl, sp, num_groups, nullptr))
+    if (!twopass_layout_ok(nullptr, L, P, sl, sp, num_groups, nullptr))
         return 0;
-    return fused_workspace(L, num_groups);
+    return twopass_workspace(L, num_groups);
 }
 
 int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols, int32_t block_rows, int32_t block_cols,
@@ -429,9 +421,9 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
 // that owns all of the device memory and hands it no workspace argument, or
 // a latency-critical path where cudaMalloc's implicit device-wide
 // synchronization is not acceptable. This entry point needs no workspace from
-// them: its scratch (the per-(group, column) amax table and the round
-// counters) lives in the fixed-size array below, which every GPU that loads
-// this library keeps for the life of the process.
+// them: its scratch (the per-(group, column) amax table) lives in the
+// fixed-size array below, which every GPU that loads this library keeps for
+// the life of the process.
 //
 // The array's host-side name is only a stand-in for the device symbol, so its
 // device address is looked up once per device with cudaGetSymbolAddress, with
@@ -526,7 +518,7 @@ int mxq_testing_set(int32_t what, int64_t value)
 {
     switch (what) {
     case MXQ_TESTING_WAIT_LIMIT_NS: g_wait_ns.store(value > 0 ? value : 1000000000LL); return MXQ_OK;
-    case MXQ_TESTING_SKIP_ARRIVAL: g_skip_arrival.store(value ? 1 : 0); return MXQ_OK;
+    case MXQ_TESTING_SKIP_ARRIVAL: g_drop_load.store(value ? 1 : 0); return MXQ_OK;
     case MXQ_TESTING_FORCE_PATH:
         if (value < 0 || value > 2)
             return MXQ_ERR_UNSUPPORTED;

@@ -54,7 +54,7 @@ def test_pure_host_functions(lib):
     assert lib.mx_blocked_grouped_rows_bound(5, 5) == 640
     # jagged workspace: only the contiguous-line layout needs one
     ws = lib.fp8_quant_jagged_workspace_bytes(65536, 4096, 4096, 1, 16, 1)
-    assert ws >= 16 * 4096 * 4 + 64 * 4
+    assert ws >= 16 * 4096 * 4  # the fp32 (group, column) amax table
     assert lib.fp8_quant_jagged_workspace_bytes(4096, 65536, 1, 4096, 16, 0) == ws
     assert lib.fp8_quant_jagged_workspace_bytes(100, 96, 1, 100, 2, 0) == 0  # cols % 16 != 0
     assert lib.fp8_quant_jagged_workspace_bytes(64, 64, 1, 64, 65, 0) == 0   # too many groups

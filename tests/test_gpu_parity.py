@@ -76,10 +76,12 @@ JAGGED = [
     (64, 64, [64]),
     (32, 8, [0, 0, 32]),
     (9600, 72, [17, 4000, 4001, 9583]),  # several position chunks per CTA range
+    (256, 64, [0, 0, 0]),                # every group empty: only inverse scales written
+    (1024, 4104, [100, 700, 1024]),      # 17 line chunks, the last one 8 lines wide
 ]
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["single_pass", "generic"])
+@pytest.mark.parametrize("path", [1, 2], ids=["two_pass", "generic"])
 @pytest.mark.parametrize("M,D,spec", JAGGED)
 def test_jagged_colwise_and_rowwise_vs_oracle(M, D, spec, path):
     mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
@@ -147,6 +149,25 @@ def test_jagged_colwise_strided_view_generic():
     assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
 
 
+@pytest.mark.parametrize("path", [1, 2], ids=["two_pass", "generic"])
+def test_jagged_colwise_padded_rows_partial_lane(path):
+    """Row stride 208 elements, 203 columns: the last lane of the two-pass
+    amax pass holds 3 of its 8 lines, and the TMA maps see a padded stride."""
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
+    try:
+        base = synth.row_scaled_normal_bf16(1024, 208, seed=11, device=DEV)
+        x = base[:, :203]
+        o = torch.tensor([300, 300, 1000], dtype=torch.int32)
+        ref_q, ref_inv = oracle.fp8_quant_jagged_colwise(words(base).reshape(-1), 1024, 203, 208, 1, o.numpy())
+        q, inv = mxq.fp8_quant_jagged_colwise(x, o.to(DEV))
+        assert status_ok()
+        got = u8(q.t())  # (203, 1024) buffer
+        assert np.array_equal(got[:, :1000], ref_q[:, :1000])
+        assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
+    finally:
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+
+
 def test_jagged_tiny_config_both_outputs():
     """The tiny jagged workload: A (256, 512), G=4 multinomial groups of 16-row units;
     colwise on A and rowwise on A^T."""
@@ -207,8 +228,8 @@ def test_jagged_full_size_backward_operands():
 def test_jagged_full_size_scales_every_unit_repeated():
     """Every (group, column) inverse scale of the full-size colwise op equals
     the fp32 reciprocal of 448 / max(amax, 1e-12) of its unit, over several
-    calls: the single-pass kernel's cross-CTA amax reduction and its TMA ring
-    reuse must never race. amax here is a max over bf16 values (exact); the
+    calls: the amax pass's merge of per-item maxima across CTAs and the reuse
+    of both passes' TMA rings must never race. amax here is a max over bf16 values (exact); the
     scale arithmetic is cross-checked against the oracle on a sample."""
     _, inp, offs = synth.jagged_bwd(device=DEV)
     o = offs.tolist()
@@ -459,9 +480,9 @@ def test_bad_offsets_are_reported_and_nothing_is_written():
 
 
 def test_barrier_timeout_is_reported_and_context_survives():
-    """One CTA skips its arrival on the amax barrier: the others' bounded waits
-    expire, the kernel returns, the status reads TIMEOUT and the next call
-    on the same context is correct."""
+    """One CTA of the cast pass leaves its first TMA load unissued: the bounded
+    waits on that ring slot expire, the kernels return, the status reads
+    TIMEOUT and the next call on the same context is correct."""
     x = synth.row_scaled_normal_bf16(4096, 128, seed=2, device=DEV)
     offs = torch.tensor([1000, 4096], dtype=torch.int32)
     try:
