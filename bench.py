@@ -58,7 +58,7 @@ def parse():
     p.add_argument("--no-per-shape", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--reps", type=int, default=20, help="reps per shape in the per-shape sweep")
+    p.add_argument("--reps", type=int, default=50, help="reps per shape in the per-shape sweep (cold and hot each)")
     p.add_argument("--profile-op", default=None, choices=list(Workload.OPS),
                    help="run only this op (for single-kernel profiler captures)")
     p.add_argument("--iters", type=int, default=3, help="calls of --profile-op after one warm-up")
@@ -77,10 +77,19 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+KERNEL_FILES = {  # source files that define each kernel (plus common.cuh)
+    "k_fp8_1x128": "rowblock.cuh", "k_fp8_128x128": "rowblock.cuh", "k_mx_1x32": "rowblock.cuh",
+    "k_jagged_amax": "jagged.cuh", "k_jagged_cast": "jagged.cuh", "k_mx_3d_colwise": "mx3d.cuh",
+    "k_blocked_grouped": "blocked.cuh",
+}
+
+
+def kernel_source_hash(kernel):
+    """Hash of the sources a kernel is built from: its own header and the
+    shared device helpers."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp8_quantization_moe_device_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in ("common.cuh", KERNEL_FILES[kernel]):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -88,14 +97,18 @@ def kernel_source_hash():
 
 def load_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    on the kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        if d.get("source_hash") != kernel_source_hash():
-            return None
-        return d["kernels"][kernel]["dram_bytes_per_launch"]
+        total = 0
+        for k in kernel.split("+"):  # an op of several kernels: their sum
+            e = d["kernels"][k]
+            if e.get("source_hash") != kernel_source_hash(k):
+                return None
+            total += e["dram_bytes_per_launch"]
+        return total
     except Exception:
         return None
 
@@ -285,7 +298,10 @@ def flush_l2(torch, buf):
 
 
 def per_shape_sweep(wl, reps):
-    """us/call and GB/s per config shape, L2 flushed (256 MB write) before each rep."""
+    """us/call and GB/s per config shape after 5 warm-up calls: the median of
+    `reps` calls with the L2 flushed (256 MB write) before each, the median of
+    `reps` back-to-back calls with a hot L2 ("us_hot", labelled as such), and
+    the median host time to enqueue one call ("enqueue_us")."""
     torch, mxq = wl.torch, wl.mxq
     from mxfp8_quantization_moe_device_b200 import synth
     dev = wl.dev
@@ -294,22 +310,33 @@ def per_shape_sweep(wl, reps):
     rows = []
 
     def run(name, shape, fn, nbytes):
-        fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(reps):
-            flush_l2(torch, flush)
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
+        for _ in range(5):
             fn()
-            b.record()
-            b.synchronize()
-            ts.append(a.elapsed_time(b) * 1e3)
+        torch.cuda.synchronize()
+        ts, hot, enq = [], [], []
+        for cold in (True, False):
+            for _ in range(reps):
+                if cold:
+                    flush_l2(torch, flush)
+                else:
+                    # keep the GPU busy (~100 us, no memory traffic) while the
+                    # host enqueues, so that the events time the call alone
+                    torch.cuda._sleep(200000)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                h0 = time.perf_counter()
+                fn()
+                h1 = time.perf_counter()
+                b.record()
+                b.synchronize()
+                (ts if cold else hot).append(a.elapsed_time(b) * 1e3)
+                enq.append((h1 - h0) * 1e6)
         us = statistics.median(ts)
         gbs = nbytes / (us * 1e-6) / 1e9
         rows.append({"op": name, "shape": shape, "us": round(us, 3), "GB/s": round(gbs, 1),
-                     "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4)})
+                     "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4),
+                     "us_hot": round(statistics.median(hot), 3), "enqueue_us": round(statistics.median(enq), 1)})
 
     # tiny jagged
     a, offs = synth.tiny_jagged(device=dev)
@@ -363,26 +390,27 @@ def oracle_samples(wl):
         return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
     full = {n: b for n, _, b in wl.ops}
-    act = words(wl.act[:512])
-    wt = words(wl.wt[:256])
-    go = words(wl.grad_out[:, :96])        # (65536, 96): rowwise on its transpose
-    inp = words(wl.inp[:, :96])
-    w3 = words(wl.w3[0, :, :160]).reshape(1, 8192, 160)
-    tok = words(wl.tok[:256])
+    act = words(wl.act[:4096])
+    wt = words(wl.wt[:2048])
+    go = words(wl.grad_out[:, :768])       # (65536, <=768): rowwise on its transpose
+    inp = words(wl.inp[:, :768])
+    w3s = wl.w3[0, :, :1280]
+    w3 = words(w3s).reshape(1, w3s.shape[0], w3s.shape[1])
+    tok = words(wl.tok[:2048])
     from mxfp8_quantization_moe_device_b200 import synth
     scales = synth.uniform_u8((65536, 224), 0, 254, seed=9).numpy()  # synthetic, never a GPU output
     offs16 = wl.offs16.cpu().numpy()
     offs64 = wl.offs64.cpu().numpy()
-    M = go.shape[0]
+    M, C = go.shape
     return [
         ("blockwise_1x128", lambda: oracle.fp8_quant_blockwise(act, 1, 128), act.size * 3 + act.size // 128 * 4,
          full["blockwise_1x128"]),
         ("blockwise_128x128", lambda: oracle.fp8_quant_blockwise(wt, 128, 128), wt.size * 3 + wt.size // 16384 * 4,
          full["blockwise_128x128"]),
-        ("jagged_rowwise", lambda: oracle.fp8_quant_jagged_rowwise(go.reshape(-1), 96, M, 1, 96, offs16),
-         go.size * 3 + 16 * 96 * 4, full["jagged_rowwise"]),
-        ("jagged_colwise", lambda: oracle.fp8_quant_jagged_colwise(inp.reshape(-1), M, 96, 96, 1, offs16),
-         inp.size * 3 + 16 * 96 * 4, full["jagged_colwise"]),
+        ("jagged_rowwise", lambda: oracle.fp8_quant_jagged_rowwise(go.reshape(-1), C, M, 1, C, offs16),
+         go.size * 3 + 16 * C * 4, full["jagged_rowwise"]),
+        ("jagged_colwise", lambda: oracle.fp8_quant_jagged_colwise(inp.reshape(-1), M, C, C, 1, offs16),
+         inp.size * 3 + 16 * C * 4, full["jagged_colwise"]),
         ("mx_3d_colwise", lambda: oracle.mx_quant_3d_colwise(w3, 0 if wl.mx3d_mode == "floor" else 1),
          w3.size * 3 + w3.size // 32, full["mx_3d_colwise"]),
         ("mx_rowwise", lambda: oracle.mx_quant_rowwise(tok, 0), tok.size * 3 + tok.size // 32, full["mx_rowwise"]),
@@ -408,9 +436,15 @@ def run_oracle_samples(samples):
     return total / est / 1e9, spent, per
 
 
-SAMPLE_DESC = ("single-threaded C oracle on a slice of every op: act rows 0-511, weight rows 0-255, "
-               "grad_out/input columns 0-95 (all 65536 rows, G=16), expert 0 columns 0-159, tokens rows 0-255, "
+SAMPLE_DESC = ("single-threaded C oracle on a slice of every op: act rows 0-4095, weight rows 0-2047, "
+               "grad_out/input columns 0-767 (all 65536 rows, G=16), expert 0 columns 0-1279, tokens rows 0-2047, "
                "the full (65536,224) scale matrix; each op's time scaled to its full-size bytes")
+
+
+REF_SAMPLE_DESC = ("single-threaded C oracle, one pass per step over a slice of every op: act rows 0-511, "
+                   "weight rows 0-255, grad_out/input columns 0-95 (all 65536 rows, G=16), expert 0 columns "
+                   "0-159, tokens rows 0-255, the full (65536,224) scale matrix; each op's time scaled to its "
+                   "full-size bytes")
 
 
 # ----------------------------------------------------------------- e2e
@@ -595,7 +629,7 @@ def main_reference(args, world, rank):
            "data": "synthetic (seeded)",
            "config": {"workload": WORKLOAD, "step_bytes": total, "parallelism": "single-threaded CPU oracle"},
            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                            "sample": SAMPLE_DESC},
+                            "sample": REF_SAMPLE_DESC},
            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
            "wall_s": round(time.perf_counter() - t0, 1)}
     print(json.dumps(out))

@@ -24,11 +24,13 @@
 //                     global (G, L) fp32 table by atomicMax only at group ends.
 //                     The cast pass has the MX 3-D kernel's structure: a TMA
 //                     ring of 128 x 64 tiles, one consumer warp per 32-row
-//                     block, scales from the finished table (prefetched a tile
-//                     ahead), and the transpose leaving through a
-//                     128B-swizzled staging tile and TMA stores. The input is
-//                     read twice (5 B of HBM traffic per element instead of
-//                     3); in exchange neither kernel synchronizes across CTAs.
+//                     block, scales from the finished table, and the
+//                     transpose leaving through a 128B-swizzled staging tile
+//                     and TMA stores; its tile indices are 32-bit (64-bit
+//                     divisions per tile cost it a fifth of its speed). The
+//                     input is read twice (5 B of HBM traffic per element
+//                     instead of 3); in exchange neither kernel synchronizes
+//                     across CTAs.
 #pragma once
 
 #include "common.cuh"
@@ -280,10 +282,8 @@ constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
 // out[l * P + p] = e4m3(x(l, p) * s(group(p), l)), s = 448 / max(amax, 1e-12)
 // from the finished amax table; inv[g * L + l] = 1 / s (written by the first
 // tiles_l CTAs). Rows past offs[G-1] are not written. A consumer warp owns a
-// 32-row block of each tile; the group and the two amax words of its next
-// tile are loaded while it works on the current one, so the table's L2
-// latency stays off the per-tile path. `drop_load`: test hook, CTA 0 never
-// issues its first tile, so the bounded waits on it expire.
+// 32-row block of each tile. `drop_load`: test hook, CTA 0 never issues its
+// first tile, so the bounded waits on it expire.
 __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
     k_jagged_cast(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out, int64_t L,
                   int64_t P, const int32_t *__restrict__ offs, int G, const unsigned *__restrict__ amax,
@@ -297,8 +297,10 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
     if (!offsets_ok(offs, G, P))
         return;
     const int64_t end_all = offs[G - 1];
-    const int64_t tiles_p = (end_all + TP - 1) / TP, tiles_l = (L + TL - 1) / TL;
-    const int64_t total = tiles_p * tiles_l;
+    // tile t = (position tile t / tiles_l, line tile t % tiles_l); the host
+    // guarantees fewer than 2^31 tiles, so tile arithmetic is 32-bit
+    const uint32_t tiles_p = (uint32_t)((end_all + TP - 1) / TP), tiles_l = (uint32_t)((L + TL - 1) / TL);
+    const uint32_t total = tiles_p * tiles_l;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -312,10 +314,10 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
     __syncthreads();
 
     // inverse scales of every (group, line), empty groups included
-    for (int64_t lt = blockIdx.x; lt < tiles_l; lt += gridDim.x)
+    for (uint32_t lt = blockIdx.x; lt < tiles_l; lt += gridDim.x)
         for (int i = threadIdx.x; i < G * TL; i += blockDim.x) {
             const int g = i / TL;
-            const int64_t l = lt * TL + (i % TL);
+            const int64_t l = (int64_t)lt * TL + (i % TL);
             if (l < L)
                 inv[(int64_t)g * L + l] = fp8_inv(fp8_scale(__uint_as_float(__ldg(amax + (int64_t)g * L + l))));
         }
@@ -324,13 +326,13 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
         // ------------------------------------------------ producer warp
         if (lane == 0) {
             int it = 0;
-            for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            for (uint32_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
                 const int s = it % STAGES;
                 if (it >= STAGES && !mbar_wait(&sm.empty[s], ((uint32_t)(it / STAGES) & 1u) ^ 1u, wait_ns))
                     break;
                 if (drop_load && blockIdx.x == 0 && it == 0)
                     continue; // test hook: this tile never arrives
-                const int64_t pt = t / tiles_l, lt = t - pt * tiles_l;
+                const uint32_t pt = t / tiles_l, lt = t - pt * tiles_l;
                 mbar_arrive_expect_tx(&sm.full[s], IN_BYTES);
                 tma_load_2d(sm.in[s], &tm_in, &sm.full[s], (int)(lt * TL), (int)(pt * TP));
             }
@@ -344,36 +346,20 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
 
     // ---------------------------------------------------- consumer warps
     const int w = warp; // rows 32w .. 32w+31 of the tile
-    // group of the block's first row and the amax words of the lane's lines
-    struct Pre {
-        int g;
-        uint32_t a0, a1;
-    };
-    auto prefetch = [&](int64_t t) {
-        Pre pr;
-        const int64_t pt = t / tiles_l, lt = t - pt * tiles_l;
-        const int64_t p0 = pt * TP + 32 * w;
-        const int64_t l0 = lt * TL + 2 * lane;
-        pr.g = group_of(sm.offs, G, p0);
-        const unsigned *row = amax + (int64_t)pr.g * L;
-        pr.a0 = l0 < L ? __ldg(row + l0) : 0u;
-        pr.a1 = l0 + 1 < L ? __ldg(row + l0 + 1) : 0u;
-        return pr;
-    };
     bool prev_stored = true;
     int it = 0;
-    Pre cur = {0, 0u, 0u};
-    if ((int64_t)blockIdx.x < total)
-        cur = prefetch(blockIdx.x);
-    for (int64_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+    for (uint32_t t = blockIdx.x; t < total; t += gridDim.x, ++it) {
         const int s = it % STAGES;
         const int ob = it & 1;
-        const int64_t pt = t / tiles_l, lt = t - pt * tiles_l;
-        const int64_t p0 = pt * TP + 32 * w;          // this warp's first position
-        const int64_t l0 = lt * TL + 2 * lane;        // this lane's lines l0, l0+1
-        Pre nxt = cur;
-        if (t + gridDim.x < total)
-            nxt = prefetch(t + gridDim.x);
+        const uint32_t pt = t / tiles_l, lt = t - pt * tiles_l;
+        const int64_t p0 = (int64_t)pt * TP + 32 * w;   // this warp's first position
+        const int64_t l0 = (int64_t)lt * TL + 2 * lane; // this lane's lines l0, l0+1
+        // group of the block's first row and the amax words of the lane's
+        // lines, loaded before the wait so their latency overlaps it
+        const int g = group_of(sm.offs, G, p0);
+        const unsigned *arow = amax + (int64_t)g * L;
+        const uint32_t am0 = l0 < L ? __ldg(arow + l0) : 0u;
+        const uint32_t am1 = l0 + 1 < L ? __ldg(arow + l0 + 1) : 0u;
         bool ok = mbar_wait(&sm.full[s], (uint32_t)(it / STAGES) & 1u, wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok)
@@ -388,11 +374,10 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
         }
         release_slot_after(&sm.empty[s], dep);
 
-        const int g = cur.g;
         uint32_t q0[8], q1[8]; // lines l0, l0+1: 32 position bytes each
         if (p0 < end_all && (int64_t)sm.offs[g] >= p0 + 32) {
             // the block lies in one group
-            const float s0 = fp8_scale(__uint_as_float(cur.a0)), s1 = fp8_scale(__uint_as_float(cur.a1));
+            const float s0 = fp8_scale(__uint_as_float(am0)), s1 = fp8_scale(__uint_as_float(am1));
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t *r = v + 4 * j;
@@ -402,20 +387,26 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
                         (e4m3x2(__fmul_rn(bf16_hi(r[2]), s1), __fmul_rn(bf16_hi(r[3]), s1)) << 16);
             }
         } else {
-            // the block crosses group ends (or offs[G-1]): per-row group
+            // the block crosses group ends (or offs[G-1]): per-row group,
+            // the scales reloaded only where the group changes
             auto scale_of = [&](int grp, int64_t l) {
                 return l < L ? fp8_scale(__uint_as_float(__ldg(amax + (int64_t)grp * L + l))) : 0.0f;
             };
             int gg = g;
+            float s0 = fp8_scale(__uint_as_float(am0)), s1 = fp8_scale(__uint_as_float(am1));
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 uint32_t a0 = 0, a1 = 0;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int64_t row = p0 + 4 * j + k;
-                    while (gg + 1 < G && (int64_t)sm.offs[gg] <= row)
-                        ++gg;
-                    const float s0 = scale_of(gg, l0), s1 = scale_of(gg, l0 + 1);
+                    if (gg + 1 < G && (int64_t)sm.offs[gg] <= row) {
+                        do {
+                            ++gg;
+                        } while (gg + 1 < G && (int64_t)sm.offs[gg] <= row);
+                        s0 = scale_of(gg, l0);
+                        s1 = scale_of(gg, l0 + 1);
+                    }
                     const uint32_t x = v[4 * j + k];
                     a0 |= e4m3x2(__fmul_rn(bf16_lo(x), s0), 0.0f) << (8 * k);
                     a1 |= e4m3x2(__fmul_rn(bf16_hi(x), s1), 0.0f) << (8 * k);
@@ -424,11 +415,10 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
                 q1[j] = a1;
             }
         }
-        cur = nxt;
 
         // a tile wholly below offs[G-1] leaves through the staging tile and a
         // TMA store; the tile holding offs[G-1] is written directly
-        const bool full_tile = pt * TP + TP <= end_all;
+        const bool full_tile = (int64_t)pt * TP + TP <= end_all;
         // staging buffer ob was read by the store of tile it-2; when tile
         // it-1 issued no store, that one may be the newest group
         if (threadIdx.x == 0) {

@@ -183,6 +183,8 @@ int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_
     pl->wpc = (int)wpc;
     pl->grid_a = (int)((chunks * wpc * 32 + jag::amx::THREADS - 1) / jag::amx::THREADS);
     const int64_t tiles = (P + jag::cst::TP - 1) / jag::cst::TP * ((L + jag::cst::TL - 1) / jag::cst::TL);
+    if (tiles >= (int64_t(1) << 31))
+        return MXQ_OK; // the cast pass indexes tiles with 32 bits
     pl->grid_c = (int)std::min<int64_t>(tiles, (int64_t)di->sms * di->cst_per_sm);
     pl->ws = twopass_workspace(L, G);
     return MXQ_OK;
