@@ -577,7 +577,7 @@ def main():
                               "mx scales to blocked grouped (65536,224) G=64"],
                       "step_bytes": step_bytes, "parallelism": f"replicas x{world}",
                       "l2": "no flush: inputs larger than L2 (each step moves >12 GB)"},
-           "roofline": roofline, "per_op": per_op, "gpu_launches": len(wl.ops) * args.steps,
+           "roofline": roofline, "per_op": per_op, "gpu_launches": sum(KERNEL_NAMES[n].count("+") + 1 for n, _, _ in wl.ops) * args.steps,
            "clocks": clocks}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
