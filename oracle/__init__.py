@@ -49,6 +49,10 @@ def lib():
             "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
+            "oracle_blocked_grouped_k_cols_bound": (_i64, [_i64, _i32]),
+            "oracle_mx_scales_to_blocked_grouped_k": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
+            "oracle_mx_quant_rowwise_blocked_grouped": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _i32p, _i32,
+                                                                       _u8p, _u8p, _i64, _i32p]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -174,6 +178,43 @@ def mx_quant_rowwise(x, mode):
     sc = np.zeros((rows, cols // 32), dtype=np.uint8)
     _check(lib().oracle_mx_quant_rowwise(_p(w, _u16p), rows, cols, mode, _p(out, _u8p), _p(sc, _u8p)))
     return out, sc
+
+
+def blocked_grouped_k_cols_bound(cols, groups):
+    return lib().oracle_blocked_grouped_k_cols_bound(int(cols), int(groups))
+
+
+def mx_scales_to_blocked_grouped_k(scales, offs, capacity_cols=None):
+    """Groups along K (scale columns): returns (flat blocked buffer of
+    128*ceil(rows/128) x capacity_cols bytes, padded group column starts)."""
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, cols = s.shape
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    if capacity_cols is None:
+        capacity_cols = blocked_grouped_k_cols_bound(cols, len(o))
+    rows_p = (rows + 127) // 128 * 128
+    out = np.full((rows_p * capacity_cols,), 0xAB, dtype=np.uint8)
+    starts = np.zeros((len(o),), dtype=np.int32)
+    _check(lib().oracle_mx_scales_to_blocked_grouped_k(_p(s, _u8p), rows, cols, _p(o, _i32p), len(o),
+                                                       _p(out, _u8p), capacity_cols, _p(starts, _i32p)))
+    return out, starts
+
+
+def mx_quant_rowwise_blocked_grouped(words, rows, cols, mode, offs, capacity_rows=None):
+    """MX rowwise quantization with the scales in the per-group blocked layout:
+    returns (e4m3 (rows, cols), flat blocked scales, padded group row starts)."""
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    if capacity_rows is None:
+        capacity_rows = blocked_grouped_rows_bound(rows, len(o))
+    cols_p = (cols // 32 + 3) // 4 * 4
+    out = np.zeros((rows, cols), dtype=np.uint8)
+    sb = np.full((capacity_rows * cols_p,), 0xAB, dtype=np.uint8)
+    starts = np.zeros((len(o),), dtype=np.int32)
+    _check(lib().oracle_mx_quant_rowwise_blocked_grouped(_p(w, _u16p), rows, cols, mode, _p(o, _i32p), len(o),
+                                                         _p(out, _u8p), _p(sb, _u8p), capacity_rows,
+                                                         _p(starts, _i32p)))
+    return out, sb, starts
 
 
 def mx_scales_to_blocked_grouped(scales, offs, capacity_rows=None):

@@ -39,6 +39,13 @@
  *      (r % 32) * 16 + (r / 32) * 4 + c; tiles are ordered row-tile major.
  *   R9 grouped blocked layout: each group's rows are padded to a multiple of
  *      128 on their own; groups are stacked in order; the rest is zero.
+ *   R12 groups along K (#3504's stack, #3505): each group's scale columns are
+ *      padded to a multiple of 4 on their own and placed side by side in one
+ *      matrix of 128-padded rows and capacity_cols columns, which is stored
+ *      in the blocked layout of R8; the rest is zero (the pages' byte count,
+ *      R*C read and R*(C + 4G) written, fits this single output matrix).
+ *   R13 MX rowwise quantization with blocked scales = the rowwise op followed
+ *      by the row-group conversion of R9 applied to its scales.
  *
  * Floating point: every step the definitions place in fp32 is done in fp32
  * (C float arithmetic, round-to-nearest, no contraction, no flush to zero);
@@ -47,6 +54,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "oracle.h"
@@ -408,3 +416,73 @@ int oracle_mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Groups along K (ao PR 3504's stack, #3505 "integrate new cuda kernel */
+/* for blocked layout for groups along K"). Group g is the scale-column */
+/* range [offs[g-1], offs[g]). Reading taken where the pages are        */
+/* silent (their byte count, R*C in and R*(C + 4G) out, fits one output */
+/* matrix): each group's columns are padded to a multiple of 4 on their */
+/* own and placed side by side from column Q_g = sum_{h<g}              */
+/* 4*ceil(size_h/4); rows are padded to a multiple of 128; the whole    */
+/* (128*ceil(rows/128), capacity_cols) matrix is stored in the 128x4    */
+/* blocked layout, every byte not taken by a scale being zero.          */
+/* ------------------------------------------------------------------ */
+int64_t oracle_blocked_grouped_k_cols_bound(int64_t cols, int32_t groups)
+{
+    /* sum_g 4*ceil(s_g/4) is a multiple of 4 and at most cols + 3*groups */
+    return 4 * ((cols + 3 * (int64_t)groups) / 4);
+}
+
+int oracle_mx_scales_to_blocked_grouped_k(const uint8_t *scales, int64_t rows, int64_t cols,
+                                          const int32_t *offs, int32_t groups,
+                                          uint8_t *out, int64_t capacity_cols,
+                                          int32_t *group_col_starts)
+{
+    int64_t rows_p, start = 0, base = 0;
+    if (rows < 0 || cols < 0 || groups <= 0 || capacity_cols < 0)
+        return ORACLE_ERR_ARG;
+    if (capacity_cols % 4 || capacity_cols < oracle_blocked_grouped_k_cols_bound(cols, groups))
+        return ORACLE_ERR_ARG;
+    if (!offsets_valid(offs, groups, cols))
+        return ORACLE_ERR_OFFSETS;
+    rows_p = (rows + 127) / 128 * 128;
+    memset(out, 0, (size_t)(rows_p * capacity_cols));
+    for (int32_t g = 0; g < groups; ++g) {
+        int64_t end = offs[g], size = end - start;
+        if (group_col_starts)
+            group_col_starts[g] = (int32_t)base;
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t c = 0; c < size; ++c)
+                out[oracle_blocked_offset(r, base + c, capacity_cols)] = scales[r * cols + start + c];
+        base += (size + 3) / 4 * 4;
+        start = end;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* MX rowwise quantization whose E8M0 scales go straight to the         */
+/* per-group blocked layout: by definition the rowwise op (a5) followed */
+/* by the row-group conversion (a6) of its scales.                     */
+/* ------------------------------------------------------------------ */
+int oracle_mx_quant_rowwise_blocked_grouped(const uint16_t *in, int64_t rows, int64_t cols, int mode,
+                                            const int32_t *offs, int32_t groups,
+                                            uint8_t *out, uint8_t *scales_blocked,
+                                            int64_t capacity_rows, int32_t *group_row_starts)
+{
+    uint8_t *scales;
+    int rc;
+    if (rows < 0 || cols < 0 || cols % 32)
+        return ORACLE_ERR_ARG;
+    scales = (uint8_t *)malloc((size_t)(rows * (cols / 32)) + 1);
+    if (!scales)
+        return ORACLE_ERR_ARG;
+    rc = oracle_mx_quant_rowwise(in, rows, cols, mode, out, scales);
+    if (rc == 0)
+        rc = oracle_mx_scales_to_blocked_grouped(scales, rows, cols / 32, offs, groups, scales_blocked,
+                                                 capacity_rows, group_row_starts);
+    free(scales);
+    return rc;
+}
+

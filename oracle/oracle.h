@@ -50,6 +50,15 @@ int oracle_mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int
                                         const int32_t *offs, int32_t groups,
                                         uint8_t *out, int64_t capacity_rows,
                                         int32_t *group_row_starts);
+int64_t oracle_blocked_grouped_k_cols_bound(int64_t cols, int32_t groups);
+int oracle_mx_scales_to_blocked_grouped_k(const uint8_t *scales, int64_t rows, int64_t cols,
+                                          const int32_t *offs, int32_t groups,
+                                          uint8_t *out, int64_t capacity_cols,
+                                          int32_t *group_col_starts);
+int oracle_mx_quant_rowwise_blocked_grouped(const uint16_t *in, int64_t rows, int64_t cols, int mode,
+                                            const int32_t *offs, int32_t groups,
+                                            uint8_t *out, uint8_t *scales_blocked,
+                                            int64_t capacity_rows, int32_t *group_row_starts);
 
 #ifdef __cplusplus
 }

@@ -312,6 +312,101 @@ def test_grouped_blocked_bound_is_tight(oracle):
         oracle.mx_scales_to_blocked_grouped(np.zeros((10, 4), np.uint8), [10], capacity_rows=0)
 
 
+def test_grouped_blocked_k_hand_examples(oracle):
+    n = 0
+    for ln in _lines("blocked_layout.txt"):
+        if ln.startswith("kgroups"):
+            lhs, rest = ln[len("kgroups"):].split("->")
+            R, C, sizes, cap = lhs.split()
+            R, C, cap = int(R), int(C), int(cap)
+            offs = np.cumsum([int(t) for t in sizes.split(",")]).astype(np.int32)
+            starts_s, places = rest.split("|")
+            s = (np.arange(R * C) % 250 + 1).astype(np.uint8).reshape(R, C)  # nonzero, s[r][c] = 6r+c+1 here
+            assert oracle.blocked_grouped_k_cols_bound(C, len(offs)) == cap, ln
+            out, starts = oracle.mx_scales_to_blocked_grouped_k(s, offs, cap)
+            assert list(starts) == [int(t) for t in starts_s.split(",")], ln
+            for p in places.split():
+                r, c, off = (int(t) for t in p.split(":"))
+                assert out[off] == s[r, c], (ln, p)
+            assert np.count_nonzero(out) == R * C, ln  # everything else is zero
+            n += 1
+    assert n == 2
+
+
+def _torch_grouped_blocked_k(s, offs, capacity):
+    """Independent construction: pad each group's columns, place them side by
+    side in a zero (R', capacity) matrix, then the library permutation."""
+    R, C = s.shape
+    Rp = (R + 127) // 128 * 128
+    full = torch.zeros((Rp, capacity), dtype=torch.uint8)
+    starts, base, start = [], 0, 0
+    for end in offs:
+        w = end - start
+        starts.append(base)
+        full[:R, base:base + w] = torch.from_numpy(s[:, start:end])
+        base += (w + 3) // 4 * 4
+        start = end
+    return _torch_to_blocked(full).numpy(), np.array(starts, dtype=np.int32)
+
+
+@pytest.mark.parametrize("rows,cols,sizes", [
+    (2, 6, [1, 5]),
+    (130, 13, [0, 3, 0, 10]),
+    (128, 224, [50, 0, 100, 74]),
+    (300, 33, [1, 2, 3, 4, 5, 6, 7, 5]),
+    (64, 40, [30]),                # columns past the last offset are ignored
+])
+def test_grouped_blocked_k_vs_torch(oracle, rows, cols, sizes):
+    rng = np.random.default_rng(rows * 7 + cols)
+    s = rng.integers(1, 255, size=(rows, cols), dtype=np.uint8)
+    offs = np.cumsum(sizes).astype(np.int32)
+    cap = oracle.blocked_grouped_k_cols_bound(cols, len(offs))
+    got, starts = oracle.mx_scales_to_blocked_grouped_k(s, offs, cap)
+    ref, ref_starts = _torch_grouped_blocked_k(s, offs, cap)
+    assert np.array_equal(starts, ref_starts)
+    assert np.array_equal(got, ref)
+
+
+def test_grouped_blocked_k_reduces_to_row_groups(oracle):
+    """One group spanning every column is the plain blocked layout, i.e. the
+    row-group conversion with one group; groups whose sizes are multiples of 4
+    leave no gaps, so the result is that plain layout of the matrix widened by
+    zero columns to the capacity."""
+    rng = np.random.default_rng(5)
+    s = rng.integers(0, 255, size=(200, 22), dtype=np.uint8)
+    got, _ = oracle.mx_scales_to_blocked_grouped_k(s, [22])
+    want, _ = oracle.mx_scales_to_blocked_grouped(s, [200])
+    assert np.array_equal(got, want)
+    s2 = rng.integers(0, 255, size=(150, 24), dtype=np.uint8)
+    offs = [8, 8, 20, 24]
+    cap = oracle.blocked_grouped_k_cols_bound(24, 4)
+    got2, _ = oracle.mx_scales_to_blocked_grouped_k(s2, offs, cap)
+    wide = np.zeros((150, cap), dtype=np.uint8)
+    wide[:, :24] = s2
+    want2, _ = oracle.mx_scales_to_blocked_grouped(wide, [150])
+    assert np.array_equal(got2, want2)
+
+
+def test_grouped_blocked_k_bound_is_tight(oracle):
+    # G one-column groups need 4 columns each; below the bound is refused
+    for G in (1, 5, 17):
+        assert oracle.blocked_grouped_k_cols_bound(G, G) == 4 * G
+    with pytest.raises(oracle.OracleError):
+        oracle.mx_scales_to_blocked_grouped_k(np.zeros((4, 6), np.uint8), [1, 6], capacity_cols=8)
+
+
+def test_rowwise_blocked_is_rowwise_then_conversion(oracle):
+    rng = np.random.default_rng(3)
+    x = torch.from_numpy(rng.standard_normal((300, 96)).astype(np.float32)).to(torch.bfloat16)
+    w = x.view(torch.int16).numpy().view(np.uint16)
+    offs = np.array([0, 100, 100, 290], dtype=np.int32)
+    for mode in (0, 1):
+        q, sb, starts = oracle.mx_quant_rowwise_blocked_grouped(w.reshape(-1), 300, 96, mode, offs)
+        q2, sc = oracle.mx_quant_rowwise(w, mode)
+        sb2, starts2 = oracle.mx_scales_to_blocked_grouped(sc, offs)
+        assert np.array_equal(q, q2) and np.array_equal(sb, sb2) and np.array_equal(starts, starts2)
+
+
 # --------------------------------------------------------------------------
 # ops: brute force, cross-op identities, invariants
 # --------------------------------------------------------------------------
