@@ -373,6 +373,27 @@ def per_shape_sweep(wl, reps):
                 lambda s=s, o=o, cap=cap, out=out, st=st: mxq.mx_scales_to_blocked_grouped(
                     s, o, capacity_rows=cap, out=out, group_row_starts=st),
                 R * C + cap * C)
+    # groups along K: the pages' sweep shapes, G=8 along the columns, capacity C + 4G
+    for R in (8192, 5120, 7168, 2048):
+        for C in (512, 1024, 2048, 4096, 32768):
+            s, o = synth.scale_sweep_k(R, C, device="cpu")
+            s, o = s.to(dev), o.to(dev)
+            out = torch.empty(R * (C + 32), dtype=torch.uint8, device=dev)
+            st = torch.empty(8, dtype=torch.int32, device=dev)
+            run("blocked_grouped_k", f"({R},{C}) G=8",
+                lambda s=s, o=o, out=out, st=st: mxq.mx_scales_to_blocked_grouped_k(
+                    s, o, capacity_cols=C + 32, out=out, group_col_starts=st),
+                R * C + R * (C + 32))
+    # MX rowwise quantization writing blocked scales directly (a5 + a6 fused)
+    tc = 7168 // 128
+    for mode in ("floor", "rceil"):
+        sbuf = torch.empty(wl.cap * tc * 4, dtype=torch.uint8, device=dev)
+        st = torch.empty(64, dtype=torch.int32, device=dev)
+        run("mx_rowwise_blocked", f"(65536,7168) G=64 {mode}",
+            lambda mode=mode, sbuf=sbuf, st=st: mxq.mx_quant_rowwise_blocked_grouped(
+                wl.tok, wl.offs64, mode, capacity_rows=wl.cap, out=wl.o["tok_q"], scales=sbuf,
+                group_row_starts=st),
+            65536 * 7168 * 3 + wl.cap * tc * 4)
     del flush
     return rows
 

@@ -191,6 +191,57 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
 int64_t mx_blocked_grouped_rows_bound(int64_t rows, int32_t num_groups);
 
 /* ------------------------------------------------------------------------ *
+ * mx_scales_to_blocked_grouped_k - #3504's stack, #3505 "integrate new cuda
+ * kernel for blocked layout for groups along K": the same 128x4 blocked
+ * layout with the groups along the COLUMNS of the scale matrix (the K
+ * dimension of the quantized operand, in 32-element block units).
+ *   scales      u8 (rows, cols) row-major (device).
+ *   offs        num_groups int32 ends along cols (device).
+ *   out         128*ceil(rows/128) x out_cols_capacity bytes, the whole
+ *               padded matrix in the blocked layout: group g's columns are
+ *               padded to a multiple of 4 on their own and start at output
+ *               column out_group_col_starts[g] = 4 * sum_{h<g} ceil(size_h/4);
+ *               pad rows, pad columns and columns past the last group are 0.
+ *               16-byte aligned.
+ *   out_cols_capacity  multiple of 4, at least
+ *               mx_blocked_grouped_k_cols_bound(cols, num_groups), else
+ *               MXQ_ERR_SHAPE. num_groups <= 4096, else MXQ_ERR_UNSUPPORTED.
+ *   out_group_col_starts  optional int32 (num_groups), may be NULL.
+ * Reading where the pages are silent: the output is one matrix (their byte
+ * count, R*C read and R*(C + 4G) written, fits it), so group g's scales form
+ * a column slice of a blocked matrix with a row-tile stride of
+ * out_cols_capacity/4 tiles.
+ * ------------------------------------------------------------------------ */
+int mx_scales_to_blocked_grouped_k(const uint8_t *scales, int64_t rows, int64_t cols,
+                                   const int32_t *offs, int32_t num_groups,
+                                   uint8_t *out, int64_t out_cols_capacity,
+                                   int32_t *out_group_col_starts,
+                                   cudaStream_t stream);
+
+/* Smallest capacity valid for any offsets: 4 * floor((cols + 3*G) / 4). */
+int64_t mx_blocked_grouped_k_cols_bound(int64_t cols, int32_t num_groups);
+
+/* ------------------------------------------------------------------------ *
+ * mx_quant_rowwise_blocked_grouped - (a5) followed by (a6) in one launch:
+ * MXFP8 1x32 rowwise quantization of a row-major (rows, cols) bf16 matrix
+ * whose E8M0 scales are written straight into the per-group blocked layout
+ * of mx_scales_to_blocked_grouped (groups = row ranges), never as a plain
+ * (rows, cols/32) matrix.
+ *   cols % 32 == 0; in, out 16-byte aligned; scales_blocked 4-byte aligned.
+ *   out         e4m3 (rows, cols) row-major, every row (as mx_quant_rowwise).
+ *   scales_blocked  out_rows_capacity x 4*ceil(cols/128) bytes, exactly the
+ *               bytes mx_scales_to_blocked_grouped writes for the scales of
+ *               mx_quant_rowwise; rows past offs[num_groups-1] get no scale.
+ *   out_rows_capacity, out_group_row_starts, num_groups as for
+ *   mx_scales_to_blocked_grouped.
+ * ------------------------------------------------------------------------ */
+int mx_quant_rowwise_blocked_grouped(const void *in, int64_t rows, int64_t cols,
+                                     int32_t mode, const int32_t *offs, int32_t num_groups,
+                                     void *out, uint8_t *scales_blocked,
+                                     int64_t out_rows_capacity, int32_t *out_group_row_starts,
+                                     cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * fp8_quant_jagged_colwise_noalloc - the source pages have no counterpart to
  * this entry point; it exists for callers that cannot allocate device memory
  * (a plugin inside a framework that owns all device memory and passes no

@@ -39,6 +39,10 @@ SIGNATURES = {
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
     "mx_blocked_grouped_rows_bound": (_i64, [_i64, _i32]),
+    "mx_scales_to_blocked_grouped_k": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
+    "mx_blocked_grouped_k_cols_bound": (_i64, [_i64, _i32]),
+    "mx_quant_rowwise_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _i64, _vp,
+                                                        _vp]),
     "mxq_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(_i32)]),
     "mxq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mxq_version": (ctypes.c_int, []),
@@ -245,6 +249,62 @@ def mx_scales_to_blocked_grouped(scales, offs, *, capacity_rows=None, out=None, 
                                             _ptr(group_row_starts), _stream(dev))
     _check("mx_scales_to_blocked_grouped", rc)
     return out, group_row_starts
+
+
+def blocked_grouped_k_cols_bound(cols, num_groups):
+    return lib().mx_blocked_grouped_k_cols_bound(cols, num_groups)
+
+
+def mx_scales_to_blocked_grouped_k(scales, offs, *, capacity_cols=None, out=None, group_col_starts=None,
+                                   with_starts=True):
+    """128x4 blocked layout of a (rows, cols) uint8 scale matrix with groups
+    along its columns (K). Returns (out flat uint8 of 128*ceil(rows/128) *
+    capacity_cols bytes, padded group column starts int32 (G) or None)."""
+    _cuda(scales, "scales")
+    if scales.dim() != 2 or not scales.is_contiguous() or scales.element_size() != 1:
+        raise TypeError("scales must be a contiguous 2-D 1-byte tensor")
+    dev = scales.device
+    _offsets(offs, dev)
+    rows, cols = scales.shape
+    G = offs.numel()
+    if capacity_cols is None:
+        capacity_cols = blocked_grouped_k_cols_bound(cols, G)
+    rows_p = (rows + 127) // 128 * 128
+    if out is None:
+        out = torch.empty(rows_p * capacity_cols, dtype=torch.uint8, device=dev)
+    if group_col_starts is None and with_starts:
+        group_col_starts = torch.empty(G, dtype=torch.int32, device=dev)
+    rc = lib().mx_scales_to_blocked_grouped_k(_ptr(scales), rows, cols, _ptr(offs), G, _ptr(out), capacity_cols,
+                                              _ptr(group_col_starts), _stream(dev))
+    _check("mx_scales_to_blocked_grouped_k", rc)
+    return out, group_col_starts
+
+
+def mx_quant_rowwise_blocked_grouped(x, offs, mode="floor", *, capacity_rows=None, out=None, scales=None,
+                                     group_row_starts=None, with_starts=True):
+    """MXFP8 1x32 rowwise quantization of x (rows, cols) with its E8M0 scales
+    written straight into the per-group (row groups) blocked layout. Returns
+    (q (rows, cols) float8_e4m3fn, blocked scales flat uint8 of capacity_rows *
+    4*ceil(cols/128) bytes, padded group row starts int32 (G) or None)."""
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous 2-D bfloat16 tensor")
+    dev = x.device
+    _offsets(offs, dev)
+    rows, cols = x.shape
+    G = offs.numel()
+    if capacity_rows is None:
+        capacity_rows = blocked_grouped_rows_bound(rows, G)
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(capacity_rows * ((cols + 127) // 128) * 4, dtype=torch.uint8, device=dev)
+    if group_row_starts is None and with_starts:
+        group_row_starts = torch.empty(G, dtype=torch.int32, device=dev)
+    rc = lib().mx_quant_rowwise_blocked_grouped(_ptr(x), rows, cols, _mode(mode), _ptr(offs), G, _ptr(out),
+                                                _ptr(scales), capacity_rows, _ptr(group_row_starts), _stream(dev))
+    _check("mx_quant_rowwise_blocked_grouped", rc)
+    return out.view(torch.float8_e4m3fn), scales, group_row_starts
 
 
 # ---------------------------------------------------------------- status

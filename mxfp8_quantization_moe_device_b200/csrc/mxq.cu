@@ -74,6 +74,7 @@ struct DevInfo {
     int cst_per_sm = 0;   // resident CTAs of the jagged cast pass
     int rb_per_sm = 0;    // resident CTAs of the 1x128 kernel
     int mx32_per_sm = 0;  // resident CTAs of the 1x32 kernel
+    int mxb_per_sm = 0;   // resident CTAs of the 1x32 kernel with blocked scales
 };
 
 DevInfo g_dev[128];
@@ -101,7 +102,8 @@ int device_info(const DevInfo **out)
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.cst_per_sm, k_jagged_cast, jag::cst::THREADS,
                                                           jag::cst::SMEM_BYTES) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.rb_per_sm, k_fp8_1x128, RB_THREADS, 0) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mx32_per_sm, k_mx_1x32, RB_THREADS, 0) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mx32_per_sm, k_mx_1x32, RB_THREADS, 0) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mxb_per_sm, k_mx_1x32_blocked, 256, 0) != cudaSuccess)
             return MXQ_ERR_CUDA;
         di.ready = true;
     }
@@ -406,12 +408,85 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
     const int64_t gx = std::max<int64_t>((tiles_c + blk::TILES - 1) / blk::TILES, 1);
     // enough CTAs to fill the GPU; each walks tile rows with stride gy
     const int64_t tile_rows = std::max<int64_t>(out_rows_capacity / 128, 1);
-    const int64_t want = std::max<int64_t>((int64_t)di->sms * 4 / gx, 1);
+    const int64_t want = std::max<int64_t>((int64_t)di->sms * 8 / gx, 1);
     const int64_t gy = std::min<int64_t>(tile_rows, std::min<int64_t>(want, 65535));
     const int words_ok = (aligned(scales, 4) && cols % 4 == 0) ? 1 : 0;
-    return launch(k_blocked_grouped, dim3((unsigned)gx, (unsigned)gy), dim3(blk::THREADS), 0, stream, false, scales,
+    return launch(k_blocked_grouped, dim3((unsigned)gx, (unsigned)gy), dim3(blk::THREADS),
+                  (size_t)num_groups * sizeof(int), stream, false, scales,
                   rows, cols, offs, (int)num_groups, out, out_group_row_starts, words_ok,
                   out_rows_capacity / 128);
+}
+
+int64_t mx_blocked_grouped_k_cols_bound(int64_t cols, int32_t num_groups)
+{
+    if (cols < 0 || num_groups < 0)
+        return -1;
+    return 4 * ((cols + 3 * (int64_t)num_groups) / 4);
+}
+
+int mx_scales_to_blocked_grouped_k(const uint8_t *scales, int64_t rows, int64_t cols, const int32_t *offs,
+                                   int32_t num_groups, uint8_t *out, int64_t out_cols_capacity,
+                                   int32_t *out_group_col_starts, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0 || num_groups < 1 || out_cols_capacity < 0 || out_cols_capacity % 4)
+        return MXQ_ERR_SHAPE;
+    const int64_t rows_p = (rows + 127) / 128 * 128;
+    if (!offs || (rows * cols > 0 && !scales) || (rows_p * out_cols_capacity > 0 && !out))
+        return MXQ_ERR_NULL;
+    if (out_cols_capacity < mx_blocked_grouped_k_cols_bound(cols, num_groups))
+        return MXQ_ERR_SHAPE;
+    if (num_groups > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if (out && !aligned(out, 16))
+        return MXQ_ERR_ALIGN;
+    if ((rows_p == 0 || out_cols_capacity == 0) && !out_group_col_starts)
+        return MXQ_OK;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t tiles_c = out_cols_capacity / 4;
+    const int64_t gx = std::max<int64_t>((tiles_c + blk::TILES - 1) / blk::TILES, 1);
+    const int64_t tile_rows = std::max<int64_t>(rows_p / 128, 1);
+    const int64_t want = std::max<int64_t>((int64_t)di->sms * 8 / gx, 1);
+    const int64_t gy = std::min<int64_t>(tile_rows, std::min<int64_t>(want, 65535));
+    if (gx > 0x7fffffff)
+        return MXQ_ERR_UNSUPPORTED;
+    const int words_ok = (aligned(scales, 4) && cols % 4 == 0) ? 1 : 0;
+    return launch(k_blocked_grouped_k, dim3((unsigned)gx, (unsigned)gy), dim3(blk::THREADS),
+                  (size_t)num_groups * sizeof(int), stream, false, scales,
+                  rows, cols, offs, (int)num_groups, out, out_group_col_starts, words_ok, out_cols_capacity);
+}
+
+int mx_quant_rowwise_blocked_grouped(const void *in, int64_t rows, int64_t cols, int32_t mode, const int32_t *offs,
+                                     int32_t num_groups, void *out, uint8_t *scales_blocked,
+                                     int64_t out_rows_capacity, int32_t *out_group_row_starts, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0 || cols % 32 || num_groups < 1 || out_rows_capacity < 0 || out_rows_capacity % 128)
+        return MXQ_ERR_SHAPE;
+    if (mode != MXQ_E8M0_FLOOR && mode != MXQ_E8M0_RCEIL)
+        return MXQ_ERR_UNSUPPORTED;
+    const int64_t tcols = (cols + 127) / 128;
+    if (!offs || (rows * cols > 0 && (!in || !out)) || (out_rows_capacity * tcols > 0 && !scales_blocked))
+        return MXQ_ERR_NULL;
+    if (out_rows_capacity < mx_blocked_grouped_rows_bound(rows, num_groups))
+        return MXQ_ERR_SHAPE;
+    if (num_groups > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if ((in && !aligned(in, 16)) || (out && !aligned(out, 16)) || (scales_blocked && !aligned(scales_blocked, 4)))
+        return MXQ_ERR_ALIGN;
+    if (rows * cols == 0 && out_rows_capacity * tcols == 0 && !out_group_row_starts)
+        return MXQ_OK;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t warps = std::max<int64_t>(rows, out_rows_capacity);
+    const int64_t grid = std::max<int64_t>(std::min<int64_t>((warps + 7) / 8, (int64_t)di->sms * di->mxb_per_sm), 1);
+    return launch(k_mx_1x32_blocked, dim3((unsigned)grid), dim3(256), (size_t)num_groups * 2 * sizeof(int), stream,
+                  false,
+                  static_cast<const uint4 *>(in), rows, cols, offs, (int)num_groups, static_cast<uint2 *>(out),
+                  reinterpret_cast<uint32_t *>(scales_blocked), out_group_row_starts, out_rows_capacity, (int)mode);
 }
 
 } // extern "C"

@@ -145,6 +145,13 @@ def mx_act(device="cpu", rows=65536, cols=7168, groups=64, seeds=(7, 8)):
     return x, offs
 
 
+def scale_sweep_k(rows, cols, device="cpu", groups=8, seeds=(9, 11)):
+    """The scale sweep with its G groups along the columns (K) instead."""
+    s = uniform_u8((rows, cols), 0, 254, seeds[0], device)
+    offs = dirichlet_offsets(cols, groups, 1.0, seeds[1])
+    return s, offs
+
+
 def scale_sweep(rows, cols, device="cpu", groups=8, seeds=(9, 10)):
     s = uniform_u8((rows, cols), 0, 254, seeds[0], device)
     offs = dirichlet_offsets(rows, groups, 1.0, seeds[1])

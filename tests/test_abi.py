@@ -52,6 +52,8 @@ def test_pure_host_functions(lib):
     assert lib.mxq_status_string(6) == b"malformed group offsets"
     assert lib.mx_blocked_grouped_rows_bound(135, 2) == 384
     assert lib.mx_blocked_grouped_rows_bound(5, 5) == 640
+    assert lib.mx_blocked_grouped_k_cols_bound(6, 2) == 12
+    assert lib.mx_blocked_grouped_k_cols_bound(224, 8) == 248
     # jagged workspace: only the contiguous-line layout needs one
     ws = lib.fp8_quant_jagged_workspace_bytes(65536, 4096, 4096, 1, 16, 1)
     assert ws >= 16 * 4096 * 4  # the fp32 (group, column) amax table
@@ -84,6 +86,23 @@ def test_host_checks_return_before_any_cuda_call(lib):
     assert lib.fp8_quant_blockwise(odd, 128, 128, 1, 128, fake, fake, null) == binding.ERR_ALIGN
     assert lib.mx_quant_3d_colwise(fake, 1, 64, 60, 0, fake, fake, null) == binding.ERR_ALIGN
     assert lib.mx_scales_to_blocked_grouped(fake, 4, 4, fake, 1, odd, 128, null, null) == binding.ERR_ALIGN
+    # groups along K and the fused rowwise op
+    assert lib.mx_scales_to_blocked_grouped_k(fake, 4, 6, null, 1, fake, 12, null, null) == binding.ERR_NULL
+    assert lib.mx_scales_to_blocked_grouped_k(fake, 4, 6, fake, 2, fake, 8, null, null) == binding.ERR_SHAPE
+    assert lib.mx_scales_to_blocked_grouped_k(fake, 4, 6, fake, 2, fake, 14, null, null) == binding.ERR_SHAPE
+    assert lib.mx_scales_to_blocked_grouped_k(fake, 4, 6, fake, 2, odd, 12, null, null) == binding.ERR_ALIGN
+    assert lib.mx_scales_to_blocked_grouped_k(fake, 4, 6, fake, 5000, fake, 20004, null, null) == \
+        binding.ERR_UNSUPPORTED
+    assert lib.mx_quant_rowwise_blocked_grouped(fake, 4, 48, 0, fake, 1, fake, fake, 128, null, null) == \
+        binding.ERR_SHAPE
+    assert lib.mx_quant_rowwise_blocked_grouped(fake, 4, 64, 0, fake, 2, fake, fake, 128, null, null) == \
+        binding.ERR_SHAPE  # capacity below the bound for 2 groups
+    assert lib.mx_quant_rowwise_blocked_grouped(fake, 4, 64, 3, fake, 1, fake, fake, 128, null, null) == \
+        binding.ERR_UNSUPPORTED
+    assert lib.mx_quant_rowwise_blocked_grouped(odd, 4, 64, 0, fake, 1, fake, fake, 128, null, null) == \
+        binding.ERR_ALIGN
+    assert lib.mx_quant_rowwise_blocked_grouped(fake, 4, 64, 0, null, 1, fake, fake, 128, null, null) == \
+        binding.ERR_NULL
 
 
 def test_binding_refuses_cpu_tensors():

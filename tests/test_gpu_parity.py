@@ -459,6 +459,102 @@ def test_blocked_grouped_config_shapes(R, C):
     assert np.array_equal(starts.cpu().numpy(), ref_starts)
 
 
+BLOCKED_K = [
+    (2, 6, [1, 5]),
+    (130, 13, [0, 3, 0, 10]),            # byte-load path (cols % 4 != 0), empty groups
+    (128, 224, [50, 0, 100, 74]),
+    (300, 33, [1, 2, 3, 4, 5, 6, 7, 5]),
+    (64, 40, [30]),                      # columns past the last group
+    (1000, 600, [131, 1, 200, 268]),     # several 32-tile chunks per row tile
+    (257, 4, [4]),
+]
+
+
+@pytest.mark.parametrize("rows,cols,sizes", BLOCKED_K)
+def test_blocked_grouped_k_vs_oracle(rows, cols, sizes):
+    s = synth.uniform_u8((rows, cols), 0, 254, seed=rows * 3 + cols)
+    offs = torch.tensor(np.cumsum(sizes), dtype=torch.int32)
+    ref, ref_starts = oracle.mx_scales_to_blocked_grouped_k(s.numpy(), offs.numpy())
+    cap = mxq.blocked_grouped_k_cols_bound(cols, len(sizes))
+    big, out = guarded(ref.size)
+    bigs, starts = guarded(len(sizes), torch.int32)
+    mxq.mx_scales_to_blocked_grouped_k(s.to(DEV), offs.to(DEV), capacity_cols=cap, out=out,
+                                       group_col_starts=starts)
+    assert status_ok()
+    assert np.array_equal(u8(out), ref)
+    assert np.array_equal(starts.cpu().numpy(), ref_starts)
+    assert margins_intact(big) and margins_intact(bigs, torch.int32)
+
+
+@pytest.mark.parametrize("R,C", [(8192, 512), (2048, 32768), (5120, 4096)])
+def test_blocked_grouped_k_sweep_shapes(R, C):
+    """The pages' scale-sweep shapes with G=8 Dirichlet(1.0) groups along K,
+    capacity C + 4G (their byte count)."""
+    s, offs = synth.scale_sweep_k(R, C)
+    ref, ref_starts = oracle.mx_scales_to_blocked_grouped_k(s.numpy(), offs.numpy(), C + 32)
+    o, starts = mxq.mx_scales_to_blocked_grouped_k(s.to(DEV), offs.to(DEV), capacity_cols=C + 32)
+    assert status_ok()
+    assert np.array_equal(o.cpu().numpy(), ref)
+    assert np.array_equal(starts.cpu().numpy(), ref_starts)
+
+
+MXB = [  # (rows, cols, group ends)
+    (300, 96, [0, 100, 100, 290]),          # empty groups, rows past the last group
+    (257, 512, [257]),
+    (1000, 224, [1, 3, 6, 506, 506, 1000]),  # cols/32 = 7: a partial last scale word
+    (4096, 7168, [1000, 1000, 3000, 4096]),
+]
+
+
+@pytest.mark.parametrize("mode", ["floor", "rceil"])
+@pytest.mark.parametrize("rows,cols,ends", MXB)
+def test_mx_rowwise_blocked_vs_oracle(rows, cols, ends, mode):
+    x = synth.normal_bf16((rows, cols), 1.0, seed=rows + cols, device=DEV)
+    offs = torch.tensor(ends, dtype=torch.int32)
+    m = 0 if mode == "floor" else 1
+    rq, rsb, rstarts = oracle.mx_quant_rowwise_blocked_grouped(words(x).reshape(-1), rows, cols, m, offs.numpy())
+    bigq, q = guarded(rows * cols)
+    bigs, sb = guarded(rsb.size)
+    _, _, starts = mxq.mx_quant_rowwise_blocked_grouped(x, offs.to(DEV), mode, out=q.view(rows, cols), scales=sb)
+    assert status_ok()
+    assert np.array_equal(u8(q).reshape(rows, cols), rq)
+    assert np.array_equal(u8(sb), rsb)
+    assert np.array_equal(starts.cpu().numpy(), rstarts)
+    assert margins_intact(bigq) and margins_intact(bigs)
+
+
+def test_mx_rowwise_blocked_full_size_is_rowwise_then_conversion():
+    """Full activation config, (65536, 7168) with G=64 Dirichlet(0.3) groups:
+    the fused op's bytes equal mx_quant_rowwise followed by
+    mx_scales_to_blocked_grouped (both verified against the oracle above),
+    and a sample of rows from every group matches the oracle."""
+    x, offs = synth.mx_act(device=DEV)
+    offs_d = offs.to(DEV)
+    for mode in ("floor", "rceil"):
+        q, sb, starts = mxq.mx_quant_rowwise_blocked_grouped(x, offs_d, mode)
+        q2, sc = mxq.mx_quant_rowwise(x, mode)
+        sb2, starts2 = mxq.mx_scales_to_blocked_grouped(sc, offs_d)
+        assert status_ok()
+        assert torch.equal(q.view(torch.uint8), q2.view(torch.uint8))
+        assert torch.equal(sb, sb2) and torch.equal(starts, starts2)
+    # oracle on the first rows of a few groups (the blocked bytes of those rows)
+    o = offs.numpy()
+    st = starts.cpu().numpy()
+    sbn = sb.cpu().numpy()
+    tc = 7168 // 128
+    for g in [0, 7, 31, 63]:
+        a = int(o[g - 1]) if g else 0
+        b = min(int(o[g]), a + 8)
+        if b <= a:
+            continue
+        _, rs = oracle.mx_quant_rowwise(words(x[a:b]), 1)
+        for i in range(b - a):
+            rb = int(st[g]) + i
+            for c in range(224):
+                off = ((rb // 128) * tc + c // 4) * 512 + (rb % 32) * 16 + ((rb % 128) // 32) * 4 + c % 4
+                assert sbn[off] == rs[i, c], (g, i, c)
+
+
 # ============================================================ errors and edges
 
 def test_bad_offsets_are_reported_and_nothing_is_written():
