@@ -46,6 +46,7 @@ def lib():
             "oracle_fp8_quant_jagged_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _i64, _i32p, _i32, _u8p, _f32p]),
             "oracle_fp8_quant_jagged_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _i64, _i32p, _i32, _u8p, _f32p]),
             "oracle_fp8_quant_blockwise": (ctypes.c_int, [_u16p, _i64, _i64, _i32, _i32, _u8p, _f32p]),
+            "oracle_fp8_quant_blockwise_transposed": (ctypes.c_int, [_u16p, _i64, _i64, _i32, _i32, _u8p, _f32p]),
             "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
@@ -158,6 +159,18 @@ def fp8_quant_blockwise(x, br, bc):
     out = np.zeros((rows, cols), dtype=np.uint8)
     inv = np.zeros((rows // br, cols // bc), dtype=np.float32)
     _check(lib().oracle_fp8_quant_blockwise(_p(w, _u16p), rows, cols, br, bc, _p(out, _u8p), _p(inv, _f32p)))
+    return out, inv
+
+
+def fp8_quant_blockwise_transposed(x, br, bc):
+    """Blockwise br x bc on x (rows, cols), written transposed. Returns
+    (out (cols, rows), inv (cols/bc, rows/br))."""
+    w = np.ascontiguousarray(_words(x))
+    rows, cols = w.shape
+    out = np.zeros((cols, rows), dtype=np.uint8)
+    inv = np.zeros((cols // bc, rows // br), dtype=np.float32)
+    _check(lib().oracle_fp8_quant_blockwise_transposed(_p(w, _u16p), rows, cols, br, bc, _p(out, _u8p),
+                                                       _p(inv, _f32p)))
     return out, inv
 
 

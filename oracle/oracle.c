@@ -321,6 +321,41 @@ int oracle_fp8_quant_blockwise(const uint16_t *in, int64_t rows, int64_t cols,
 }
 
 /* ------------------------------------------------------------------ */
+/* Blockwise with transposed output (#2827 description: the (blocksize */
+/* x 1) tiles of the blockwise linear, and the transposed weight). The  */
+/* row-major (rows, cols) input is quantized in br x bc blocks          */
+/* (br = 128; bc = 1 or 128) and written transposed: out[c*rows + r],   */
+/* one inverse scale per block at inv[(c/bc) * (rows/br) + r/br], i.e.  */
+/* the (cols/bc, rows/br) row-major scale matrix of the transpose.      */
+/* ------------------------------------------------------------------ */
+int oracle_fp8_quant_blockwise_transposed(const uint16_t *in, int64_t rows, int64_t cols,
+                                          int32_t br, int32_t bc, uint8_t *out, float *inv_scales)
+{
+    int64_t nbr, nbc;
+    if (rows < 0 || cols < 0 || br <= 0 || bc <= 0 || rows % br || cols % bc)
+        return ORACLE_ERR_ARG;
+    nbr = rows / br;
+    nbc = cols / bc;
+    for (int64_t bj = 0; bj < nbc; ++bj) {
+        for (int64_t bi = 0; bi < nbr; ++bi) {
+            float amax = 0.0f, s;
+            for (int64_t r = bi * br; r < (bi + 1) * br; ++r)
+                for (int64_t c = bj * bc; c < (bj + 1) * bc; ++c) {
+                    float a = absf(bf16_value(in[r * cols + c]));
+                    if (a > amax)
+                        amax = a;
+                }
+            s = oracle_fp8_scale(amax);
+            inv_scales[bj * nbr + bi] = 1.0f / s;
+            for (int64_t r = bi * br; r < (bi + 1) * br; ++r)
+                for (int64_t c = bj * bc; c < (bj + 1) * bc; ++c)
+                    out[c * rows + r] = oracle_e4m3_from_float(bf16_value(in[r * cols + c]) * s);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* (a4) MX 3-D colwise: expert weights (E, N, K) quantized along N in   */
 /* 32x1 blocks, each expert written column-major:                       */
 /* out[e*N*K + k*N + n], scales (E, K, N/32). #3002 Summary.            */

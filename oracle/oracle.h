@@ -42,6 +42,8 @@ int oracle_fp8_quant_jagged_colwise(const uint16_t *in, int64_t rows, int64_t co
                                     uint8_t *out, float *inv_scales);
 int oracle_fp8_quant_blockwise(const uint16_t *in, int64_t rows, int64_t cols,
                                int32_t br, int32_t bc, uint8_t *out, float *inv_scales);
+int oracle_fp8_quant_blockwise_transposed(const uint16_t *in, int64_t rows, int64_t cols,
+                                          int32_t br, int32_t bc, uint8_t *out, float *inv_scales);
 int oracle_mx_quant_3d_colwise(const uint16_t *in, int64_t E, int64_t N, int64_t K,
                                int mode, uint8_t *out, uint8_t *scales);
 int oracle_mx_quant_rowwise(const uint16_t *in, int64_t rows, int64_t cols, int mode,

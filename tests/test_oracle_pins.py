@@ -395,6 +395,34 @@ def test_grouped_blocked_k_bound_is_tight(oracle):
         oracle.mx_scales_to_blocked_grouped_k(np.zeros((4, 6), np.uint8), [1, 6], capacity_cols=8)
 
 
+@pytest.mark.parametrize("br,bc", [(128, 1), (128, 128)])
+def test_blockwise_transposed_is_blockwise_of_the_transpose(oracle, br, bc):
+    """A br x bc block of x is a bc x br block of x^T: the transposed op equals
+    the (pinned) blockwise op on the contiguous transpose, whose blocks are
+    1 x 128 for br x bc = 128 x 1 and 128 x 128 for 128 x 128."""
+    rng = np.random.default_rng(br + bc)
+    x = torch.from_numpy((rng.standard_normal((256, 384)) * np.exp2(rng.integers(-6, 6, (256, 1)))).astype(
+        np.float32)).to(torch.bfloat16)
+    q, inv = oracle.fp8_quant_blockwise_transposed(x, br, bc)
+    q2, inv2 = oracle.fp8_quant_blockwise(x.t().contiguous(), bc, br)
+    assert np.array_equal(q, q2)
+    assert np.array_equal(inv.view(np.uint32), inv2.view(np.uint32))
+
+
+def test_blockwise_transposed_hand_example(oracle):
+    """A 128 x 1 block whose amax is 2 (a power of two): s = 224, inv = 1/224;
+    x = 1 -> 224 -> 0x76, x = -2 -> -448 -> 0xFE, x = 0.5 -> 112 -> 0x6E; the
+    other column of zeros keeps amax 0: s = 448 / 1e-12, every byte 0x00."""
+    x = torch.zeros((128, 1), dtype=torch.float32)
+    x[0, 0], x[1, 0], x[2, 0] = 1.0, -2.0, 0.5
+    x = torch.cat([x, torch.zeros((128, 1))], dim=1).to(torch.bfloat16)
+    q, inv = oracle.fp8_quant_blockwise_transposed(x, 128, 1)
+    assert list(q[0, :3]) == [0x76, 0xFE, 0x6E]
+    assert np.float32(inv[0, 0]) == np.float32(1.0) / np.float32(224.0)
+    assert not q[1].any()
+    assert np.float32(inv[1, 0]) == np.float32(1.0) / (np.float32(448.0) / np.float32(1e-12))
+
+
 def test_rowwise_blocked_is_rowwise_then_conversion(oracle):
     rng = np.random.default_rng(3)
     x = torch.from_numpy(rng.standard_normal((300, 96)).astype(np.float32)).to(torch.bfloat16)
