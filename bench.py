@@ -373,6 +373,18 @@ def per_shape_sweep(wl, reps):
                 lambda s=s, o=o, cap=cap, out=out, st=st: mxq.mx_scales_to_blocked_grouped(
                     s, o, capacity_rows=cap, out=out, group_row_starts=st),
                 R * C + cap * C)
+    # blockwise with transposed output: activations 128x1, weight 128x128
+    qt_a = torch.empty(4096 * 16384, dtype=torch.uint8, device=dev)
+    it_a = torch.empty((4096, 128), dtype=torch.float32, device=dev)
+    run("blockwise_128x1_t", "(16384,4096)",
+        lambda: mxq.fp8_quant_blockwise_transposed(wl.act, 1, out=qt_a.view(4096, 16384), inv_scales=it_a),
+        16384 * 4096 * 3 + 4096 * 128 * 4)
+    qt_w = torch.empty(4096 * 14336, dtype=torch.uint8, device=dev)
+    it_w = torch.empty((32, 112), dtype=torch.float32, device=dev)
+    run("blockwise_128x128_t", "(14336,4096)",
+        lambda: mxq.fp8_quant_blockwise_transposed(wl.wt, 128, out=qt_w.view(4096, 14336), inv_scales=it_w),
+        14336 * 4096 * 3 + 32 * 112 * 4)
+    del qt_a, qt_w
     # groups along K: the pages' sweep shapes, G=8 along the columns, capacity C + 4G
     for R in (8192, 5120, 7168, 2048):
         for C in (512, 1024, 2048, 4096, 32768):

@@ -140,6 +140,25 @@ int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols,
                         void *out, float *inv_scales, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * fp8_quant_blockwise_transposed - #2827 description (the blocksize x 1
+ * tiles of the blockwise linear): e4m3 with one scale per 128 x block_cols
+ * block of a row-major (rows, cols) bf16 matrix, written TRANSPOSED.
+ *   block_rows  128; block_cols 1 (activations as the column-major right
+ *               operand) or 128 (the transposed weight); else
+ *               MXQ_ERR_UNSUPPORTED. rows % 128 == 0 and cols % 128 == 0,
+ *               else MXQ_ERR_SHAPE.
+ *   in, out     16-byte aligned; out[c * rows + r], i.e. (cols, rows)
+ *               row-major.
+ *   inv_scales  fp32 (cols / block_cols, rows / 128) row-major: the scale
+ *               matrix of the transpose. The result equals
+ *               fp8_quant_blockwise on the contiguous transpose with blocks
+ *               block_cols x 128.
+ * ------------------------------------------------------------------------ */
+int fp8_quant_blockwise_transposed(const void *in, int64_t rows, int64_t cols,
+                                   int32_t block_rows, int32_t block_cols,
+                                   void *out, float *inv_scales, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * (a4) mx_quant_3d_colwise - #3002 Summary: MXFP8 quantization of expert
  * weights (E, N, K) along N in 32 x 1 blocks, written straight into each
  * expert's column-major layout.

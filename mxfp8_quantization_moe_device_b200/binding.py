@@ -35,6 +35,7 @@ SIGNATURES = {
     "fp8_quant_jagged_colwise_noalloc": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp]),
     "fp8_quant_jagged_colwise_noalloc_max_scratch_bytes": (_sz, []),
     "fp8_quant_blockwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "fp8_quant_blockwise_transposed": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
@@ -189,6 +190,24 @@ def fp8_quant_blockwise(x, block_rows=1, block_cols=128, *, out=None, inv_scales
 
 
 # ---------------------------------------------------------------- MX
+
+def fp8_quant_blockwise_transposed(x, block_cols=1, *, out=None, inv_scales=None):
+    """e4m3 quantization of row-major x (rows, cols) in 128 x block_cols blocks
+    (block_cols 1 or 128), written transposed. Returns (q (cols, rows)
+    float8_e4m3fn, inv (cols / block_cols, rows / 128) fp32)."""
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    if inv_scales is None:
+        inv_scales = torch.empty((cols // block_cols, rows // 128), dtype=torch.float32, device=x.device)
+    rc = lib().fp8_quant_blockwise_transposed(_ptr(x), rows, cols, 128, block_cols, _ptr(out), _ptr(inv_scales),
+                                              _stream(x.device))
+    _check("fp8_quant_blockwise_transposed", rc)
+    return out.view(torch.float8_e4m3fn), inv_scales
+
 
 def mx_quant_3d_colwise(w, mode="floor", *, out=None, scales=None):
     """MXFP8 quantization of expert weights w (E, N, K) along N (32x1 blocks).

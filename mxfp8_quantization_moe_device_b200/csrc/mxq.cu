@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "rowblock.cuh"
+#include "blockt.cuh"
 #include "mx3d.cuh"
 #include "jagged.cuh"
 #include "blocked.cuh"
@@ -94,6 +95,8 @@ int device_info(const DevInfo **out)
             return MXQ_ERR_CUDA;
         if (cudaFuncSetAttribute(mx3d::k_mx_3d_colwise, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mx3d::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_blockwise_t, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)bt::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(k_jagged_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)jag::cst::SMEM_BYTES) != cudaSuccess)
             return MXQ_ERR_CUDA;
@@ -310,6 +313,47 @@ int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols, int32_t bloc
         return MXQ_ERR_UNSUPPORTED;
     return launch(k_fp8_128x128, dim3((unsigned)(cols / 128), (unsigned)(rows / 128)), dim3(256), 0, stream, false,
                   static_cast<const uint4 *>(in), cols, static_cast<uint2 *>(out), inv_scales);
+}
+
+int fp8_quant_blockwise_transposed(const void *in, int64_t rows, int64_t cols, int32_t block_rows,
+                                   int32_t block_cols, void *out, float *inv_scales, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0)
+        return MXQ_ERR_SHAPE;
+    if (block_rows != 128 || (block_cols != 1 && block_cols != 128))
+        return MXQ_ERR_UNSUPPORTED;
+    if (rows % 128 || cols % 128)
+        return MXQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0)
+        return MXQ_OK;
+    if (!in || !out || !inv_scales)
+        return MXQ_ERR_NULL;
+    if (!aligned(in, 16) || !aligned(out, 16) || !aligned(inv_scales, 4))
+        return MXQ_ERR_ALIGN;
+    if ((rows / 128) * (cols / 128) >= (int64_t(1) << 31) || rows >= (int64_t(1) << 31) ||
+        cols >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    CUtensorMap tin, tout;
+    const uint64_t din[2] = {(uint64_t)cols, (uint64_t)rows};
+    const uint64_t sin[1] = {(uint64_t)cols * 2};
+    const uint32_t bin[2] = {bt::TH, bt::TR};
+    rc = make_map(&tin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, din, sin, bin, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t dout[2] = {(uint64_t)rows, (uint64_t)cols};
+    const uint64_t sout[1] = {(uint64_t)rows};
+    const uint32_t bout[2] = {bt::TR, bt::TH};
+    rc = make_map(&tout, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t items = (rows / 128) * (cols / 128);
+    const int64_t grid = std::min<int64_t>(items, (int64_t)di->sms * bt::CTAS_PER_SM);
+    return launch(k_fp8_blockwise_t, dim3((unsigned)grid), dim3(bt::THREADS), bt::SMEM_BYTES, stream, false, tin,
+                  tout, inv_scales, rows, cols, (int)block_cols, wait_ns());
 }
 
 int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t mode, void *out, uint8_t *scales,

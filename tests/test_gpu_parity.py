@@ -416,6 +416,42 @@ def test_mx_rowwise_full_size_tokens():
         assert np.array_equal(s[torch.from_numpy(rows).to(DEV)].cpu().numpy(), rs)
 
 
+# ============================================================ blockwise, transposed output
+
+@pytest.mark.parametrize("bc", [1, 128])
+@pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (1024, 640), (384, 2048)])
+def test_blockwise_transposed_vs_oracle(rows, cols, bc):
+    x = synth.outlier_normal_bf16(rows, cols, seed=rows + cols + bc, device=DEV)
+    rq, rinv = oracle.fp8_quant_blockwise_transposed(x, 128, bc)
+    bigq, q = guarded(rows * cols)
+    bigi, inv = guarded(rinv.size, torch.float32)
+    mxq.fp8_quant_blockwise_transposed(x, bc, out=q.view(cols, rows), inv_scales=inv.view(rinv.shape))
+    assert status_ok()
+    assert np.array_equal(u8(q).reshape(cols, rows), rq)
+    assert np.array_equal(f32bits(inv.cpu().numpy()).reshape(rinv.shape), f32bits(rinv))
+    assert margins_intact(bigq) and margins_intact(bigi, torch.float32)
+
+
+@pytest.mark.parametrize("which", ["act_128x1", "weight_128x128"])
+def test_blockwise_transposed_config_shapes(which):
+    """The blockwise linear's shapes: activations (16384, 4096) in 128x1 blocks
+    and the weight (14336, 4096) in 128x128 blocks, both written transposed;
+    compared in full with the oracle, and with the (already verified)
+    row-major kernel run on the contiguous transpose."""
+    if which == "act_128x1":
+        x, bc = synth.blockwise_act(device=DEV), 1
+    else:
+        x, bc = synth.blockwise_weight(device=DEV), 128
+    q, inv = mxq.fp8_quant_blockwise_transposed(x, bc)
+    assert status_ok()
+    rq, rinv = oracle.fp8_quant_blockwise_transposed(x, 128, bc)
+    assert np.array_equal(u8(q), rq)
+    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(rinv))
+    q2, inv2 = mxq.fp8_quant_blockwise(x.t().contiguous(), bc, 128)
+    assert torch.equal(q.view(torch.uint8), q2.view(torch.uint8))
+    assert torch.equal(inv.view(torch.int32), inv2.view(torch.int32))
+
+
 # ============================================================ blocked layout
 
 BLOCKED = [
