@@ -59,7 +59,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--reps", type=int, default=50, help="reps per shape in the per-shape sweep (cold and hot each)")
-    p.add_argument("--profile-op", default=None, choices=list(Workload.OPS),
+    p.add_argument("--profile-op", default=None, choices=list(Workload.OPS) + list(Workload.EXTRA),
                    help="run only this op (for single-kernel profiler captures)")
     p.add_argument("--iters", type=int, default=3, help="calls of --profile-op after one warm-up")
     return p.parse_args()
@@ -80,7 +80,8 @@ def load_peaks():
 KERNEL_FILES = {  # source files that define each kernel (plus common.cuh)
     "k_fp8_1x128": "rowblock.cuh", "k_fp8_128x128": "rowblock.cuh", "k_mx_1x32": "rowblock.cuh",
     "k_jagged_amax": "jagged.cuh", "k_jagged_cast": "jagged.cuh", "k_mx_3d_colwise": "mx3d.cuh",
-    "k_blocked_grouped": "blocked.cuh",
+    "k_blocked_grouped": "blocked.cuh", "k_blocked_grouped_k": "blocked.cuh", "k_mx_1x32_blocked": "blocked.cuh",
+    "k_fp8_blockwise_t": "blockt.cuh",
 }
 
 
@@ -171,6 +172,8 @@ class Workload:
 
     OPS = ("blockwise_1x128", "blockwise_128x128", "jagged_rowwise", "jagged_colwise", "mx_3d_colwise",
            "mx_rowwise", "blocked_grouped")
+    # ops outside the step (the widened rows), built only when asked for by name
+    EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked")
 
     def __init__(self, dev, experts, mx3d_mode, only=None):
         import torch
@@ -235,6 +238,36 @@ class Workload:
                 self.ops.append(("blocked_grouped", lambda: mxq.mx_scales_to_blocked_grouped(
                     self.o["tok_s"], self.offs64, capacity_rows=self.cap, out=self.o["blk"],
                     group_row_starts=self.o["blk_starts"]), T * (KT // 32) + self.cap * c4))
+
+        if "blockwise_128x1_t" in want:
+            self.act = synth.blockwise_act(device=dev)
+            self.o.update(act_qt=t.empty((4096, 16384), **u8), act_st=t.empty((4096, 128), **f32))
+            self.ops.append(("blockwise_128x1_t", lambda: mxq.fp8_quant_blockwise_transposed(
+                self.act, 1, out=self.o["act_qt"], inv_scales=self.o["act_st"]), 16384 * 4096 * 3 + 4096 * 128 * 4))
+        if "blockwise_128x128_t" in want:
+            self.wt = synth.blockwise_weight(device=dev)
+            self.o.update(wt_qt=t.empty((4096, 14336), **u8), wt_st=t.empty((32, 112), **f32))
+            self.ops.append(("blockwise_128x128_t", lambda: mxq.fp8_quant_blockwise_transposed(
+                self.wt, 128, out=self.o["wt_qt"], inv_scales=self.o["wt_st"]), 14336 * 4096 * 3 + 32 * 112 * 4))
+        if "blocked_grouped_k" in want:
+            R, C = 8192, 32768
+            self.sk, ok = synth.scale_sweep_k(R, C, device=dev)
+            self.offs_k = ok.to(dev)
+            self.o.update(blk_k=t.empty(R * (C + 32), **u8), blk_k_starts=t.empty(8, dtype=t.int32, device=dev))
+            self.ops.append(("blocked_grouped_k", lambda: mxq.mx_scales_to_blocked_grouped_k(
+                self.sk, self.offs_k, capacity_cols=C + 32, out=self.o["blk_k"],
+                group_col_starts=self.o["blk_k_starts"]), R * C + R * (C + 32)))
+        if "mx_rowwise_blocked" in want:
+            self.tok, offs64 = synth.mx_act(device=dev)
+            self.offs64 = offs64.to(dev)
+            T, KT = self.tok.shape
+            self.cap = mxq.blocked_grouped_rows_bound(T, 64)
+            sbytes = self.cap * (KT // 128) * 4
+            self.o.update(tok_q=t.empty((T, KT), **u8), tok_sb=t.empty(sbytes, **u8),
+                          tok_sb_starts=t.empty(64, dtype=t.int32, device=dev))
+            self.ops.append(("mx_rowwise_blocked", lambda: mxq.mx_quant_rowwise_blocked_grouped(
+                self.tok, self.offs64, "floor", capacity_rows=self.cap, out=self.o["tok_q"], scales=self.o["tok_sb"],
+                group_row_starts=self.o["tok_sb_starts"]), T * KT * 3 + sbytes))
 
     def step_bytes(self):
         return sum(b for _, _, b in self.ops)

@@ -1,0 +1,128 @@
+"""torch.library registration (torch.ops.mxq.*): fake (shape-only)
+implementations on CPU meta tensors; on a GPU, the registered ops against the
+binding, torch.library.opcheck, and capture by torch.compile."""
+import numpy as np
+import pytest
+import torch
+
+import mxfp8_quantization_moe_device_b200.ops  # noqa: F401  (registers torch.ops.mxq)
+from mxfp8_quantization_moe_device_b200 import binding as mxq
+from mxfp8_quantization_moe_device_b200 import synth
+
+OPS = ["fp8_quant_jagged_rowwise", "fp8_quant_jagged_colwise", "fp8_quant_blockwise",
+       "fp8_quant_blockwise_transposed", "mx_quant_3d_colwise", "mx_quant_rowwise", "mx_scales_to_blocked_grouped",
+       "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped"]
+
+
+def _cases(dev):
+    x = synth.row_scaled_normal_bf16(256, 512, seed=3, device=dev)
+    offs = torch.tensor([64, 64, 200, 256], dtype=torch.int32, device=dev)
+    offs_c = torch.tensor([100, 300, 512], dtype=torch.int32, device=dev)
+    s = synth.uniform_u8((300, 7), 0, 254, seed=4, device=dev)
+    offs_s = torch.tensor([1, 150, 300], dtype=torch.int32, device=dev)
+    offs_k = torch.tensor([2, 2, 7], dtype=torch.int32, device=dev)
+    w = synth.normal_bf16((2, 64, 96), 0.02, seed=5, device=dev)
+    return [
+        ("fp8_quant_jagged_rowwise", (x.t(), offs)),
+        ("fp8_quant_jagged_colwise", (x, offs)),
+        ("fp8_quant_jagged_rowwise", (x, offs_c)),
+        ("fp8_quant_blockwise", (x, 1)),
+        ("fp8_quant_blockwise", (x, 128)),
+        ("fp8_quant_blockwise_transposed", (x, 1)),
+        ("fp8_quant_blockwise_transposed", (x, 128)),
+        ("mx_quant_3d_colwise", (w, "floor")),
+        ("mx_quant_rowwise", (x, "rceil")),
+        ("mx_scales_to_blocked_grouped", (s, offs_s)),
+        ("mx_scales_to_blocked_grouped_k", (s, offs_k)),
+        ("mx_quant_rowwise_blocked_grouped", (x, offs, "floor")),
+    ]
+
+
+def _meta(t):
+    return torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, device="meta") if isinstance(t, torch.Tensor) else t
+
+
+def test_every_op_is_registered():
+    for name in OPS:
+        assert hasattr(torch.ops.mxq, name), name
+
+
+def test_fake_shapes_on_meta_tensors():
+    want = {  # (shapes, dtypes) of each case's outputs
+        0: ([(512, 256), (4, 512)], [torch.float8_e4m3fn, torch.float32]),
+        1: ([(512, 256), (4, 512)], [torch.float8_e4m3fn, torch.float32]),
+        2: ([(256, 512), (3, 256)], [torch.float8_e4m3fn, torch.float32]),
+        3: ([(256, 512), (256, 4)], [torch.float8_e4m3fn, torch.float32]),
+        4: ([(256, 512), (2, 4)], [torch.float8_e4m3fn, torch.float32]),
+        5: ([(512, 256), (512, 2)], [torch.float8_e4m3fn, torch.float32]),
+        6: ([(512, 256), (4, 2)], [torch.float8_e4m3fn, torch.float32]),
+        7: ([(2, 96, 64), (2, 96, 2)], [torch.float8_e4m3fn, torch.uint8]),
+        8: ([(256, 512), (256, 16)], [torch.float8_e4m3fn, torch.uint8]),
+        9: ([(128 * ((300 + 127 * 3) // 128) * 8,), (3,)], [torch.uint8, torch.int32]),
+        10: ([(384 * 4 * ((7 + 9) // 4),), (3,)], [torch.uint8, torch.int32]),
+        11: ([(256, 512), (128 * ((256 + 127 * 4) // 128) * 16,), (4,)],
+             [torch.float8_e4m3fn, torch.uint8, torch.int32]),
+    }
+    for i, (name, args) in enumerate(_cases("cpu")):
+        out = getattr(torch.ops.mxq, name)(*[_meta(a) for a in args])
+        shapes, dtypes = want[i]
+        assert [tuple(o.shape) for o in out] == shapes, (i, name)
+        assert [o.dtype for o in out] == dtypes, (i, name)
+
+
+gpu = pytest.mark.gpu
+
+
+def _bytes(t):
+    return t.contiguous().view(torch.uint8) if t.dtype != torch.uint8 else t
+
+
+@gpu
+def test_registered_ops_match_the_binding():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    for name, args in _cases("cuda"):
+        got = getattr(torch.ops.mxq, name)(*args)
+        fn = getattr(mxq, name)
+        if name == "fp8_quant_blockwise":
+            ref = fn(args[0], args[1], 128)
+        elif name in ("fp8_quant_blockwise_transposed",):
+            ref = fn(*args)
+        elif name == "mx_quant_3d_colwise":
+            q, sc = fn(*args)
+            ref = (q.transpose(1, 2), sc)
+        elif name == "fp8_quant_jagged_colwise":
+            q, inv = fn(*args)
+            ref = (q.t(), inv)
+        else:
+            ref = fn(*args)
+        assert mxq.device_status() == 0
+        for g, r in zip(got, ref):
+            assert torch.equal(_bytes(g), _bytes(r)), name
+
+
+@gpu
+def test_opcheck():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    for name, args in _cases("cuda"):
+        torch.library.opcheck(getattr(torch.ops.mxq, name).default, args,
+                              test_utils=("test_schema", "test_faketensor", "test_autograd_registration"))
+
+
+@gpu
+def test_torch_compile_captures_the_ops_without_graph_breaks():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    x = synth.row_scaled_normal_bf16(256, 512, seed=3, device="cuda")
+    offs = torch.tensor([64, 64, 200, 256], dtype=torch.int32, device="cuda")
+
+    def step(x, offs):
+        qt, inv = torch.ops.mxq.fp8_quant_jagged_colwise(x, offs)
+        q, sb, starts = torch.ops.mxq.mx_quant_rowwise_blocked_grouped(x, offs, "floor")
+        return qt, inv, q, sb, starts
+
+    eager = step(x, offs)
+    compiled = torch.compile(step, fullgraph=True, backend="aot_eager")(x, offs)
+    for a, b in zip(eager, compiled):
+        assert np.array_equal(_bytes(a).cpu().numpy(), _bytes(b).cpu().numpy())
