@@ -47,6 +47,8 @@ def lib():
             "oracle_fp8_quant_jagged_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _i64, _i32p, _i32, _u8p, _f32p]),
             "oracle_fp8_quant_blockwise": (ctypes.c_int, [_u16p, _i64, _i64, _i32, _i32, _u8p, _f32p]),
             "oracle_fp8_quant_blockwise_transposed": (ctypes.c_int, [_u16p, _i64, _i64, _i32, _i32, _u8p, _f32p]),
+            "oracle_fp8_grouped_gemm_rowwise": (ctypes.c_int, [_u8p, _f32p, _u8p, _f32p, _i64, _i64, _i64, _i32p,
+                                                               _i32, ctypes.POINTER(ctypes.c_double)]),
             "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
@@ -172,6 +174,24 @@ def fp8_quant_blockwise_transposed(x, br, bc):
     _check(lib().oracle_fp8_quant_blockwise_transposed(_p(w, _u16p), rows, cols, br, bc, _p(out, _u8p),
                                                        _p(inv, _f32p)))
     return out, inv
+
+
+def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, out=None):
+    """a (M, K) e4m3 codes, inv_a (M,), w (E, N, K) codes, inv_w (E, N),
+    offs (E,) group ends along M. Returns out (M, N) float64; rows past the
+    last offset keep the values of `out` (zeros when not given)."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    w = np.ascontiguousarray(w, dtype=np.uint8)
+    ia = np.ascontiguousarray(inv_a, dtype=np.float32)
+    iw = np.ascontiguousarray(inv_w, dtype=np.float32)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    M, K = a.shape
+    E, N, K2 = w.shape
+    assert K2 == K and len(o) == E
+    res = np.zeros((M, N), dtype=np.float64) if out is None else np.ascontiguousarray(out, dtype=np.float64)
+    _check(lib().oracle_fp8_grouped_gemm_rowwise(_p(a, _u8p), _p(ia, _f32p), _p(w, _u8p), _p(iw, _f32p), M, N, K,
+                                                 _p(o, _i32p), E, res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return res
 
 
 def mx_quant_3d_colwise(x, mode):

@@ -521,3 +521,38 @@ int oracle_mx_quant_rowwise_blocked_grouped(const uint16_t *in, int64_t rows, in
     return rc;
 }
 
+/* ------------------------------------------------------------------ */
+/* FP8 rowwise-scaled grouped GEMM, the consumer of these buffers       */
+/* (#2064 Motivation and #2077 Summary: the differentiable scaled       */
+/* grouped mm the quantization feeds). Row m of A belongs to the group  */
+/* g with offs[g-1] <= m < offs[g]; its output row is                    */
+/*   out[m][n] = (sum_k e4m3(a[m][k]) * e4m3(w[g][n][k])) * inv_a[m]     */
+/*               * inv_w[g][n]                                           */
+/* computed in double (every e4m3 product is exact in double; the sum of */
+/* K of them is exact to far below fp32 resolution). Rows past          */
+/* offs[G-1] are not written.                                            */
+/* ------------------------------------------------------------------ */
+int oracle_fp8_grouped_gemm_rowwise(const uint8_t *a, const float *inv_a, const uint8_t *w, const float *inv_w,
+                                    int64_t M, int64_t N, int64_t K, const int32_t *offs, int32_t groups,
+                                    double *out)
+{
+    int64_t start = 0;
+    if (M < 0 || N < 0 || K < 0 || groups <= 0)
+        return ORACLE_ERR_ARG;
+    if (!offsets_valid(offs, groups, M))
+        return ORACLE_ERR_OFFSETS;
+    for (int32_t g = 0; g < groups; ++g) {
+        const uint8_t *wg = w + (int64_t)g * N * K;
+        for (int64_t m = start; m < offs[g]; ++m) {
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += oracle_e4m3_value(a[m * K + k]) * oracle_e4m3_value(wg[n * K + k]);
+                out[m * N + n] = acc * (double)inv_a[m] * (double)inv_w[(int64_t)g * N + n];
+            }
+        }
+        start = offs[g];
+    }
+    return 0;
+}
+

@@ -423,6 +423,39 @@ def test_blockwise_transposed_hand_example(oracle):
     assert np.float32(inv[1, 0]) == np.float32(1.0) / (np.float32(448.0) / np.float32(1e-12))
 
 
+def test_grouped_gemm_vs_numpy_matmul(oracle):
+    """The grouped GEMM against numpy's float64 matmul of the decoded e4m3
+    values, group by group, with the scales applied afterwards."""
+    rng = np.random.default_rng(11)
+    M, N, K, E = 70, 24, 48, 3
+    a = rng.integers(0, 256, size=(M, K), dtype=np.uint8)
+    w = rng.integers(0, 256, size=(E, N, K), dtype=np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0   # no NaN codes
+    w[(w & 0x7F) == 0x7F] = 0
+    ia = rng.uniform(0.5, 2.0, M).astype(np.float32)
+    iw = rng.uniform(0.5, 2.0, (E, N)).astype(np.float32)
+    offs = np.array([20, 20, 64], dtype=np.int32)   # empty group; rows 64.. past the last group
+    got = oracle.fp8_grouped_gemm_rowwise(a, ia, w, iw, offs)
+    dec = np.array([oracle.e4m3_value(c) for c in range(256)])
+    A, W = dec[a], dec[w]
+    start = 0
+    for g, end in enumerate(offs):
+        ref = (A[start:end] @ W[g].T) * ia[start:end, None].astype(np.float64) * iw[g][None, :].astype(np.float64)
+        assert np.allclose(got[start:end], ref, rtol=1e-13, atol=0)
+        start = end
+    assert not got[64:].any()
+
+
+def test_grouped_gemm_hand_example(oracle):
+    """One row, one column, K = 2: a = [1, 2] (0x38, 0x40), w = [0.5, -3]
+    (0x30, 0xC4): 1*0.5 + 2*(-3) = -5.5; scales 2 and 0.25 give -2.75."""
+    a = np.array([[0x38, 0x40]], dtype=np.uint8)
+    w = np.array([[[0x30, 0xC4]]], dtype=np.uint8)
+    got = oracle.fp8_grouped_gemm_rowwise(a, np.array([2.0], np.float32), w, np.array([[0.25]], np.float32),
+                                          np.array([1], np.int32))
+    assert got[0, 0] == -2.75
+
+
 def test_rowwise_blocked_is_rowwise_then_conversion(oracle):
     rng = np.random.default_rng(3)
     x = torch.from_numpy(rng.standard_normal((300, 96)).astype(np.float32)).to(torch.bfloat16)
