@@ -159,6 +159,28 @@ int fp8_quant_blockwise_transposed(const void *in, int64_t rows, int64_t cols,
                                    void *out, float *inv_scales, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * fp8_grouped_gemm_rowwise - the consumer of these buffers (#2064
+ * Motivation, #2077 Summary: the scaled grouped mm the quantization feeds):
+ * a grouped GEMM on the tensor cores (tcgen05, fp32 accumulation in TMEM)
+ *   out[m][n] = bf16((sum_k a[m][k] * w[g][n][k]) * inv_a[m] * inv_w[g][n])
+ * for each row m of group g = [offs[g-1], offs[g]).
+ *   a       e4m3 (M, K) row-major (K contiguous), 16-byte aligned.
+ *   inv_a   fp32 (M): per-row inverse scales (fp8_quant_jagged_rowwise of A
+ *           with one group spanning K).
+ *   w       e4m3 (num_groups, N, K) row-major, 16-byte aligned.
+ *   inv_w   fp32 (num_groups, N): per-(expert, row) inverse scales.
+ *   offs    num_groups int32 ends along M (device).
+ *   out     bf16 (M, N) row-major, 16-byte aligned; rows past
+ *           offs[num_groups-1] are not written.
+ *   N % 128 == 0 and K % 128 == 0 (K > 0), else MXQ_ERR_SHAPE;
+ *   num_groups <= 4096, else MXQ_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, const float *inv_w,
+                             int64_t M, int64_t N, int64_t K,
+                             const int32_t *offs, int32_t num_groups, void *out,
+                             cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * (a4) mx_quant_3d_colwise - #3002 Summary: MXFP8 quantization of expert
  * weights (E, N, K) along N in 32 x 1 blocks, written straight into each
  * expert's column-major layout.

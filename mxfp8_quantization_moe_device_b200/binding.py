@@ -37,6 +37,7 @@ SIGNATURES = {
     "fp8_quant_blockwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "fp8_quant_blockwise_transposed": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "fp8_grouped_gemm_rowwise": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
     "mx_blocked_grouped_rows_bound": (_i64, [_i64, _i32]),
@@ -324,6 +325,35 @@ def mx_quant_rowwise_blocked_grouped(x, offs, mode="floor", *, capacity_rows=Non
                                                 _ptr(scales), capacity_rows, _ptr(group_row_starts), _stream(dev))
     _check("mx_quant_rowwise_blocked_grouped", rc)
     return out.view(torch.float8_e4m3fn), scales, group_row_starts
+
+
+# ---------------------------------------------------------------- GEMM
+
+def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, *, out=None):
+    """Grouped GEMM on the tensor cores: out[m] = (a[m] . w[g]^T) * inv_a[m] *
+    inv_w[g] for the rows m of group g. a (M, K) e4m3 row-major, inv_a (M,)
+    fp32, w (E, N, K) e4m3, inv_w (E, N) fp32, offs (E,) int32 group ends
+    along M. Returns out (M, N) bf16; rows past offs[-1] are not written."""
+    for t, n in ((a, "a"), (inv_a, "inv_a"), (w, "w"), (inv_w, "inv_w")):
+        _cuda(t, n)
+        if not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous")
+    if a.element_size() != 1 or w.element_size() != 1 or a.dim() != 2 or w.dim() != 3:
+        raise TypeError("a must be (M, K) and w (E, N, K), one byte per element (e4m3)")
+    if inv_a.dtype != torch.float32 or inv_w.dtype != torch.float32:
+        raise TypeError("inv_a and inv_w must be float32")
+    dev = a.device
+    _offsets(offs, dev)
+    M, K = a.shape
+    E, N, K2 = w.shape
+    if K2 != K or offs.numel() != E or inv_a.numel() != M or inv_w.numel() != E * N:
+        raise TypeError("shape mismatch between a, w, inv_a, inv_w and offs")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    rc = lib().fp8_grouped_gemm_rowwise(_ptr(a), _ptr(inv_a), _ptr(w), _ptr(inv_w), M, N, K, _ptr(offs), E,
+                                        _ptr(out), _stream(dev))
+    _check("fp8_grouped_gemm_rowwise", rc)
+    return out
 
 
 # ---------------------------------------------------------------- status

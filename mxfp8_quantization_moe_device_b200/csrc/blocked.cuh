@@ -33,8 +33,9 @@ constexpr int MAX_G = 4096;
 
 // padded start of every group in units of 2^shift: T[g] = sum_{h<g}
 // ceil(size_h / 2^shift) (shift 7: tile rows of 128; shift 2: tile columns of
-// 4), by a block scan in chunks of THREADS groups (warp shuffles plus one
-// step across warps); returns false on bad offsets
+// 4), by a block scan in chunks of blockDim.x groups (warp shuffles plus one
+// step across warps; blockDim.x a multiple of 32, at most THREADS); returns
+// false on bad offsets
 MXQ_DEV bool padded_starts(const int32_t *__restrict__ offs, int G, int64_t extent, int shift, int *T, int *Tend)
 {
     using namespace blk;
@@ -46,7 +47,7 @@ MXQ_DEV bool padded_starts(const int32_t *__restrict__ offs, int G, int64_t exte
     if (threadIdx.x == 0)
         carry = 0;
     __syncthreads();
-    for (int g0 = 0; g0 < G; g0 += THREADS) {
+    for (int g0 = 0; g0 < G; g0 += blockDim.x) {
         const int g = g0 + threadIdx.x;
         const int n = g < G ? (offs[g] - (g ? offs[g - 1] : 0) + (1 << shift) - 1) >> shift : 0;
         int x = n; // inclusive warp scan
@@ -65,7 +66,7 @@ MXQ_DEV bool padded_starts(const int32_t *__restrict__ offs, int G, int64_t exte
         if (g < G)
             T[g] = before + x - n;
         __syncthreads();
-        if (threadIdx.x == THREADS - 1)
+        if (threadIdx.x == blockDim.x - 1)
             carry = before + x;
         __syncthreads();
     }

@@ -11,6 +11,7 @@
 #include "mx3d.cuh"
 #include "jagged.cuh"
 #include "blocked.cuh"
+#include "gemm.cuh"
 
 using namespace mxq;
 
@@ -97,6 +98,8 @@ int device_info(const DevInfo **out)
                                  (int)mx3d::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_blockwise_t, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)bt::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gm::SMEM_FIXED + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_jagged_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)jag::cst::SMEM_BYTES) != cudaSuccess)
             return MXQ_ERR_CUDA;
@@ -354,6 +357,48 @@ int fp8_quant_blockwise_transposed(const void *in, int64_t rows, int64_t cols, i
     const int64_t grid = std::min<int64_t>(items, (int64_t)di->sms * bt::CTAS_PER_SM);
     return launch(k_fp8_blockwise_t, dim3((unsigned)grid), dim3(bt::THREADS), bt::SMEM_BYTES, stream, false, tin,
                   tout, inv_scales, rows, cols, (int)block_cols, wait_ns());
+}
+
+int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, const float *inv_w, int64_t M,
+                             int64_t N, int64_t K, const int32_t *offs, int32_t num_groups, void *out,
+                             cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % gm::BN || K % gm::BK)
+        return MXQ_ERR_SHAPE;
+    if (num_groups > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0)
+        return MXQ_OK;
+    if (K == 0)
+        return MXQ_ERR_SHAPE;
+    if (!a || !inv_a || !w || !inv_w || !offs || !out)
+        return MXQ_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(w, 16) || !aligned(out, 16) || !aligned(inv_a, 4) || !aligned(inv_w, 4))
+        return MXQ_ERR_ALIGN;
+    if (M >= (int64_t(1) << 31) || (int64_t)num_groups * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    CUtensorMap ta, tw;
+    const uint64_t da[2] = {(uint64_t)K, (uint64_t)M};
+    const uint64_t sa[1] = {(uint64_t)K};
+    const uint32_t box[2] = {gm::BK, gm::BM};
+    rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t dw[2] = {(uint64_t)K, (uint64_t)(num_groups * N)};
+    const uint32_t boxw[2] = {gm::BK, gm::BN};
+    rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, dw, sa, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    // work items: at most (M / 128 + G) m-tiles times N / 128 n-tiles
+    const int64_t items = (M / gm::BM + num_groups) * (N / gm::BN);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, di->sms));
+    return launch(k_fp8_grouped_gemm, dim3((unsigned)grid), dim3(gm::THREADS),
+                  gm::SMEM_FIXED + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M, N, K, offs,
+                  (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
 }
 
 int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t mode, void *out, uint8_t *scales,

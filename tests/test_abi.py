@@ -86,6 +86,13 @@ def test_host_checks_return_before_any_cuda_call(lib):
     assert lib.fp8_quant_blockwise(odd, 128, 128, 1, 128, fake, fake, null) == binding.ERR_ALIGN
     assert lib.mx_quant_3d_colwise(fake, 1, 64, 60, 0, fake, fake, null) == binding.ERR_ALIGN
     assert lib.mx_scales_to_blocked_grouped(fake, 4, 4, fake, 1, odd, 128, null, null) == binding.ERR_ALIGN
+    # grouped GEMM
+    assert lib.fp8_grouped_gemm_rowwise(fake, fake, fake, fake, 128, 100, 128, fake, 1, fake, null) == binding.ERR_SHAPE
+    assert lib.fp8_grouped_gemm_rowwise(fake, fake, fake, fake, 128, 128, 96, fake, 1, fake, null) == binding.ERR_SHAPE
+    assert lib.fp8_grouped_gemm_rowwise(fake, fake, fake, fake, 128, 128, 128, fake, 5000, fake, null) == \
+        binding.ERR_UNSUPPORTED
+    assert lib.fp8_grouped_gemm_rowwise(fake, null, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_NULL
+    assert lib.fp8_grouped_gemm_rowwise(odd, fake, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_ALIGN
     # blockwise with transposed output
     assert lib.fp8_quant_blockwise_transposed(fake, 128, 128, 1, 128, fake, fake, null) == binding.ERR_UNSUPPORTED
     assert lib.fp8_quant_blockwise_transposed(fake, 128, 128, 128, 64, fake, fake, null) == binding.ERR_UNSUPPORTED

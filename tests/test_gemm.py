@@ -1,0 +1,101 @@
+"""Grouped GEMM on the tensor cores (tcgen05) against the fp64 oracle.
+
+Tolerance, per element (derived from the arithmetic, stated here): the kernel
+accumulates the exact e4m3 products in fp32 on the tensor cores, multiplies by
+the two fp32 scales and rounds to bf16. With S = (sum_k |a_k w_k|) * inv_a *
+inv_w, the fp32 accumulation error is at most K * 2^-24 * S (the gamma_K bound
+of a sum of K terms, with a factor 2 of slack: K * 2^-23 * S); the two scale
+multiplications add at most 2^-23 |ref|; rounding to bf16 adds at most half a
+bf16 ulp, 2^-9 |result|. So |out - ref| <= 2^-8 |ref| + K * 2^-23 * S.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp8_quantization_moe_device_b200 import binding as mxq
+from mxfp8_quantization_moe_device_b200 import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    mxq.lib()
+    mxq.testing_set(mxq.TESTING_WAIT_LIMIT_NS, 200_000_000)
+    yield
+    mxq.testing_set(mxq.TESTING_WAIT_LIMIT_NS, 0)
+
+
+def _operands(M, N, K, E, seed):
+    """A (M, K) and W (E, N, K) quantized by this library's rowwise op with
+    one group spanning K: e4m3 codes and per-row inverse scales."""
+    a = synth.row_scaled_normal_bf16(M, K, seed=seed, device=DEV)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=seed + 1, device=DEV, lo=-2.0, hi=2.0)
+    kk = torch.tensor([K], dtype=torch.int32, device=DEV)
+    aq, ia = mxq.fp8_quant_jagged_rowwise(a, kk)
+    wq, iw = mxq.fp8_quant_jagged_rowwise(w, kk)
+    return aq.view(torch.uint8), ia.reshape(M).contiguous(), wq.view(torch.uint8).reshape(E, N, K), \
+        iw.reshape(E, N).contiguous()
+
+
+def _check(out, aq, ia, wq, iw, offs, K):
+    a_c, w_c = aq.cpu().numpy(), wq.cpu().numpy()
+    ia_n, iw_n, o = ia.cpu().numpy(), iw.cpu().numpy(), offs.cpu().numpy()
+    ref = oracle.fp8_grouped_gemm_rowwise(a_c, ia_n, w_c, iw_n, o)
+    dec = np.abs(np.array([oracle.e4m3_value(c) for c in range(256)]))
+    absref = np.zeros_like(ref)
+    start = 0
+    for g, end in enumerate(o):
+        if end > start:
+            S = (dec[a_c[start:end]] @ dec[w_c[g]].T) * ia_n[start:end, None] * iw_n[g][None, :]
+            absref[start:end] = S
+        start = end
+    end = int(o[-1])
+    got = out[:end].float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref[:end])
+    bound = 2.0 ** -8 * np.abs(ref[:end]) + K * 2.0 ** -23 * absref[:end]
+    worst = np.max(err - bound)
+    assert worst <= 0, f"max excess over the bound {worst}"
+
+
+@pytest.mark.parametrize("M,N,K,ends", [
+    (300, 128, 256, [100, 100, 290]),          # an empty group; rows past the last group
+    (129, 256, 128, [1, 129]),                 # a one-row group; K of one stage
+    (1000, 384, 1024, [250, 300, 700, 1000]),
+])
+def test_grouped_gemm_vs_oracle(M, N, K, ends):
+    E = len(ends)
+    aq, ia, wq, iw = _operands(M, N, K, E, seed=M + N)
+    offs = torch.tensor(ends, dtype=torch.int32, device=DEV)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mxq.fp8_grouped_gemm_rowwise(aq, ia, wq, iw, offs, out=out)
+    assert mxq.device_status() == 0
+    _check(out, aq, ia, wq, iw, offs, K)
+    assert bool(torch.isnan(out[ends[-1]:]).all())  # rows past the last group untouched
+
+
+def test_grouped_gemm_moe_shape_sampled():
+    """An MoE-like case: (8192 tokens, K 2048) x 8 experts of N 1024, Dirichlet
+    groups; every output row of a few groups checked against the oracle."""
+    M, N, K, E = 8192, 1024, 2048, 8
+    aq, ia, wq, iw = _operands(M, N, K, E, seed=77)
+    offs = synth.dirichlet_offsets(M, E, 0.5, 78).to(DEV)
+    out = mxq.fp8_grouped_gemm_rowwise(aq, ia, wq, iw, offs)
+    assert mxq.device_status() == 0
+    o = offs.cpu().numpy()
+    sel = []
+    for g in range(E):
+        a = int(o[g - 1]) if g else 0
+        sel += list(range(a, min(a + 3, int(o[g]))))
+    rows = torch.tensor(sel, dtype=torch.long)
+    # the oracle on the selected rows only (each row keeps its group)
+    a_sel = aq.cpu()[rows].numpy()
+    ia_sel = ia.cpu()[rows].numpy()
+    groups = np.searchsorted(o, np.array(sel), side="right")
+    ends = np.array([np.sum(groups <= g) for g in range(E)], dtype=np.int32)
+    sub = torch.from_numpy(ends).to(DEV)
+    _check(out[rows.to(DEV)], torch.from_numpy(a_sel), torch.from_numpy(ia_sel), wq, iw, sub, K)
