@@ -439,8 +439,57 @@ def per_shape_sweep(wl, reps):
                 wl.tok, wl.offs64, mode, capacity_rows=wl.cap, out=wl.o["tok_q"], scales=sbuf,
                 group_row_starts=st),
             65536 * 7168 * 3 + wl.cap * tc * 4)
+    # grouped GEMM on the tensor cores, fed by the rowwise quantization:
+    # tokens (65536, 7168) in the 64 Dirichlet(0.3) groups x 64 experts (2048, 7168)
+    rows += gemm_rows(wl, flush, reps)
     del flush
     return rows
+
+
+def gemm_rows(wl, flush, reps):
+    """TFLOP/s of fp8_grouped_gemm_rowwise on the MoE shape, against the FP8
+    dense peak taken as the measured bf16 GEMM peak times the nominal FP8/bf16
+    ratio of 2."""
+    torch, mxq = wl.torch, wl.mxq
+    from mxfp8_quantization_moe_device_b200 import synth
+    dev = wl.dev
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        kind = "measured bf16 x 2"
+    except Exception:
+        bf16, kind = 1590.0, "fallback bf16 x 2"
+    fp8_peak = 2.0 * bf16
+    T, K = wl.tok.shape
+    E, N = 64, 2048
+    kk = torch.tensor([K], dtype=torch.int32, device=dev)
+    aq, ia = mxq.fp8_quant_jagged_rowwise(wl.tok, kk)
+    w = synth.normal_bf16((E * N, K), 0.02, seed=12, device=dev)
+    wq, iw = mxq.fp8_quant_jagged_rowwise(w, kk)
+    del w
+    aq, ia = aq.view(torch.uint8), ia.reshape(T).contiguous()
+    wq, iw = wq.view(torch.uint8).reshape(E, N, K), iw.reshape(E, N).contiguous()
+    out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    fn = lambda: mxq.fp8_grouped_gemm_rowwise(aq, ia, wq, iw, wl.offs64, out=out)
+    for _ in range(5):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush_l2(torch, flush)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    us = statistics.median(ts)
+    flops = 2.0 * T * N * K
+    tf = flops / (us * 1e-6) / 1e12
+    return [{"op": "fp8_grouped_gemm", "shape": f"({T},{K}) G=64 x (64,{N},{K})", "us": round(us, 3),
+             "TFLOP/s": round(tf, 1), "frac_fp8_peak": round(tf / fp8_peak, 4), "peak_TFLOP/s": round(fp8_peak, 1),
+             "peak_kind": kind}]
 
 
 # ----------------------------------------------------------------- oracle side

@@ -14,13 +14,14 @@
 // Design: a persistent grid, one CTA per SM, walks (m-tile, n-tile) work items
 // with n fastest; a group's m-tiles start at its first row, so a tile never
 // mixes experts (rows past the group's end are computed and dropped).
-//   warp 4       TMA producer: 128 x 128-byte tiles of A and W (128B swizzle)
-//                into a 4-stage ring;
-//   warp 5       allocates 256 TMEM columns (two 128 x 128 fp32 accumulators)
-//                and, from one thread, issues tcgen05.mma kind::f8f6f4
-//                (M 128, N 128, K 32) four times per stage, releasing each
-//                stage with tcgen05.commit and handing a finished
-//                accumulator to the epilogue the same way;
+//   warp 4       TMA producer: 128 x 128-byte tiles of A and BN x 128-byte
+//                tiles of W (128B swizzle) into a 4-stage ring; BN = 256 when
+//                N allows, else 128;
+//   warp 5       allocates 2 * BN TMEM columns (two 128 x BN fp32
+//                accumulators) and, from one thread, issues tcgen05.mma
+//                kind::f8f6f4 (M 128, N BN, K 32) four times per stage,
+//                releasing each stage with tcgen05.commit and handing a
+//                finished accumulator to the epilogue the same way;
 //   warps 0-3    epilogue: tcgen05.ld of their 32 TMEM lanes (rows), scale,
 //                round to bf16, store; the accumulator is then released, so
 //                the next tile's MMAs overlap this tile's epilogue.
@@ -34,17 +35,17 @@
 namespace mxq {
 namespace gm {
 
-constexpr int BM = 128, BN = 128, BK = 128; // BK in bytes = e4m3 elements
+constexpr int BM = 128, BK = 128; // BK in bytes = e4m3 elements
 constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK;            // 16 KB
-constexpr int B_BYTES = BN * BK;            // 16 KB
+constexpr int A_BYTES = BM * BK;  // 16 KB
 constexpr int THREADS = 6 * 32;
-constexpr int ACC = 2;                      // accumulators in TMEM
-constexpr int TMEM_COLS = ACC * BN;         // 256
+constexpr int ACC = 2;            // accumulators in TMEM
 
-struct __align__(1024) Smem {
+// tile width BN (128 or 256): a stage holds the A tile and a BN x 128-byte W
+// tile; two BM x BN fp32 accumulators take 2 * BN TMEM columns
+template <int BN> struct __align__(1024) Smem {
     uint8_t a[STAGES][A_BYTES];
-    uint8_t b[STAGES][B_BYTES];
+    uint8_t b[STAGES][BN * BK];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t acc_full[ACC];
@@ -54,7 +55,7 @@ struct __align__(1024) Smem {
     int abort_flag;
     int Tend;
 };
-constexpr size_t SMEM_FIXED = sizeof(Smem) + 1024;
+template <int BN> constexpr size_t smem_fixed() { return sizeof(Smem<BN>) + 1024; }
 
 // shared-memory matrix descriptor of a K-major tile of 128-byte rows stored
 // with the 128-byte swizzle (8-row groups 1024 bytes apart): start address,
@@ -67,21 +68,21 @@ MXQ_DEV uint64_t smem_desc_k128(uint32_t addr)
 }
 
 // instruction descriptor: fp32 accumulator, e4m3 x e4m3, both K-major, N, M
-constexpr uint32_t IDESC = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                           ((uint32_t)(BM >> 4) << 24);
+template <int BN>
+constexpr uint32_t idesc() { return (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24); }
 
 MXQ_DEV int aborted(const int *flag) { return *reinterpret_cast<const volatile int *>(flag); }
 
 MXQ_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 MXQ_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-MXQ_DEV void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+MXQ_DEV void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -116,6 +117,7 @@ MXQ_DEV uint32_t pack_bf16x2(float lo, float hi)
 
 } // namespace gm
 
+template <int BN>
 __global__ void __launch_bounds__(gm::THREADS, 1)
     k_fp8_grouped_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                        const float *__restrict__ inv_a, const float *__restrict__ inv_w, int64_t M, int64_t N,
@@ -123,8 +125,11 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
                        uint64_t wait_ns)
 {
     using namespace gm;
+    constexpr int B_BYTES = BN * BK;
+    constexpr int TMEM_COLS = ACC * BN;
+    constexpr uint32_t IDESC = idesc<BN>();
     extern __shared__ uint8_t smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<BN> &sm = *reinterpret_cast<Smem<BN> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     int *T = reinterpret_cast<int *>(&sm + 1); // G group m-tile starts, after the fixed part
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -221,7 +226,7 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
                     const uint64_t bd = smem_desc_k128(smem_u32(sm.b[s]));
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k) // K 32 per instruction: +32 bytes = +2 in the address field
-                        tc_mma(d, ad + 2 * k, bd + 2 * k, (kb > 0 || k > 0) ? 1u : 0u);
+                        tc_mma(d, ad + 2 * k, bd + 2 * k, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
                     issued = true;
                     tc_commit(&sm.empty[s]); // the stage is free once these MMAs are done
                 }

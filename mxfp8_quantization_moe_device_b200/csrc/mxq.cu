@@ -98,8 +98,10 @@ int device_info(const DevInfo **out)
                                  (int)mx3d::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_blockwise_t, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)bt::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(k_fp8_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(gm::SMEM_FIXED + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_grouped_gemm<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gm::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_grouped_gemm<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gm::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_jagged_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)jag::cst::SMEM_BYTES) != cudaSuccess)
             return MXQ_ERR_CUDA;
@@ -363,7 +365,7 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
                              int64_t N, int64_t K, const int32_t *offs, int32_t num_groups, void *out,
                              cudaStream_t stream)
 {
-    if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % gm::BN || K % gm::BK)
+    if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % 128 || K % gm::BK)
         return MXQ_ERR_SHAPE;
     if (num_groups > blk::MAX_G)
         return MXQ_ERR_UNSUPPORTED;
@@ -388,17 +390,23 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
     rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
+    // tiles 128 x 256 when N allows, else 128 x 128
+    const int bn = N % 256 == 0 ? 256 : 128;
     const uint64_t dw[2] = {(uint64_t)K, (uint64_t)(num_groups * N)};
-    const uint32_t boxw[2] = {gm::BK, gm::BN};
+    const uint32_t boxw[2] = {gm::BK, (uint32_t)bn};
     rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, dw, sa, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
-    // work items: at most (M / 128 + G) m-tiles times N / 128 n-tiles
-    const int64_t items = (M / gm::BM + num_groups) * (N / gm::BN);
+    // work items: at most (M / 128 + G) m-tiles times N / bn n-tiles
+    const int64_t items = (M / gm::BM + num_groups) * (N / bn);
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, di->sms));
-    return launch(k_fp8_grouped_gemm, dim3((unsigned)grid), dim3(gm::THREADS),
-                  gm::SMEM_FIXED + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M, N, K, offs,
-                  (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+    if (bn == 256)
+        return launch(k_fp8_grouped_gemm<256>, dim3((unsigned)grid), dim3(gm::THREADS),
+                      gm::smem_fixed<256>() + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M,
+                      N, K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+    return launch(k_fp8_grouped_gemm<128>, dim3((unsigned)grid), dim3(gm::THREADS),
+                  gm::smem_fixed<128>() + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M, N,
+                  K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
 }
 
 int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t mode, void *out, uint8_t *scales,
