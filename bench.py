@@ -81,7 +81,7 @@ KERNEL_FILES = {  # source files that define each kernel (plus common.cuh)
     "k_fp8_1x128": "rowblock.cuh", "k_fp8_128x128": "rowblock.cuh", "k_mx_1x32": "rowblock.cuh",
     "k_jagged_amax": "jagged.cuh", "k_jagged_cast": "jagged.cuh", "k_mx_3d_colwise": "mx3d.cuh",
     "k_blocked_grouped": "blocked.cuh", "k_blocked_grouped_k": "blocked.cuh", "k_mx_1x32_blocked": "blocked.cuh",
-    "k_fp8_blockwise_t": "blockt.cuh",
+    "k_fp8_blockwise_t": "blockt.cuh", "k_fp8_grouped_gemm": "gemm.cuh",
 }
 
 
@@ -173,7 +173,7 @@ class Workload:
     OPS = ("blockwise_1x128", "blockwise_128x128", "jagged_rowwise", "jagged_colwise", "mx_3d_colwise",
            "mx_rowwise", "blocked_grouped")
     # ops outside the step (the widened rows), built only when asked for by name
-    EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked")
+    EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked", "grouped_gemm")
 
     def __init__(self, dev, experts, mx3d_mode, only=None):
         import torch
@@ -268,6 +268,22 @@ class Workload:
             self.ops.append(("mx_rowwise_blocked", lambda: mxq.mx_quant_rowwise_blocked_grouped(
                 self.tok, self.offs64, "floor", capacity_rows=self.cap, out=self.o["tok_q"], scales=self.o["tok_sb"],
                 group_row_starts=self.o["tok_sb_starts"]), T * KT * 3 + sbytes))
+
+        if "grouped_gemm" in want:
+            # tokens (16384, 7168) in 16 Dirichlet(0.3) groups x 16 experts (2048, 7168): a 1 GB capture
+            T, K, E, N = 16384, 7168, 16, 2048
+            x = synth.normal_bf16((T, K), 1.0, seed=7, device=dev)
+            w = synth.normal_bf16((E * N, K), 0.02, seed=12, device=dev)
+            kk = t.tensor([K], dtype=t.int32, device=dev)
+            aq, ia = mxq.fp8_quant_jagged_rowwise(x, kk)
+            wq, iw = mxq.fp8_quant_jagged_rowwise(w, kk)
+            del x, w
+            self.g_a, self.g_ia = aq.view(t.uint8), ia.reshape(T).contiguous()
+            self.g_w, self.g_iw = wq.view(t.uint8).reshape(E, N, K), iw.reshape(E, N).contiguous()
+            self.g_offs = synth.dirichlet_offsets(T, E, 0.3, 8).to(dev)
+            self.o.update(g_out=t.empty((T, N), dtype=t.bfloat16, device=dev))
+            self.ops.append(("grouped_gemm", lambda: mxq.fp8_grouped_gemm_rowwise(
+                self.g_a, self.g_ia, self.g_w, self.g_iw, self.g_offs, out=self.o["g_out"]), 2 * T * N * K))
 
     def step_bytes(self):
         return sum(b for _, _, b in self.ops)
