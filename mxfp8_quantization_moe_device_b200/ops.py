@@ -212,3 +212,23 @@ def _(x, offs, mode):
     return (x.new_empty((rows, cols), dtype=_F8),
             x.new_empty((_rows_cap(rows, G) * ((cols + 127) // 128) * 4,), dtype=torch.uint8),
             x.new_empty((G,), dtype=torch.int32))
+
+
+# ---------------------------------------------------------------- GEMM
+
+@torch.library.custom_op("mxq::fp8_grouped_gemm_rowwise", mutates_args=())
+def fp8_grouped_gemm_rowwise(a: torch.Tensor, inv_a: torch.Tensor, w: torch.Tensor, inv_w: torch.Tensor,
+                             offs: torch.Tensor) -> torch.Tensor:
+    """Grouped GEMM on the tensor cores: (M, N) bf16, row m of group g =
+    (a[m] . w[g]^T) * inv_a[m] * inv_w[g]; rows past offs[-1] are zero."""
+    M = a.shape[0]
+    N = w.shape[1]
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device=a.device)
+    _b.fp8_grouped_gemm_rowwise(a.view(torch.uint8), inv_a, w.view(torch.uint8), inv_w, offs, out=out)
+    return out
+
+
+@fp8_grouped_gemm_rowwise.register_fake
+def _(a, inv_a, w, inv_w, offs):
+    return a.new_empty((a.shape[0], w.shape[1]), dtype=torch.bfloat16)
+

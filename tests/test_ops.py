@@ -11,7 +11,7 @@ from mxfp8_quantization_moe_device_b200 import synth
 
 OPS = ["fp8_quant_jagged_rowwise", "fp8_quant_jagged_colwise", "fp8_quant_blockwise",
        "fp8_quant_blockwise_transposed", "mx_quant_3d_colwise", "mx_quant_rowwise", "mx_scales_to_blocked_grouped",
-       "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped"]
+       "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped", "fp8_grouped_gemm_rowwise"]
 
 
 def _cases(dev):
@@ -45,6 +45,15 @@ def _meta(t):
 def test_every_op_is_registered():
     for name in OPS:
         assert hasattr(torch.ops.mxq, name), name
+
+
+def test_gemm_fake_shape_on_meta_tensors():
+    a = torch.empty((300, 256), dtype=torch.float8_e4m3fn, device="meta")
+    w = torch.empty((3, 128, 256), dtype=torch.float8_e4m3fn, device="meta")
+    out = torch.ops.mxq.fp8_grouped_gemm_rowwise(a, torch.empty(300, device="meta"), w,
+                                                 torch.empty((3, 128), device="meta"),
+                                                 torch.empty(3, dtype=torch.int32, device="meta"))
+    assert tuple(out.shape) == (300, 128) and out.dtype == torch.bfloat16
 
 
 def test_fake_shapes_on_meta_tensors():
@@ -99,6 +108,22 @@ def test_registered_ops_match_the_binding():
         assert mxq.device_status() == 0
         for g, r in zip(got, ref):
             assert torch.equal(_bytes(g), _bytes(r)), name
+
+
+@gpu
+def test_gemm_op_matches_the_binding():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    kk = torch.tensor([256], dtype=torch.int32, device="cuda")
+    a, ia = mxq.fp8_quant_jagged_rowwise(synth.normal_bf16((300, 256), 1.0, seed=1, device="cuda"), kk)
+    w, iw = mxq.fp8_quant_jagged_rowwise(synth.normal_bf16((3 * 128, 256), 0.02, seed=2, device="cuda"), kk)
+    offs = torch.tensor([100, 100, 290], dtype=torch.int32, device="cuda")
+    got = torch.ops.mxq.fp8_grouped_gemm_rowwise(a, ia.reshape(300), w.reshape(3, 128, 256), iw.reshape(3, 128), offs)
+    ref = torch.zeros_like(got)
+    mxq.fp8_grouped_gemm_rowwise(a.view(torch.uint8), ia.reshape(300).contiguous(),
+                                 w.view(torch.uint8).reshape(3, 128, 256), iw.reshape(3, 128).contiguous(), offs,
+                                 out=ref)
+    assert torch.equal(got, ref)
 
 
 @gpu
