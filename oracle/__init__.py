@@ -49,6 +49,8 @@ def lib():
             "oracle_fp8_quant_blockwise_transposed": (ctypes.c_int, [_u16p, _i64, _i64, _i32, _i32, _u8p, _f32p]),
             "oracle_fp8_grouped_gemm_rowwise": (ctypes.c_int, [_u8p, _f32p, _u8p, _f32p, _i64, _i64, _i64, _i32p,
                                                                _i32, ctypes.POINTER(ctypes.c_double)]),
+            "oracle_fp8_grouped_gemm_wgrad": (ctypes.c_int, [_u8p, _f32p, _u8p, _f32p, _i64, _i64, _i64, _i32p,
+                                                             _i32, ctypes.POINTER(ctypes.c_double)]),
             "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
@@ -191,6 +193,24 @@ def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, out=None):
     res = np.zeros((M, N), dtype=np.float64) if out is None else np.ascontiguousarray(out, dtype=np.float64)
     _check(lib().oracle_fp8_grouped_gemm_rowwise(_p(a, _u8p), _p(ia, _f32p), _p(w, _u8p), _p(iw, _f32p), M, N, K,
                                                  _p(o, _i32p), E, res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return res
+
+
+def fp8_grouped_gemm_wgrad(a, inv_a, b, inv_b, offs):
+    """a (N, M) and b (K, M) e4m3 codes (M contiguous), inv_a (G, N), inv_b
+    (G, K), offs (G,) ends along M. Returns out (G, N, K) float64."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    ia = np.ascontiguousarray(inv_a, dtype=np.float32)
+    ib = np.ascontiguousarray(inv_b, dtype=np.float32)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    N, M = a.shape
+    K, M2 = b.shape
+    assert M2 == M and ia.shape == (len(o), N) and ib.shape == (len(o), K)
+    res = np.zeros((len(o), N, K), dtype=np.float64)
+    _check(lib().oracle_fp8_grouped_gemm_wgrad(_p(a, _u8p), _p(ia, _f32p), _p(b, _u8p), _p(ib, _f32p), N, K, M,
+                                               _p(o, _i32p), len(o),
+                                               res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
     return res
 
 

@@ -556,3 +556,37 @@ int oracle_fp8_grouped_gemm_rowwise(const uint8_t *a, const float *inv_a, const 
     return 0;
 }
 
+/* ------------------------------------------------------------------ */
+/* Weight-gradient grouped GEMM, the backward consumer of the jagged    */
+/* ops (#2064 Summary: the per-group scaled operands of the grad_weight */
+/* grouped GEMM). The contraction runs over each group's own positions: */
+/*   out[g][n][k] = (sum_{m in group g} e4m3(a[n][m]) * e4m3(b[k][m]))   */
+/*                  * inv_a[g][n] * inv_b[g][k]                          */
+/* with a (N, M) = grad_out^T quantized rowwise per (row, group) and    */
+/* b (K, M) = the input quantized colwise per (column, group), both     */
+/* stored with M contiguous. Empty groups give zeros. In double.        */
+/* ------------------------------------------------------------------ */
+int oracle_fp8_grouped_gemm_wgrad(const uint8_t *a, const float *inv_a, const uint8_t *b, const float *inv_b,
+                                  int64_t N, int64_t K, int64_t M, const int32_t *offs, int32_t groups,
+                                  double *out)
+{
+    int64_t start = 0;
+    if (M < 0 || N < 0 || K < 0 || groups <= 0)
+        return ORACLE_ERR_ARG;
+    if (!offsets_valid(offs, groups, M))
+        return ORACLE_ERR_OFFSETS;
+    for (int32_t g = 0; g < groups; ++g) {
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t k = 0; k < K; ++k) {
+                double acc = 0.0;
+                for (int64_t m = start; m < offs[g]; ++m)
+                    acc += oracle_e4m3_value(a[n * M + m]) * oracle_e4m3_value(b[k * M + m]);
+                out[((int64_t)g * N + n) * K + k] =
+                    acc * (double)inv_a[(int64_t)g * N + n] * (double)inv_b[(int64_t)g * K + k];
+            }
+        }
+        start = offs[g];
+    }
+    return 0;
+}
+

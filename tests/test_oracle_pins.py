@@ -456,6 +456,31 @@ def test_grouped_gemm_hand_example(oracle):
     assert got[0, 0] == -2.75
 
 
+def test_wgrad_gemm_vs_numpy_matmul(oracle):
+    """The weight-gradient GEMM against numpy's float64 matmul of the decoded
+    values over each group's columns, scales applied afterwards; an empty group
+    gives zeros."""
+    rng = np.random.default_rng(13)
+    N, K, M = 20, 12, 90
+    a = rng.integers(0, 256, size=(N, M), dtype=np.uint8)
+    b = rng.integers(0, 256, size=(K, M), dtype=np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0
+    b[(b & 0x7F) == 0x7F] = 0
+    offs = np.array([17, 17, 60, 85], dtype=np.int32)   # an empty group; columns 85.. in no group
+    ia = rng.uniform(0.5, 2.0, (4, N)).astype(np.float32)
+    ib = rng.uniform(0.5, 2.0, (4, K)).astype(np.float32)
+    got = oracle.fp8_grouped_gemm_wgrad(a, ia, b, ib, offs)
+    dec = np.array([oracle.e4m3_value(c) for c in range(256)])
+    A, B = dec[a], dec[b]
+    start = 0
+    for g, end in enumerate(offs):
+        ref = (A[:, start:end] @ B[:, start:end].T) * ia[g][:, None].astype(np.float64) * \
+            ib[g][None, :].astype(np.float64)
+        assert np.allclose(got[g], ref, rtol=1e-13, atol=0)
+        start = end
+    assert not got[1].any()
+
+
 def test_rowwise_blocked_is_rowwise_then_conversion(oracle):
     rng = np.random.default_rng(3)
     x = torch.from_numpy(rng.standard_normal((300, 96)).astype(np.float32)).to(torch.bfloat16)
