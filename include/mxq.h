@@ -181,6 +181,26 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
                              cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * fp8_grouped_gemm_wgrad - the backward consumer of the jagged ops (#2064
+ * Summary: the per-group scaled operands of the grad_weight grouped GEMM),
+ * on the tensor cores:
+ *   out[g][n][k] = bf16((sum_{m in group g} a[n][m] * b[k][m])
+ *                       * inv_a[g][n] * inv_b[g][k])
+ *   a       e4m3 (N, M) row-major (M contiguous): fp8_quant_jagged_rowwise
+ *           of grad_out^T; inv_a fp32 (num_groups, N), its inverse scales.
+ *   b       e4m3 (K, M) row-major: the buffer of fp8_quant_jagged_colwise of
+ *           the input; inv_b fp32 (num_groups, K).
+ *   offs    num_groups int32 ends along M (device).
+ *   out     bf16 (num_groups, N, K); empty groups give zeros.
+ *   N % 128 == 0, K % 128 == 0, M % 16 == 0, else MXQ_ERR_SHAPE; a, b, out
+ *   16-byte aligned.
+ * ------------------------------------------------------------------------ */
+int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, const float *inv_b,
+                           int64_t N, int64_t K, int64_t M,
+                           const int32_t *offs, int32_t num_groups, void *out,
+                           cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * (a4) mx_quant_3d_colwise - #3002 Summary: MXFP8 quantization of expert
  * weights (E, N, K) along N in 32 x 1 blocks, written straight into each
  * expert's column-major layout.

@@ -38,6 +38,7 @@ SIGNATURES = {
     "fp8_quant_blockwise_transposed": (ctypes.c_int, [_vp, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "fp8_grouped_gemm_rowwise": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
+    "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
     "mx_blocked_grouped_rows_bound": (_i64, [_i64, _i32]),
@@ -353,6 +354,36 @@ def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, *, out=None):
     rc = lib().fp8_grouped_gemm_rowwise(_ptr(a), _ptr(inv_a), _ptr(w), _ptr(inv_w), M, N, K, _ptr(offs), E,
                                         _ptr(out), _stream(dev))
     _check("fp8_grouped_gemm_rowwise", rc)
+    return out
+
+
+def fp8_grouped_gemm_wgrad(a, inv_a, b, inv_b, offs, *, out=None):
+    """Weight-gradient grouped GEMM on the tensor cores: out[g] = (a[:, group
+    g] . b[:, group g]^T) * inv_a[g][:, None] * inv_b[g][None, :]. a (N, M)
+    and b (K, M) e4m3 with M contiguous (the buffers of
+    fp8_quant_jagged_rowwise on grad_out^T and fp8_quant_jagged_colwise on the
+    input), inv_a (G, N), inv_b (G, K), offs (G,) ends along M. Returns out
+    (G, N, K) bf16."""
+    for t, n in ((a, "a"), (inv_a, "inv_a"), (b, "b"), (inv_b, "inv_b")):
+        _cuda(t, n)
+        if not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous")
+    if a.element_size() != 1 or b.element_size() != 1 or a.dim() != 2 or b.dim() != 2:
+        raise TypeError("a must be (N, M) and b (K, M), one byte per element (e4m3)")
+    if inv_a.dtype != torch.float32 or inv_b.dtype != torch.float32:
+        raise TypeError("inv_a and inv_b must be float32")
+    dev = a.device
+    _offsets(offs, dev)
+    N, M = a.shape
+    K, M2 = b.shape
+    G = offs.numel()
+    if M2 != M or inv_a.numel() != G * N or inv_b.numel() != G * K:
+        raise TypeError("shape mismatch between a, b, inv_a, inv_b and offs")
+    if out is None:
+        out = torch.empty((G, N, K), dtype=torch.bfloat16, device=dev)
+    rc = lib().fp8_grouped_gemm_wgrad(_ptr(a), _ptr(inv_a), _ptr(b), _ptr(inv_b), N, K, M, _ptr(offs), G, _ptr(out),
+                                      _stream(dev))
+    _check("fp8_grouped_gemm_wgrad", rc)
     return out
 
 

@@ -293,4 +293,246 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Weight-gradient grouped GEMM, the backward consumer of the jagged ops:
+//
+//   out[g][n][k] = bf16( (sum_{m in group g} a[n][m] * b[k][m])
+//                        * inv_a[g][n] * inv_b[g][k] )
+//
+// a (N, M) is grad_out^T quantized rowwise with per-(row, group) scales, b
+// (K, M) the input quantized colwise with per-(column, group) scales; both
+// keep the grouped dimension M contiguous, so both are K-major operands of
+// the MMA and the contraction of group g runs over its own positions.
+//
+// Same roles as above, on (group, n-tile, k-tile) items. The producer streams
+// 128-position chunks of the group starting at the 16-aligned position at or
+// below its first one (TMA coordinates must be 16-byte aligned); where a chunk
+// reaches outside the group, the MMA warp zeroes those position columns of
+// both tiles in shared memory (the bytes past the last group are not data),
+// fences the async proxy, and only then issues the MMAs. Items of empty
+// groups write zeros.
+// ---------------------------------------------------------------------------
+namespace gm {
+
+// zero position columns outside [lo, hi) of a `rows` x 128-byte tile stored
+// with the 128-byte swizzle (byte c of row r at r*128 + ((c/16) ^ (r%8))*16 +
+// c%16); lane l of the warp takes rows l, l+32, ...
+MXQ_DEV void zero_outside(uint8_t *tile, int rows, int lo, int hi)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int r = lane; r < rows; r += 32) {
+        uint8_t *row = tile + r * 128;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+            uint8_t *chunk = row + ((c ^ (r & 7)) << 4);
+            const int b0 = 16 * c, b1 = b0 + 16;
+            if (b1 <= lo || b0 >= hi) {
+                *reinterpret_cast<uint4 *>(chunk) = make_uint4(0u, 0u, 0u, 0u);
+            } else if (b0 < lo || b1 > hi) {
+                for (int j = 0; j < 16; ++j)
+                    if (b0 + j < lo || b0 + j >= hi)
+                        chunk[j] = 0;
+            }
+        }
+    }
+}
+
+} // namespace gm
+
+template <int BN>
+__global__ void __launch_bounds__(gm::THREADS, 1)
+    k_fp8_grouped_gemm_wgrad(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                             const float *__restrict__ inv_a, const float *__restrict__ inv_b, int64_t N, int64_t K,
+                             int64_t M, const int32_t *__restrict__ offs, int G, uint16_t *__restrict__ out,
+                             uint64_t wait_ns)
+{
+    using namespace gm;
+    constexpr int B_BYTES = BN * BK;
+    constexpr int TMEM_COLS = ACC * BN;
+    constexpr uint32_t IDESC = idesc<BN>();
+    extern __shared__ uint8_t smem_raw[];
+    Smem<BN> &sm = *reinterpret_cast<Smem<BN> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int i = 0; i < ACC; ++i) {
+            mbar_init(&sm.acc_full[i], 1);
+            mbar_init(&sm.acc_empty[i], 4);
+        }
+        mbar_init(&sm.mma_done, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (!offsets_ok(offs, G, M))
+        return;
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    const int64_t ntn = N / BM, ktn = K / BN;
+    const int64_t per_g = ntn * ktn, total = per_g * G;
+    // item it -> group, tiles, the group's positions [s, e), first chunk x0
+    struct Item {
+        int g;
+        int64_t nt, kt, s, e, x0, nch;
+    };
+    auto item = [&](int64_t it) {
+        Item q;
+        q.g = (int)(it / per_g);
+        const int64_t rem = it - (int64_t)q.g * per_g;
+        q.nt = rem / ktn;
+        q.kt = rem - q.nt * ktn;
+        q.s = q.g ? offs[q.g - 1] : 0;
+        q.e = offs[q.g];
+        q.x0 = q.s & ~int64_t(15);
+        q.nch = q.e > q.s ? (q.e - q.x0 + BK - 1) / BK : 0;
+        return q;
+    };
+
+    if (warp == 4) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int seq = 0;
+            for (int64_t it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+                const Item q = item(it);
+                for (int64_t j = 0; j < q.nch; ++j, ++seq) {
+                    const int s = seq % STAGES;
+                    if (seq >= STAGES && !mbar_wait(&sm.empty[s], ((uint32_t)(seq / STAGES) & 1u) ^ 1u, wait_ns)) {
+                        *reinterpret_cast<volatile int *>(&sm.abort_flag) = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
+                    tma_load_2d(sm.a[s], &tm_a, &sm.full[s], (int)(q.x0 + j * BK), (int)(q.nt * BM));
+                    tma_load_2d(sm.b[s], &tm_b, &sm.full[s], (int)(q.x0 + j * BK), (int)(q.kt * BN));
+                }
+            }
+            for (int j = seq - STAGES; j < seq; ++j)
+                if (j >= 0)
+                    mbar_wait(&sm.full[j % STAGES], (uint32_t)(j / STAGES) & 1u, wait_ns);
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMA issuer (the whole warp fixes tiles up)
+        int seq = 0, t = 0;
+        bool issued = false;
+        for (int64_t it = blockIdx.x; it < total && !aborted(&sm.abort_flag); it += gridDim.x) {
+            const Item q = item(it);
+            if (q.nch == 0)
+                continue;
+            const int acc = t & 1;
+            bool ok = t < ACC || mbar_wait(&sm.acc_empty[acc], ((uint32_t)(t / ACC) & 1u) ^ 1u, wait_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                *reinterpret_cast<volatile int *>(&sm.abort_flag) = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)(acc * BN);
+            for (int64_t j = 0; j < q.nch; ++j, ++seq) {
+                const int s = seq % STAGES;
+                ok = mbar_wait(&sm.full[s], (uint32_t)(seq / STAGES) & 1u, wait_ns);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok)
+                    break;
+                const int64_t c0 = q.x0 + j * BK;
+                const int lo = (int)max((int64_t)0, q.s - c0), hi = (int)min((int64_t)BK, q.e - c0);
+                if (lo > 0 || hi < BK) {
+                    // both tiles: positions past offs[G-1] were never written
+                    // by the quantization and may hold any byte, NaN codes
+                    // included, and 0 * NaN is NaN
+                    zero_outside(sm.a[s], BM, lo, hi);
+                    zero_outside(sm.b[s], BN, lo, hi);
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_k128(smem_u32(sm.a[s]));
+                    const uint64_t bd = smem_desc_k128(smem_u32(sm.b[s]));
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k)
+                        tc_mma(d, ad + 2 * k, bd + 2 * k, IDESC, (j > 0 || k > 0) ? 1u : 0u);
+                    tc_commit(&sm.empty[s]);
+                }
+                issued = true;
+                __syncwarp();
+            }
+            if (!ok) {
+                *reinterpret_cast<volatile int *>(&sm.abort_flag) = 1;
+                break;
+            }
+            if (lane == 0)
+                tc_commit(&sm.acc_full[acc]);
+            ++t;
+        }
+        if (issued && lane == 0) { // every issued MMA completes before TMEM is freed
+            tc_commit(&sm.mma_done);
+            mbar_wait(&sm.mma_done, 0u, wait_ns);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (warps 0-3, TMEM lanes 32w..32w+31)
+        int t = 0;
+        for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
+            const Item q = item(it);
+            const int64_t n = q.nt * BM + 32 * warp + lane; // this thread's output row
+            uint16_t *dst = out + ((int64_t)q.g * N + n) * K + q.kt * BN;
+            if (q.nch == 0) { // empty group: the sum is zero
+                for (int c = 0; c < BN; c += 8)
+                    st_v4(dst + c, 0u, 0u, 0u, 0u);
+                continue;
+            }
+            const int acc = t & 1;
+            bool ok = mbar_wait(&sm.acc_full[acc], (uint32_t)(t / ACC) & 1u, wait_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok || aborted(&sm.abort_flag)) {
+                *reinterpret_cast<volatile int *>(&sm.abort_flag) = 1;
+                break;
+            }
+            tc_fence_after();
+            const float sa = __ldg(inv_a + (int64_t)q.g * N + n);
+            const float *sb = inv_b + (int64_t)q.g * K + q.kt * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tc_ld32(tmem + (uint32_t)(acc * BN + c * 32) + ((uint32_t)(32 * warp) << 16), r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(r[2 * j]), sa), __ldg(sb + c * 32 + 2 * j));
+                    const float v1 =
+                        __fmul_rn(__fmul_rn(__uint_as_float(r[2 * j + 1]), sa), __ldg(sb + c * 32 + 2 * j + 1));
+                    pk[j] = pack_bf16x2(v0, v1);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    st_v4(dst + c * 32 + 8 * j, pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.acc_empty[acc]);
+            ++t;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+}
+
 } // namespace mxq
+

@@ -102,6 +102,10 @@ int device_info(const DevInfo **out)
                                  (int)(gm::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(gm::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gm::smem_fixed<128>()) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gm::smem_fixed<256>()) != cudaSuccess ||
             cudaFuncSetAttribute(k_jagged_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)jag::cst::SMEM_BYTES) != cudaSuccess)
             return MXQ_ERR_CUDA;
@@ -407,6 +411,49 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
     return launch(k_fp8_grouped_gemm<128>, dim3((unsigned)grid), dim3(gm::THREADS),
                   gm::smem_fixed<128>() + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M, N,
                   K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+}
+
+int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, const float *inv_b, int64_t N,
+                           int64_t K, int64_t M, const int32_t *offs, int32_t num_groups, void *out,
+                           cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % gm::BM || K % 128 || M % 16)
+        return MXQ_ERR_SHAPE;
+    if (N == 0 || K == 0)
+        return MXQ_OK;
+    if (!a || !inv_a || !b || !inv_b || !offs || !out)
+        return MXQ_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(inv_a, 4) || !aligned(inv_b, 4))
+        return MXQ_ERR_ALIGN;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    const int bn = K % 256 == 0 ? 256 : 128;
+    CUtensorMap ta, tb;
+    const uint64_t mm = (uint64_t)std::max<int64_t>(M, 16); // a map needs a non-zero extent
+    const uint64_t da[2] = {mm, (uint64_t)N};
+    const uint64_t sa[1] = {mm};
+    const uint32_t boxa[2] = {gm::BK, gm::BM};
+    rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, boxa, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t db[2] = {mm, (uint64_t)K};
+    const uint32_t boxb[2] = {gm::BK, (uint32_t)bn};
+    rc = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, db, sa, boxb, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t items = (int64_t)num_groups * (N / gm::BM) * (K / bn);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, di->sms));
+    if (bn == 256)
+        return launch(k_fp8_grouped_gemm_wgrad<256>, dim3((unsigned)grid), dim3(gm::THREADS), gm::smem_fixed<256>(),
+                      stream, false, ta, tb, inv_a, inv_b, N, K, M, offs, (int)num_groups,
+                      static_cast<uint16_t *>(out), wait_ns());
+    return launch(k_fp8_grouped_gemm_wgrad<128>, dim3((unsigned)grid), dim3(gm::THREADS), gm::smem_fixed<128>(),
+                  stream, false, ta, tb, inv_a, inv_b, N, K, M, offs, (int)num_groups, static_cast<uint16_t *>(out),
+                  wait_ns());
 }
 
 int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t mode, void *out, uint8_t *scales,

@@ -93,6 +93,10 @@ def test_host_checks_return_before_any_cuda_call(lib):
         binding.ERR_UNSUPPORTED
     assert lib.fp8_grouped_gemm_rowwise(fake, null, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_NULL
     assert lib.fp8_grouped_gemm_rowwise(odd, fake, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_ALIGN
+    assert lib.fp8_grouped_gemm_wgrad(fake, fake, fake, fake, 100, 128, 128, fake, 1, fake, null) == binding.ERR_SHAPE
+    assert lib.fp8_grouped_gemm_wgrad(fake, fake, fake, fake, 128, 128, 120, fake, 1, fake, null) == binding.ERR_SHAPE
+    assert lib.fp8_grouped_gemm_wgrad(fake, fake, null, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_NULL
+    assert lib.fp8_grouped_gemm_wgrad(fake, fake, odd, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_ALIGN
     # blockwise with transposed output
     assert lib.fp8_quant_blockwise_transposed(fake, 128, 128, 1, 128, fake, fake, null) == binding.ERR_UNSUPPORTED
     assert lib.fp8_quant_blockwise_transposed(fake, 128, 128, 128, 64, fake, fake, null) == binding.ERR_UNSUPPORTED

@@ -99,3 +99,47 @@ def test_grouped_gemm_moe_shape_sampled():
     ends = np.array([np.sum(groups <= g) for g in range(E)], dtype=np.int32)
     sub = torch.from_numpy(ends).to(DEV)
     _check(out[rows.to(DEV)], torch.from_numpy(a_sel), torch.from_numpy(ia_sel), wq, iw, sub, K)
+
+
+# ---------------------------------------------------------------- weight gradient
+
+def _wgrad_operands(M, N, K, ends, seed):
+    """grad_out (M, N) and input (M, K) bf16 quantized by the jagged ops:
+    rowwise on grad_out^T gives a (N, M) and inv_a (G, N); colwise on the input
+    gives the (K, M) buffer b and inv_b (G, K)."""
+    go = synth.student_t3_bf16(M, N, seed, DEV)
+    x = synth.row_scaled_normal_bf16(M, K, seed=seed + 1, device=DEV)
+    offs = torch.tensor(ends, dtype=torch.int32, device=DEV)
+    a, ia = mxq.fp8_quant_jagged_rowwise(go.t(), offs)
+    bq, ib = mxq.fp8_quant_jagged_colwise(x, offs)
+    return a.view(torch.uint8), ia, bq.t().view(torch.uint8), ib, offs
+
+
+def _check_wgrad(out, a, ia, b, ib, offs):
+    a_c, b_c = a.cpu().numpy(), b.cpu().numpy()
+    ia_n, ib_n, o = ia.cpu().numpy(), ib.cpu().numpy(), offs.cpu().numpy()
+    ref = oracle.fp8_grouped_gemm_wgrad(a_c, ia_n, b_c, ib_n, o)
+    dec = np.abs(np.array([oracle.e4m3_value(c) for c in range(256)]))
+    A, B = dec[a_c], dec[b_c]
+    got = out.float().cpu().numpy().astype(np.float64)
+    start = 0
+    for g, end in enumerate(o):
+        S = (A[:, start:end] @ B[:, start:end].T) * ia_n[g][:, None] * ib_n[g][None, :]
+        bound = 2.0 ** -8 * np.abs(ref[g]) + max(end - start, 1) * 2.0 ** -23 * S
+        excess = np.max(np.abs(got[g] - ref[g]) - bound)
+        assert excess <= 0, (g, excess)
+        start = end
+
+
+@pytest.mark.parametrize("M,N,K,ends", [
+    (512, 128, 256, [128, 128, 384, 512]),      # aligned groups, an empty one
+    (1008, 256, 384, [3, 250, 251, 700, 992]),   # unaligned starts and ends, one-row group, tail positions
+    (4096, 384, 512, [1000, 1016, 3000, 4096]),
+])
+def test_wgrad_gemm_vs_oracle(M, N, K, ends):
+    a, ia, b, ib, offs = _wgrad_operands(M, N, K, ends, seed=M + K)
+    out = mxq.fp8_grouped_gemm_wgrad(a, ia, b, ib, offs)
+    assert mxq.device_status() == 0
+    _check_wgrad(out, a, ia, b, ib, offs)
+    assert bool((out[1] == 0).all()) if ends[1] == ends[0] else True
+
