@@ -503,9 +503,38 @@ def gemm_rows(wl, flush, reps):
     us = statistics.median(ts)
     flops = 2.0 * T * N * K
     tf = flops / (us * 1e-6) / 1e12
-    return [{"op": "fp8_grouped_gemm", "shape": f"({T},{K}) G=64 x (64,{N},{K})", "us": round(us, 3),
+    rows = [{"op": "fp8_grouped_gemm", "shape": f"({T},{K}) G=64 x (64,{N},{K})", "us": round(us, 3),
              "TFLOP/s": round(tf, 1), "frac_fp8_peak": round(tf / fp8_peak, 4), "peak_TFLOP/s": round(fp8_peak, 1),
              "peak_kind": kind}]
+    del aq, wq, out
+    # weight gradient of the jagged backward config: grad_out^T (4096, 65536)
+    # rowwise and input (65536, 4096) colwise, G=16, -> (16, 4096, 4096)
+    if hasattr(wl, "grad_out"):
+        M, D = wl.inp.shape
+        a, ia = mxq.fp8_quant_jagged_rowwise(wl.grad_out.t(), wl.offs16)
+        b, ib = mxq.fp8_quant_jagged_colwise(wl.inp, wl.offs16)
+        a, b = a.view(torch.uint8), b.t().view(torch.uint8)
+        gw = torch.empty((16, D, D), dtype=torch.bfloat16, device=dev)
+        fn = lambda: mxq.fp8_grouped_gemm_wgrad(a, ia, b, ib, wl.offs16, out=gw)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(max(reps // 5, 3)):
+            flush_l2(torch, flush)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        us = statistics.median(ts)
+        tf = 2.0 * M * D * D / (us * 1e-6) / 1e12
+        rows.append({"op": "fp8_grouped_gemm_wgrad", "shape": f"({D},{M})x({D},{M}) G=16 -> (16,{D},{D})",
+                     "us": round(us, 3), "TFLOP/s": round(tf, 1), "frac_fp8_peak": round(tf / fp8_peak, 4),
+                     "peak_TFLOP/s": round(fp8_peak, 1), "peak_kind": kind})
+    return rows
 
 
 # ----------------------------------------------------------------- oracle side

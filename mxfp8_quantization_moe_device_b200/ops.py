@@ -232,3 +232,19 @@ def fp8_grouped_gemm_rowwise(a: torch.Tensor, inv_a: torch.Tensor, w: torch.Tens
 def _(a, inv_a, w, inv_w, offs):
     return a.new_empty((a.shape[0], w.shape[1]), dtype=torch.bfloat16)
 
+
+@torch.library.custom_op("mxq::fp8_grouped_gemm_wgrad", mutates_args=())
+def fp8_grouped_gemm_wgrad(a: torch.Tensor, inv_a: torch.Tensor, b: torch.Tensor, inv_b: torch.Tensor,
+                           offs: torch.Tensor) -> torch.Tensor:
+    """Weight-gradient grouped GEMM on the tensor cores: (G, N, K) bf16, out[g]
+    = (a[:, group g] . b[:, group g]^T) * inv_a[g][:, None] * inv_b[g]."""
+    G, N, K = offs.shape[0], a.shape[0], b.shape[0]
+    out = torch.empty((G, N, K), dtype=torch.bfloat16, device=a.device)
+    _b.fp8_grouped_gemm_wgrad(a.view(torch.uint8), inv_a, b.view(torch.uint8), inv_b, offs, out=out)
+    return out
+
+
+@fp8_grouped_gemm_wgrad.register_fake
+def _(a, inv_a, b, inv_b, offs):
+    return a.new_empty((offs.shape[0], a.shape[0], b.shape[0]), dtype=torch.bfloat16)
+

@@ -11,7 +11,8 @@ from mxfp8_quantization_moe_device_b200 import synth
 
 OPS = ["fp8_quant_jagged_rowwise", "fp8_quant_jagged_colwise", "fp8_quant_blockwise",
        "fp8_quant_blockwise_transposed", "mx_quant_3d_colwise", "mx_quant_rowwise", "mx_scales_to_blocked_grouped",
-       "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped", "fp8_grouped_gemm_rowwise"]
+       "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped", "fp8_grouped_gemm_rowwise",
+       "fp8_grouped_gemm_wgrad"]
 
 
 def _cases(dev):
@@ -54,6 +55,15 @@ def test_gemm_fake_shape_on_meta_tensors():
                                                  torch.empty((3, 128), device="meta"),
                                                  torch.empty(3, dtype=torch.int32, device="meta"))
     assert tuple(out.shape) == (300, 128) and out.dtype == torch.bfloat16
+
+
+def test_wgrad_fake_shape_on_meta_tensors():
+    a = torch.empty((256, 512), dtype=torch.float8_e4m3fn, device="meta")
+    b = torch.empty((384, 512), dtype=torch.float8_e4m3fn, device="meta")
+    out = torch.ops.mxq.fp8_grouped_gemm_wgrad(a, torch.empty((3, 256), device="meta"), b,
+                                               torch.empty((3, 384), device="meta"),
+                                               torch.empty(3, dtype=torch.int32, device="meta"))
+    assert tuple(out.shape) == (3, 256, 384) and out.dtype == torch.bfloat16
 
 
 def test_fake_shapes_on_meta_tensors():
