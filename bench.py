@@ -81,7 +81,7 @@ KERNEL_FILES = {  # source files that define each kernel (plus common.cuh)
     "k_fp8_1x128": "rowblock.cuh", "k_fp8_128x128": "rowblock.cuh", "k_mx_1x32": "rowblock.cuh",
     "k_jagged_amax": "jagged.cuh", "k_jagged_cast": "jagged.cuh", "k_mx_3d_colwise": "mx3d.cuh",
     "k_blocked_grouped": "blocked.cuh", "k_blocked_grouped_k": "blocked.cuh", "k_mx_1x32_blocked": "blocked.cuh",
-    "k_fp8_blockwise_t": "blockt.cuh", "k_fp8_grouped_gemm": "gemm.cuh",
+    "k_fp8_blockwise_t": "blockt.cuh", "k_fp8_grouped_gemm": "gemm.cuh", "k_fp8_grouped_gemm_wgrad": "gemm.cuh",
 }
 
 
@@ -173,7 +173,8 @@ class Workload:
     OPS = ("blockwise_1x128", "blockwise_128x128", "jagged_rowwise", "jagged_colwise", "mx_3d_colwise",
            "mx_rowwise", "blocked_grouped")
     # ops outside the step (the widened rows), built only when asked for by name
-    EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked", "grouped_gemm")
+    EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked", "grouped_gemm",
+             "grouped_gemm_wgrad")
 
     def __init__(self, dev, experts, mx3d_mode, only=None):
         import torch
@@ -284,6 +285,19 @@ class Workload:
             self.o.update(g_out=t.empty((T, N), dtype=t.bfloat16, device=dev))
             self.ops.append(("grouped_gemm", lambda: mxq.fp8_grouped_gemm_rowwise(
                 self.g_a, self.g_ia, self.g_w, self.g_iw, self.g_offs, out=self.o["g_out"]), 2 * T * N * K))
+
+        if "grouped_gemm_wgrad" in want:
+            # the jagged backward config: grad_out^T (4096, 65536) and input (65536, 4096), G=16
+            go, x, offs16 = synth.jagged_bwd(device=dev)
+            self.offs16 = offs16.to(dev)
+            M, D = x.shape
+            a, ia = mxq.fp8_quant_jagged_rowwise(go.t(), self.offs16)
+            b, ib = mxq.fp8_quant_jagged_colwise(x, self.offs16)
+            del go, x
+            self.w_a, self.w_ia, self.w_b, self.w_ib = a.view(t.uint8), ia, b.t().view(t.uint8), ib
+            self.o.update(w_out=t.empty((16, D, D), dtype=t.bfloat16, device=dev))
+            self.ops.append(("grouped_gemm_wgrad", lambda: mxq.fp8_grouped_gemm_wgrad(
+                self.w_a, self.w_ia, self.w_b, self.w_ib, self.offs16, out=self.o["w_out"]), 2 * M * D * D))
 
     def step_bytes(self):
         return sum(b for _, _, b in self.ops)
