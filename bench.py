@@ -623,37 +623,84 @@ REF_SAMPLE_DESC = ("single-threaded C oracle, one pass per step over a slice of 
 
 # ----------------------------------------------------------------- e2e
 
+# inputs (host -> device) and outputs (device -> host) of each op of the step
+E2E_IO = {
+    "blockwise_1x128": (("act",), ("act_q", "act_s")),
+    "blockwise_128x128": (("wt",), ("wt_q", "wt_s")),
+    "jagged_rowwise": (("grad_out", "offs16"), ("go_q", "go_s")),
+    "jagged_colwise": (("inp",), ("in_q", "in_s")),
+    "mx_3d_colwise": (("w3",), ("w3_q", "w3_s")),
+    "mx_rowwise": (("tok", "offs64"), ("tok_q", "tok_s")),
+    "blocked_grouped": ((), ("blk", "blk_starts")),
+}
+
+
 def run_e2e(wl, steps):
-    """The same step through the public API from pinned host buffers: each step
-    copies its inputs host->device, runs every op, and copies every output
-    back to pinned host memory, all inside the timed region."""
+    """The same step through the public API from pinned host buffers: every
+    step copies every op's inputs host->device (the group offsets included),
+    runs every op, and copies every output back to pinned host memory, all
+    inside the timed region. Three streams (copy in, compute, copy out) with
+    events: an op's outputs travel back while the next op's inputs come in
+    (PCIe is full duplex), and a step's copies into a buffer wait for the
+    previous step's use of it."""
     torch = wl.torch
     host_in = {}
-    for name in ("act", "wt", "grad_out", "inp", "w3", "tok"):
+    for name in ("act", "wt", "grad_out", "inp", "w3", "tok", "offs16", "offs64"):
         t = getattr(wl, name)
         h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
         h.copy_(t)
         host_in[name] = h
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in wl.o.items()}
-    bi = sum(h.numel() * h.element_size() for h in host_in.values()) + 2 * 4 * (16 + 64)
+    bi = sum(h.numel() * h.element_size() for h in host_in.values())
     bo = sum(h.numel() * h.element_size() for h in host_out.values())
-    stream = torch.cuda.current_stream()
+    # the largest transfer first: its results return while the rest come in
+    order = sorted(wl.ops, key=lambda op: op[0] != "mx_3d_colwise")
+    s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    done_c = {n: None for n, _, _ in order}   # last compute of each op
+    done_o = {n: None for n, _, _ in order}   # last copy-out of each op
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(s_in)
     for _ in range(steps):
-        for name, h in host_in.items():
-            getattr(wl, name).copy_(h, non_blocking=True)
-        for _, fn, _ in wl.ops:
-            fn()
-        for k, h in host_out.items():
-            h.copy_(wl.o[k], non_blocking=True)
-    b.record(stream)
+        for name, fn, _ in order:
+            ins, outs = E2E_IO[name]
+            if done_c[name] is not None:
+                s_in.wait_event(done_c[name])      # the previous step has read these inputs
+            with torch.cuda.stream(s_in):
+                for k in ins:
+                    getattr(wl, k).copy_(host_in[k], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+            s_c.wait_event(ev_in)
+            if done_o[name] is not None:
+                s_c.wait_event(done_o[name])       # the previous step's outputs are back on the host
+            with torch.cuda.stream(s_c):
+                fn()
+            ev_c = torch.cuda.Event()
+            ev_c.record(s_c)
+            done_c[name] = ev_c
+            s_out.wait_event(ev_c)
+            with torch.cuda.stream(s_out):
+                for k in outs:
+                    host_out[k].copy_(wl.o[k], non_blocking=True)
+            ev_o = torch.cuda.Event()
+            ev_o.record(s_out)
+            done_o[name] = ev_o
+    s_in.wait_stream(s_c)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
+    # the results that reached the host are the device's (first and last MB of each)
+    ok = True
+    for k, h in host_out.items():
+        d = wl.o[k].reshape(-1).view(torch.uint8) if wl.o[k].element_size() == 1 else wl.o[k].reshape(-1)
+        hv = h.reshape(-1).view(torch.uint8) if h.element_size() == 1 else h.reshape(-1)
+        n = min(d.numel(), 1 << 20)
+        ok = ok and torch.equal(hv[:n], d[:n].cpu()) and torch.equal(hv[-n:], d[-n:].cpu())
     del host_in, host_out
-    return ms, bi, bo
+    return ms, bi, bo, ok
 
 
 # ----------------------------------------------------------------- ranks
@@ -760,11 +807,11 @@ def main():
         out["cpu_baseline"] = {"value": round(gbs, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
                                "sample": SAMPLE_DESC, "seconds": round(spent, 2), "per_op_GB/s": per_o}
     if not args.no_e2e:
-        ms, bi, bo = run_e2e(wl, max(1, args.e2e_steps))
+        ms, bi, bo, ok = run_e2e(wl, max(1, args.e2e_steps))
         ms = max_over_ranks(ms, dev, world)
         out["e2e"] = {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                       "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 3),
-                      "steps": max(1, args.e2e_steps)}
+                      "steps": max(1, args.e2e_steps), "results_match_device": ok}
     if not args.no_per_shape and rank == 0:
         out["per_shape"] = per_shape_sweep(wl, args.reps)
     if world > 1:
