@@ -17,6 +17,8 @@
 // Kernels:
 //   k_jagged_generic  any strides, small problems: one warp per (line, group),
 //                     the group read into registers, reduced, then cast.
+//   k_jagged_rows     positions contiguous (rowwise on a row-major matrix):
+//                     one warp per line, 16-byte loads, two passes per group.
 //   k_jagged_amax +   contiguous lines, two streaming passes. The amax pass
 //   k_jagged_cast     runs warp workers, each owning 256 lines (16 bytes per
 //                     lane per row) and an equal run of positions, keeping 16
@@ -119,6 +121,74 @@ __global__ void __launch_bounds__(256) k_jagged_generic(const uint16_t *__restri
                         dst[p] = (uint8_t)e4m3x2(__fmul_rn(v[i], s), 0.0f);
                 }
             }
+        }
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Positions contiguous (stride 1 along the grouped dimension, e.g. rowwise on
+// a row-major matrix): one warp per line. For each group in turn the warp
+// reads the group's run of the line with 16-byte loads (8 elements per lane,
+// elements outside the group masked in the two boundary vectors), reduces the
+// amax, then reads the run again (now in L1/L2), casts, and writes 8 bytes per
+// lane; a vector that straddles a group end is written byte by byte, so each
+// byte is written by exactly one group's pass. Needs 16-byte aligned lines
+// (base and line stride) and an 8-byte aligned output with P % 8 == 0.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_jagged_rows(const uint16_t *__restrict__ in, int64_t L, int64_t P,
+                                                     int64_t s_line, const int32_t *__restrict__ offs, int G,
+                                                     uint8_t *__restrict__ out, float *__restrict__ inv)
+{
+    if (!offsets_ok(offs, G, P))
+        return;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t l = warp; l < L; l += nwarps) {
+        const uint16_t *src = in + l * s_line;
+        uint8_t *dst = out + l * P;
+        int64_t s = 0;
+        for (int g = 0; g < G; ++g) {
+            const int64_t e = offs[g];
+            // vectors of 8 covering [s, e), from the 8-aligned position at or below s
+            const int64_t v0 = s & ~int64_t(7);
+            uint32_t acc = 0;
+#pragma unroll 4
+            for (int64_t p = v0 + 8 * lane; p < e; p += 256) {
+                uint4 v = *reinterpret_cast<const uint4 *>(src + p);
+                if (p < s || p + 8 > e) { // boundary vector: drop elements outside [s, e)
+                    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (p + j < s || p + j >= e)
+                            w[j >> 1] &= (j & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+                    v = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                acc = absmax_bf16x2(absmax_bf16x2(acc, v.x), v.y);
+                acc = absmax_bf16x2(absmax_bf16x2(acc, v.z), v.w);
+            }
+            float amax = absmax_of_pair(acc);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const float sc = fp8_scale(amax);
+            if (lane == 0)
+                inv[(int64_t)g * L + l] = fp8_inv(sc);
+#pragma unroll 4
+            for (int64_t p = v0 + 8 * lane; p < e; p += 256) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + p);
+                const uint32_t q0 = quant4(v.x, v.y, sc), q1 = quant4(v.z, v.w, sc);
+                if (p >= s && p + 8 <= e) {
+                    st_v2(dst + p, q0, q1);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (p + j >= s && p + j < e)
+                            dst[p + j] = (uint8_t)((j < 4 ? q0 : q1) >> (8 * (j & 3)));
+                }
+            }
+            s = e;
         }
     }
 }

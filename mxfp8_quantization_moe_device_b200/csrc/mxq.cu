@@ -253,6 +253,13 @@ int jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, 
     rc = device_info(&di);
     if (rc != MXQ_OK)
         return rc;
+    if (g_force_path.load() != 2 && s_pos == 1 && s_line % 8 == 0 && s_line >= P && P % 8 == 0 && aligned(in, 16) &&
+        aligned(out, 16)) {
+        // positions contiguous: one warp per line, vector loads
+        const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((L + 7) / 8, (int64_t)di->sms * 16));
+        return launch(k_jagged_rows, dim3((unsigned)grid), dim3(256), 0, stream, false,
+                      static_cast<const uint16_t *>(in), L, P, s_line, offs, G, static_cast<uint8_t *>(out), inv);
+    }
     const int64_t warps = L * G;
     const int64_t grid = std::min<int64_t>((warps + 7) / 8, (int64_t)di->sms * 16);
     return launch(k_jagged_generic, dim3((unsigned)std::max<int64_t>(grid, 1)), dim3(256), 0, stream, false,

@@ -120,20 +120,59 @@ def test_jagged_colwise_and_rowwise_vs_oracle(M, D, spec, path):
         mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
 
 
-@pytest.mark.parametrize("R,C,offs", [(24, 160, [7, 7, 100, 150]), (5, 33, [33]), (130, 64, [1, 2, 64])])
-def test_jagged_rowwise_contiguous_rows_generic(R, C, offs):
-    """Groups along the contiguous dimension (not the transposed view): generic path."""
-    x = synth.row_scaled_normal_bf16(R, C, seed=R * C, device=DEV)
-    o = torch.tensor(offs, dtype=torch.int32)
-    ref_q, ref_inv = oracle.fp8_quant_jagged_rowwise(words(x).reshape(-1), R, C, C, 1, o.numpy())
-    out = torch.full((R, C), SENT, dtype=torch.uint8, device=DEV)
-    q, inv = mxq.fp8_quant_jagged_rowwise(x, o.to(DEV), out=out)
-    assert status_ok()
-    end = offs[-1]
-    got = u8(out)
-    assert np.array_equal(got[:, :end], ref_q[:, :end])
-    assert np.all(got[:, end:] == SENT)
-    assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
+ROWS_CASES = [
+    (24, 160, [7, 7, 100, 150]),             # empty group, boundaries inside 8-element vectors
+    (5, 33, [33]),                           # odd width: generic only
+    (130, 64, [1, 2, 64]),
+    (300, 520, [0, 3, 3, 261, 262, 500]),    # rows past the last group, one-element group
+    (64, 4096, [1000, 1001, 1009, 3000]),    # long groups, several vector rounds per lane
+    (1, 7168, [7168]),                       # a single line
+    (2048, 7168, "multinomial"),             # groups of 16-column units
+]
+
+
+@pytest.mark.parametrize("path", [0, 2], ids=["auto", "generic"])
+@pytest.mark.parametrize("R,C,offs", ROWS_CASES)
+def test_jagged_rowwise_contiguous_rows(R, C, offs, path):
+    """Groups along the contiguous dimension of a row-major matrix: the
+    positions-contiguous kernel (auto) and the generic kernel (forced) against
+    the oracle, with guard margins around both outputs."""
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
+    try:
+        x = synth.row_scaled_normal_bf16(R, C, seed=R * C, device=DEV)
+        o = synth.multinomial_offsets(C, 8, 16, 3) if isinstance(offs, str) else torch.tensor(offs, dtype=torch.int32)
+        ref_q, ref_inv = oracle.fp8_quant_jagged_rowwise(words(x).reshape(-1), R, C, C, 1, o.numpy())
+        big, out = guarded(R * C)
+        bigi, inv = guarded(o.numel() * R, torch.float32)
+        q, inv = mxq.fp8_quant_jagged_rowwise(x, o.to(DEV), out=out.view(R, C), inv_scales=inv.view(-1, R))
+        assert status_ok()
+        end = int(o[-1])
+        got = u8(out).reshape(R, C)
+        assert np.array_equal(got[:, :end], ref_q[:, :end])
+        assert np.all(got[:, end:] == SENT)
+        assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
+        assert margins_intact(big) and margins_intact(bigi, torch.float32)
+    finally:
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+
+
+@pytest.mark.parametrize("path", [0, 2], ids=["auto", "generic"])
+def test_jagged_colwise_on_column_major_input(path):
+    """colwise on a column-major matrix (the transpose of a row-major one) has
+    contiguous positions too: same kernel choice as rowwise on row-major."""
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
+    try:
+        base = synth.row_scaled_normal_bf16(96, 1032, seed=11, device=DEV)  # (cols, rows) storage
+        x = base.t()                                                        # (rows=1032, cols=96)
+        o = torch.tensor([9, 9, 517, 1000], dtype=torch.int32)
+        ref_q, ref_inv = oracle.fp8_quant_jagged_colwise(words(base).reshape(-1), 1032, 96, 1, 1032, o.numpy())
+        q, inv = mxq.fp8_quant_jagged_colwise(x, o.to(DEV))
+        assert status_ok()
+        got = u8(q.t().contiguous()).reshape(96, 1032)
+        assert np.array_equal(got[:, :1000], ref_q[:, :1000])
+        assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
+    finally:
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
 
 
 def test_jagged_colwise_strided_view_generic():
