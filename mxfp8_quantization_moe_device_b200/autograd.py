@@ -1,0 +1,114 @@
+"""Differentiable FP8 rowwise-scaled grouped matmul for MoE layers.
+
+out[m] = a[m] . w[g]^T for the tokens m of expert g (groups given by device
+int32 ends `offs` along the token dimension), with every operand quantized
+to float8 e4m3 by this library's kernels and every product computed by its
+tcgen05 grouped GEMMs. This is the training use that "[scaled grouped mm] add
+triton kernels for float8 rowwise quantization with per-group/jagged scales"
+(Motivation) describes: the weight gradient contracts over each expert's own
+tokens, so its operands need one scale per (expert group, row) and per
+(expert group, column), which is what the jagged ops produce.
+
+Scale granularity of each GEMM (one e4m3 scale per listed unit, amax over the
+contracted dimension):
+  forward   out = A W^T      A per token (over K), W per (expert, n) (over K)
+  input     dA  = dY W       dY per token (over N), W per (expert, k) (over N)
+  weight    dW  = dY^T A     dY per (group, n) and A per (group, k), both over
+                             the group's tokens (the jagged rowwise and
+                             colwise ops)
+
+Rows of out and dA past offs[-1] (tokens routed to no expert) are zero.
+Nothing here computes on the host or through torch kernels besides output
+allocation: quantization and GEMMs are the library's CUDA kernels, so a
+missing library raises instead of falling back.
+"""
+import torch
+
+from . import binding as mxq
+
+
+def _check(a, w, offs):
+    for t, n in ((a, "a"), (w, "w"), (offs, "offs")):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+            raise TypeError(f"{n} must be a CUDA tensor")
+    if a.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("a and w must be bfloat16")
+    if a.dim() != 2 or w.dim() != 3 or not a.is_contiguous() or not w.is_contiguous():
+        raise TypeError("a must be a contiguous (M, K) and w a contiguous (E, N, K) tensor")
+    if offs.dtype != torch.int32 or offs.dim() != 1 or offs.numel() != w.shape[0]:
+        raise TypeError("offs must be an int32 vector of one group end per expert")
+    M, K = a.shape
+    E, N, K2 = w.shape
+    if K2 != K or N % 128 or K % 128 or M % 16:
+        raise ValueError("need w.shape[2] == a.shape[1], N % 128 == 0, K % 128 == 0 and M % 16 == 0")
+
+
+def _rowwise(x, length):
+    """e4m3 codes of a row-major (R, C) tensor, one scale per row over all C
+    columns, and the (R,) inverse scales."""
+    R, C = x.shape
+    q, inv = mxq.fp8_quant_jagged_rowwise(x, torch.tensor([length], dtype=torch.int32, device=x.device))
+    return q.view(torch.uint8), inv.reshape(R)
+
+
+def _forward(a, w, offs):
+    M, K = a.shape
+    E, N, _ = w.shape
+    aq, ia = _rowwise(a, K)
+    wq, iw = _rowwise(w.view(E * N, K), K)
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device=a.device)
+    return mxq.fp8_grouped_gemm_rowwise(aq, ia, wq.view(E, N, K), iw.view(E, N), offs, out=out)
+
+
+def _grad_input(dy, w, offs):
+    M, N = dy.shape
+    E, _, K = w.shape
+    dyq, idy = _rowwise(dy, N)
+    # W_e^T per expert: the colwise op on W_e (N, K) with one group over all
+    # N rows writes the column-major buffer, i.e. W_e^T (K, N) row-major, with
+    # one scale per (expert, k)
+    wt = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
+    iwt = torch.empty((E, K), dtype=torch.float32, device=w.device)
+    nn = torch.tensor([N], dtype=torch.int32, device=w.device)
+    for e in range(E):
+        mxq.fp8_quant_jagged_colwise(w[e], nn, out=wt[e], inv_scales=iwt[e].view(1, K))
+    da = torch.zeros((M, K), dtype=torch.bfloat16, device=dy.device)
+    return mxq.fp8_grouped_gemm_rowwise(dyq, idy, wt, iwt, offs, out=da)
+
+
+def _grad_weight(dy, a, offs):
+    M, N = dy.shape
+    _, K = a.shape
+    G = offs.numel()
+    # dY^T (N, M) with one scale per (group, n), A's columns with one scale per
+    # (group, k): both column-major over the tokens, the layout the
+    # weight-gradient GEMM reads
+    dytq, idyt = mxq.fp8_quant_jagged_rowwise(dy.t(), offs)
+    acq, iac = mxq.fp8_quant_jagged_colwise(a, offs)
+    return mxq.fp8_grouped_gemm_wgrad(dytq.view(torch.uint8), idyt.reshape(G, N),
+                                      acq.t().view(torch.uint8), iac.reshape(G, K), offs)
+
+
+class FP8GroupedMM(torch.autograd.Function):
+    """autograd.Function over the three grouped GEMMs; see the module text."""
+
+    @staticmethod
+    def forward(ctx, a, w, offs):
+        _check(a, w, offs)
+        ctx.save_for_backward(a, w, offs)
+        return _forward(a, w, offs)
+
+    @staticmethod
+    def backward(ctx, dy):
+        a, w, offs = ctx.saved_tensors
+        dy = dy.to(torch.bfloat16).contiguous()
+        da = _grad_input(dy, w, offs) if ctx.needs_input_grad[0] else None
+        dw = _grad_weight(dy, a, offs) if ctx.needs_input_grad[1] else None
+        return da, dw, None
+
+
+def fp8_grouped_mm(a, w, offs):
+    """out (M, N) bf16 = the FP8 rowwise-scaled grouped product of a (M, K)
+    bf16 tokens sorted by expert and w (E, N, K) bf16 expert weights, with
+    offs (E,) int32 group ends on the device; differentiable in a and w."""
+    return FP8GroupedMM.apply(a, w, offs)

@@ -1,0 +1,145 @@
+"""The differentiable FP8 grouped matmul (autograd wrapper over the jagged
+ops and the grouped GEMMs) against the same pipeline run by the oracle.
+
+The oracle quantizes the bf16 operands exactly as the pages define (bit-exact
+with the CUDA ops, tested elsewhere) and contracts the e4m3 codes in fp64, so
+every output, dA and dW element is checked against the grouped-GEMM bound
+|got - ref| <= 2^-8 |ref| + K * 2^-23 * S, S = sum_k |a_k w_k| * inv_a * inv_w,
+with K the contraction length (tests/test_gemm.py derives it)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp8_quantization_moe_device_b200 import synth
+from mxfp8_quantization_moe_device_b200.autograd import fp8_grouped_mm
+
+DEC = np.abs(np.array([oracle.e4m3_value(c) for c in range(256)]))
+
+
+def _words(t):
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+
+
+def _check_grouped(got, ref, a, ia, w, iw, offs, K):
+    """forward-type product: rows of group g against w[g]; rows past the last
+    group must be zero."""
+    end = int(offs[-1])
+    S = np.zeros_like(ref)
+    start = 0
+    for g, e in enumerate(offs):
+        if e > start:
+            S[start:e] = (DEC[a[start:e]] @ DEC[w[g]].T) * ia[start:e, None] * iw[g][None, :]
+        start = e
+    got = got.float().cpu().numpy().astype(np.float64)
+    excess = np.abs(got[:end] - ref[:end]) - (2.0 ** -8 * np.abs(ref[:end]) + K * 2.0 ** -23 * S[:end])
+    assert np.max(excess) <= 0, np.max(excess)
+    assert np.all(got[end:] == 0)
+
+
+def _check_wgrad(got, ref, a, ia, b, ib, offs):
+    got = got.float().cpu().numpy().astype(np.float64)
+    start = 0
+    for g, e in enumerate(offs):
+        S = (DEC[a[:, start:e]] @ DEC[b[:, start:e]].T) * ia[g][:, None] * ib[g][None, :]
+        bound = 2.0 ** -8 * np.abs(ref[g]) + max(e - start, 1) * 2.0 ** -23 * S
+        assert np.max(np.abs(got[g] - ref[g]) - bound) <= 0, g
+        start = e
+
+
+def _oracle_pipeline(a, w, dy, offs):
+    """out, dA, dW of the FP8 grouped matmul, every step by the oracle."""
+    M, K = a.shape
+    E, N, _ = w.shape
+    o = np.asarray(offs, dtype=np.int32)
+    aq, ia = oracle.fp8_quant_jagged_rowwise(_words(a), M, K, K, 1, [K])
+    wq, iw = oracle.fp8_quant_jagged_rowwise(_words(w), E * N, K, K, 1, [K])
+    ia, iw, wq = ia.reshape(M), iw.reshape(E, N), wq.reshape(E, N, K)
+    out = oracle.fp8_grouped_gemm_rowwise(aq, ia, wq, iw, o)
+    # dA = dY W: dY per token over N, W_e^T per (expert, k) over N
+    dyq, idy = oracle.fp8_quant_jagged_rowwise(_words(dy), M, N, N, 1, [N])
+    idy = idy.reshape(M)
+    wt, iwt = np.zeros((E, K, N), np.uint8), np.zeros((E, K), np.float32)
+    for e in range(E):
+        q, inv = oracle.fp8_quant_jagged_colwise(_words(w[e]), N, K, K, 1, [N])
+        wt[e], iwt[e] = q, inv.reshape(K)
+    da = oracle.fp8_grouped_gemm_rowwise(dyq, idy, wt, iwt, o)
+    # dW = dY^T A over each group's tokens: jagged rowwise on dY^T, colwise on A
+    dytq, idyt = oracle.fp8_quant_jagged_rowwise(_words(dy), N, M, 1, N, o)
+    acq, iac = oracle.fp8_quant_jagged_colwise(_words(a), M, K, K, 1, o)
+    dw = oracle.fp8_grouped_gemm_wgrad(dytq, idyt, acq, iac, o)
+    return dict(out=(out, aq, ia, wq, iw), da=(da, dyq, idy, wt, iwt), dw=(dw, dytq, idyt, acq, iac))
+
+
+def test_oracle_pipeline_approximates_the_exact_products():
+    """Pins what the pipeline computes: the oracle's out, dA and dW are the
+    exact grouped products A W_g^T, dY W_g and dY_g^T A_g up to e4m3 rounding
+    of the operands (a few percent in Frobenius norm); a transposed operand,
+    a wrong contraction dimension or a token in the wrong group is off by
+    order one."""
+    M, N, K, ends = 256, 128, 256, [64, 64, 240]
+    E = len(ends)
+    a = synth.row_scaled_normal_bf16(M, K, seed=11)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=12, lo=-2.0, hi=2.0).reshape(E, N, K)
+    dy = synth.row_scaled_normal_bf16(M, N, seed=13, lo=-3.0, hi=1.0)
+    r = _oracle_pipeline(a, w, dy, ends)
+    A, W, D = a.double().numpy(), w.double().numpy(), dy.double().numpy()
+    out, da, dw = np.zeros((M, N)), np.zeros((M, K)), np.zeros((E, N, K))
+    s = 0
+    for g, e in enumerate(ends):
+        out[s:e], da[s:e], dw[g] = A[s:e] @ W[g].T, D[s:e] @ W[g], D[s:e].T @ A[s:e]
+        s = e
+    end = ends[-1]
+    for got, want in ((r["out"][0][:end], out[:end]), (r["da"][0][:end], da[:end]), (r["dw"][0], dw)):
+        assert np.linalg.norm(got - want) <= 0.06 * np.linalg.norm(want)
+
+
+def test_wrapper_refuses_host_tensors():
+    a = torch.zeros((128, 128), dtype=torch.bfloat16)
+    w = torch.zeros((1, 128, 128), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        fp8_grouped_mm(a, w, torch.tensor([128], dtype=torch.int32))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K,ends", [
+    (256, 128, 256, [64, 64, 240]),          # an empty expert, tokens past the last group
+    (384, 256, 128, [5, 200, 384]),          # a 5-token expert, unaligned group boundaries
+])
+def test_forward_and_backward_vs_oracle(M, N, K, ends):
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    E = len(ends)
+    a = synth.row_scaled_normal_bf16(M, K, seed=M + K)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=N + 1, lo=-2.0, hi=2.0).reshape(E, N, K)
+    dy = synth.row_scaled_normal_bf16(M, N, seed=K + 2, lo=-3.0, hi=1.0)
+    ref = _oracle_pipeline(a, w, dy, ends)
+
+    offs = torch.tensor(ends, dtype=torch.int32, device="cuda")
+    ad = a.cuda().requires_grad_(True)
+    wd = w.cuda().requires_grad_(True)
+    out = fp8_grouped_mm(ad, wd, offs)
+    out.backward(dy.cuda())
+
+    r, aq, ia, wq, iw = ref["out"]
+    _check_grouped(out.detach(), r, aq, ia, wq, iw, ends, K)
+    r, dyq, idy, wt, iwt = ref["da"]
+    _check_grouped(ad.grad, r, dyq, idy, wt, iwt, ends, N)
+    r, dytq, idyt, acq, iac = ref["dw"]
+    _check_wgrad(wd.grad, r, dytq, idyt, acq, iac, ends)
+
+
+@pytest.mark.gpu
+def test_weight_only_gradient():
+    """Only w requires grad: the input-gradient GEMM is skipped, dW matches."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    M, N, K, ends = 256, 128, 128, [100, 256]
+    a = synth.row_scaled_normal_bf16(M, K, seed=5)
+    w = synth.row_scaled_normal_bf16(2 * N, K, seed=6).reshape(2, N, K)
+    dy = synth.row_scaled_normal_bf16(M, N, seed=7)
+    wd = w.cuda().requires_grad_(True)
+    out = fp8_grouped_mm(a.cuda(), wd, torch.tensor(ends, dtype=torch.int32, device="cuda"))
+    out.backward(dy.cuda())
+    r, dytq, idyt, acq, iac = _oracle_pipeline(a, w, dy, ends)["dw"]
+    _check_wgrad(wd.grad, r, dytq, idyt, acq, iac, ends)
