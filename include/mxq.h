@@ -181,6 +181,37 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
                              cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * mx_grouped_gemm - the MXFP8 consumer of the MX rowwise quantization and of
+ * the per-group 128x4 blocked scale layout (#3504 title: per-group blocked
+ * scales for MXFP8 MoE training, read here as the operands of the MoE
+ * layer's grouped GEMM; one E8M0 scale per 32 elements along K as the MX
+ * format defines), on the tensor cores
+ * (tcgen05.mma kind::mxf8f6f4.block_scale, fp32 accumulation in TMEM):
+ *   out[m][n] = bf16(sum_k a[m][k] 2^(sa[m][k/32]-127)
+ *                          * w[g][n][k] 2^(sw[g][n][k/32]-127))
+ * for each row m of group g = [offs[g-1], offs[g]).
+ *   a       e4m3 (M, K) row-major, 16-byte aligned.
+ *   sfa     A's E8M0 scales in the grouped blocked layout of
+ *           mx_scales_to_blocked_grouped (groups along rows, each group's
+ *           rows padded to 128): mx_blocked_grouped_rows_bound(M, G) * K/32
+ *           bytes, as mx_quant_rowwise_blocked_grouped writes them; 16-byte
+ *           aligned.
+ *   w       e4m3 (num_groups, N, K) row-major, 16-byte aligned.
+ *   sfw     W's E8M0 scales, the (num_groups * N, K/32) matrix in the same
+ *           blocked layout with one group (N % 128 == 0, so experts need no
+ *           padding); 16-byte aligned.
+ *   offs    num_groups int32 ends along M (device).
+ *   out     bf16 (M, N) row-major, 16-byte aligned; rows past
+ *           offs[num_groups-1] are not written.
+ *   N % 128 == 0 and K % 128 == 0 (K > 0), else MXQ_ERR_SHAPE;
+ *   num_groups <= 4096, else MXQ_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------ */
+int mx_grouped_gemm(const void *a, const void *sfa, const void *w, const void *sfw,
+                    int64_t M, int64_t N, int64_t K,
+                    const int32_t *offs, int32_t num_groups, void *out,
+                    cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * fp8_grouped_gemm_wgrad - the backward consumer of the jagged ops (#2064
  * Summary: the per-group scaled operands of the grad_weight grouped GEMM),
  * on the tensor cores:

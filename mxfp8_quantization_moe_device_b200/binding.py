@@ -39,6 +39,7 @@ SIGNATURES = {
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "fp8_grouped_gemm_rowwise": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
+    "mx_grouped_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
     "mx_blocked_grouped_rows_bound": (_i64, [_i64, _i32]),
@@ -354,6 +355,39 @@ def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, *, out=None):
     rc = lib().fp8_grouped_gemm_rowwise(_ptr(a), _ptr(inv_a), _ptr(w), _ptr(inv_w), M, N, K, _ptr(offs), E,
                                         _ptr(out), _stream(dev))
     _check("fp8_grouped_gemm_rowwise", rc)
+    return out
+
+
+def mx_grouped_gemm(a, sfa, w, sfw, offs, *, out=None):
+    """MXFP8 block-scaled grouped GEMM on the tensor cores: out[m] = sum_k
+    a[m][k] 2^(sa-127) * w[g][n][k] 2^(sw-127) for the rows m of group g.
+    a (M, K) e4m3 row-major; sfa the flat blocked E8M0 scales of A with groups
+    along rows (as mx_quant_rowwise_blocked_grouped or
+    mx_scales_to_blocked_grouped returns them); w (E, N, K) e4m3; sfw the flat
+    blocked scales of W viewed as (E*N, K/32) with one group; offs (E,) int32
+    group ends along M. Returns out (M, N) bf16; rows past offs[-1] are not
+    written."""
+    for t, n in ((a, "a"), (sfa, "sfa"), (w, "w"), (sfw, "sfw")):
+        _cuda(t, n)
+        if not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous")
+    if a.element_size() != 1 or w.element_size() != 1 or a.dim() != 2 or w.dim() != 3:
+        raise TypeError("a must be (M, K) and w (E, N, K), one byte per element (e4m3)")
+    if sfa.element_size() != 1 or sfw.element_size() != 1:
+        raise TypeError("sfa and sfw must be byte (E8M0) tensors")
+    dev = a.device
+    _offsets(offs, dev)
+    M, K = a.shape
+    E, N, K2 = w.shape
+    if K2 != K or offs.numel() != E or K % 128 or N % 128:
+        raise TypeError("shape mismatch between a, w and offs, or N, K not multiples of 128")
+    if sfa.numel() < blocked_grouped_rows_bound(M, E) * (K // 32) or sfw.numel() < E * N * (K // 32):
+        raise TypeError("scale buffers smaller than the blocked layout needs")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    rc = lib().mx_grouped_gemm(_ptr(a), _ptr(sfa), _ptr(w), _ptr(sfw), M, N, K, _ptr(offs), E, _ptr(out),
+                               _stream(dev))
+    _check("mx_grouped_gemm", rc)
     return out
 
 

@@ -12,6 +12,7 @@
 #include "jagged.cuh"
 #include "blocked.cuh"
 #include "gemm.cuh"
+#include "gemm_mx.cuh"
 
 using namespace mxq;
 
@@ -102,6 +103,8 @@ int device_info(const DevInfo **out)
                                  (int)(gm::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(gm::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mx_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gmx::smem_fixed() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::smem_fixed<128>()) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -418,6 +421,47 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
     return launch(k_fp8_grouped_gemm<128>, dim3((unsigned)grid), dim3(gm::THREADS),
                   gm::smem_fixed<128>() + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M, N,
                   K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+}
+
+int mx_grouped_gemm(const void *a, const void *sfa, const void *w, const void *sfw, int64_t M, int64_t N, int64_t K,
+                    const int32_t *offs, int32_t num_groups, void *out, cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % 128 || K % gmx::BK)
+        return MXQ_ERR_SHAPE;
+    if (num_groups > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0)
+        return MXQ_OK;
+    if (K == 0)
+        return MXQ_ERR_SHAPE;
+    if (!a || !sfa || !w || !sfw || !offs || !out)
+        return MXQ_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(w, 16) || !aligned(out, 16) || !aligned(sfa, 16) || !aligned(sfw, 16))
+        return MXQ_ERR_ALIGN;
+    if (M >= (int64_t(1) << 31) || (int64_t)num_groups * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    CUtensorMap ta, tw;
+    const uint64_t da[2] = {(uint64_t)K, (uint64_t)M};
+    const uint64_t sa[1] = {(uint64_t)K};
+    const uint32_t box[2] = {gmx::BK, gmx::BM};
+    rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t dw[2] = {(uint64_t)K, (uint64_t)(num_groups * N)};
+    const uint32_t boxw[2] = {gmx::BK, (uint32_t)gmx::BN};
+    rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, dw, sa, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t items = (M / gmx::BM + num_groups) * (N / gmx::BN);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, di->sms));
+    return launch(k_mx_grouped_gemm, dim3((unsigned)grid), dim3(gmx::THREADS),
+                  gmx::smem_fixed() + (size_t)num_groups * sizeof(int), stream, false, ta, tw,
+                  static_cast<const uint8_t *>(sfa), static_cast<const uint8_t *>(sfw), M, N, K, offs,
+                  (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
 }
 
 int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, const float *inv_b, int64_t N,

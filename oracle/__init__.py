@@ -51,6 +51,8 @@ def lib():
                                                                _i32, ctypes.POINTER(ctypes.c_double)]),
             "oracle_fp8_grouped_gemm_wgrad": (ctypes.c_int, [_u8p, _f32p, _u8p, _f32p, _i64, _i64, _i64, _i32p,
                                                              _i32, ctypes.POINTER(ctypes.c_double)]),
+            "oracle_mx_grouped_gemm": (ctypes.c_int, [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i32p, _i32,
+                                                      ctypes.POINTER(ctypes.c_double)]),
             "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
@@ -193,6 +195,24 @@ def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, out=None):
     res = np.zeros((M, N), dtype=np.float64) if out is None else np.ascontiguousarray(out, dtype=np.float64)
     _check(lib().oracle_fp8_grouped_gemm_rowwise(_p(a, _u8p), _p(ia, _f32p), _p(w, _u8p), _p(iw, _f32p), M, N, K,
                                                  _p(o, _i32p), E, res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return res
+
+
+def mx_grouped_gemm(a, sa, w, sw, offs):
+    """a (M, K) e4m3 codes with E8M0 scales sa (M, K/32), w (E, N, K) codes
+    with sw (E, N, K/32), offs (E,) group ends along M (plain row-major scale
+    layouts). Returns out (M, N) float64; rows past the last offset are 0."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    w = np.ascontiguousarray(w, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.uint8)
+    sw = np.ascontiguousarray(sw, dtype=np.uint8)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    M, K = a.shape
+    E, N, K2 = w.shape
+    assert K2 == K and len(o) == E and sa.shape == (M, K // 32) and sw.shape == (E, N, K // 32)
+    res = np.zeros((M, N), dtype=np.float64)
+    _check(lib().oracle_mx_grouped_gemm(_p(a, _u8p), _p(sa, _u8p), _p(w, _u8p), _p(sw, _u8p), M, N, K,
+                                        _p(o, _i32p), E, res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
     return res
 
 

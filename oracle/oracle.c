@@ -557,6 +557,49 @@ int oracle_fp8_grouped_gemm_rowwise(const uint8_t *a, const float *inv_a, const 
 }
 
 /* ------------------------------------------------------------------ */
+/* MXFP8 block-scaled grouped GEMM, the consumer of the MX rowwise      */
+/* quantization and of the blocked scale layout (#3504 title: blocked   */
+/* scales per group for MXFP8 MoE training; reading R18: they feed the  */
+/* MoE layer's grouped GEMM). By the OCP MX definition an element's     */
+/* value is its e4m3 value times 2^(e - 127)                            */
+/* of its block's E8M0 byte e (255 is NaN), blocks being 32 consecutive */
+/* elements along K. Row m of group g:                                  */
+/*   out[m][n] = sum_k x(a[m][k], sa[m][k/32]) * x(w[g][n][k], sw[g][n][k/32]) */
+/* with x(c, e) = e4m3(c) * 2^(e-127); the scales are passed in their    */
+/* plain row-major layouts, sa (M, K/32) and sw (G, N, K/32). In double */
+/* (each product is exact; the sum of K of them is exact far below fp32 */
+/* resolution). Rows past offs[G-1] are not written.                     */
+/* ------------------------------------------------------------------ */
+static double e8m0_value(uint8_t e)
+{
+    return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
+}
+
+int oracle_mx_grouped_gemm(const uint8_t *a, const uint8_t *sa, const uint8_t *w, const uint8_t *sw,
+                           int64_t M, int64_t N, int64_t K, const int32_t *offs, int32_t groups, double *out)
+{
+    int64_t start = 0, kb = K / 32;
+    if (M < 0 || N < 0 || K < 0 || K % 32 || groups <= 0)
+        return ORACLE_ERR_ARG;
+    if (!offsets_valid(offs, groups, M))
+        return ORACLE_ERR_OFFSETS;
+    for (int32_t g = 0; g < groups; ++g) {
+        const uint8_t *wg = w + (int64_t)g * N * K, *swg = sw + (int64_t)g * N * kb;
+        for (int64_t m = start; m < offs[g]; ++m) {
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += oracle_e4m3_value(a[m * K + k]) * e8m0_value(sa[m * kb + k / 32]) *
+                           (oracle_e4m3_value(wg[n * K + k]) * e8m0_value(swg[n * kb + k / 32]));
+                out[m * N + n] = acc;
+            }
+        }
+        start = offs[g];
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Weight-gradient grouped GEMM, the backward consumer of the jagged    */
 /* ops (#2064 Summary: the per-group scaled operands of the grad_weight */
 /* grouped GEMM). The contraction runs over each group's own positions: */

@@ -47,6 +47,8 @@ int oracle_fp8_quant_blockwise_transposed(const uint16_t *in, int64_t rows, int6
 int oracle_fp8_grouped_gemm_rowwise(const uint8_t *a, const float *inv_a, const uint8_t *w, const float *inv_w,
                                     int64_t M, int64_t N, int64_t K, const int32_t *offs, int32_t groups,
                                     double *out);
+int oracle_mx_grouped_gemm(const uint8_t *a, const uint8_t *sa, const uint8_t *w, const uint8_t *sw,
+                           int64_t M, int64_t N, int64_t K, const int32_t *offs, int32_t groups, double *out);
 int oracle_fp8_grouped_gemm_wgrad(const uint8_t *a, const float *inv_a, const uint8_t *b, const float *inv_b,
                                   int64_t N, int64_t K, int64_t M, const int32_t *offs, int32_t groups,
                                   double *out);

@@ -143,3 +143,52 @@ def test_wgrad_gemm_vs_oracle(M, N, K, ends):
     _check_wgrad(out, a, ia, b, ib, offs)
     assert bool((out[1] == 0).all()) if ends[1] == ends[0] else True
 
+
+
+# ---------------------------------------------------------------- MXFP8 block-scaled
+
+def _mx_operands(M, N, K, E, ends, mode, seed):
+    """A (M, K) and W (E*N, K) bf16 quantized by the oracle (codes, plain
+    scales) and by this library's fused MX rowwise op with blocked scales."""
+    a = synth.row_scaled_normal_bf16(M, K, seed=seed)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=seed + 1, lo=-2.0, hi=2.0)
+    m = oracle.FLOOR if mode == "floor" else oracle.RCEIL
+    qa, sa = oracle.mx_quant_rowwise(a, m)
+    qw, sw = oracle.mx_quant_rowwise(w, m)
+    offs = torch.tensor(ends, dtype=torch.int32, device=DEV)
+    dqa, dsa, _ = mxq.mx_quant_rowwise_blocked_grouped(a.to(DEV), offs, mode)
+    one = torch.tensor([E * N], dtype=torch.int32, device=DEV)
+    dqw, dsw, _ = mxq.mx_quant_rowwise_blocked_grouped(w.to(DEV), one, mode)
+    assert np.array_equal(dqa.view(torch.uint8).cpu().numpy(), qa)  # the quantization itself is bit-exact
+    return (qa, sa, qw.reshape(E, N, K), sw.reshape(E, N, K // 32)), \
+        (dqa.view(torch.uint8), dsa, dqw.view(torch.uint8).reshape(E, N, K), dsw, offs)
+
+
+def _check_mx(out, qa, sa, qw, sw, ends, K):
+    ref = oracle.mx_grouped_gemm(qa, sa, qw, sw, ends)
+    dec = np.abs(np.array([oracle.e4m3_value(c) for c in range(256)]))
+    xa = dec[qa] * np.repeat(2.0 ** (sa.astype(np.float64) - 127), 32, axis=1)
+    xw = dec[qw] * np.repeat(2.0 ** (sw.astype(np.float64) - 127), 32, axis=2)
+    end, start = ends[-1], 0
+    got = out[:end].float().cpu().numpy().astype(np.float64)
+    for g, e in enumerate(ends):
+        if e > start:
+            S = xa[start:e] @ xw[g].T
+            bound = 2.0 ** -8 * np.abs(ref[start:e]) + K * 2.0 ** -23 * S
+            excess = np.max(np.abs(got[start:e] - ref[start:e]) - bound)
+            assert excess <= 0, (g, excess)
+        start = e
+
+
+@pytest.mark.parametrize("M,N,K,ends,mode", [
+    (300, 128, 256, [100, 100, 290], "floor"),     # an empty group; rows past the last group
+    (129, 256, 128, [1, 129], "rceil"),            # a one-row group; K of one stage
+    (1000, 384, 1024, [250, 300, 700, 1000], "floor"),
+])
+def test_mx_grouped_gemm_vs_oracle(M, N, K, ends, mode):
+    (qa, sa, qw, sw), (dqa, dsa, dqw, dsw, offs) = _mx_operands(M, N, K, len(ends), ends, mode, seed=M + K)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    mxq.mx_grouped_gemm(dqa, dsa, dqw, dsw, offs, out=out)
+    assert mxq.device_status() == 0
+    _check_mx(out, qa, sa, qw, sw, ends, K)
+    assert bool(torch.isnan(out[ends[-1]:]).all())  # rows past the last group untouched

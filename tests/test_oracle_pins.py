@@ -669,3 +669,80 @@ def test_oracle_rejects_bad_offsets(oracle):
         with pytest.raises(oracle.OracleError) as ei:
             oracle.fp8_quant_jagged_colwise(w, 16, 4, 4, 1, offs)
         assert ei.value.code == oracle.ERR_OFFSETS
+
+
+# ---------------------------------------------------------------- MXFP8 grouped GEMM (R18)
+
+def test_mx_gemm_unit_scales_equal_the_fp8_gemm(oracle):
+    """With every E8M0 byte 127 (factor 2^0) the MX grouped GEMM is the FP8
+    grouped GEMM with unit inverse scales: pins the e4m3 decoding, the
+    grouping and the rows past the last group through the other GEMM."""
+    rng = np.random.default_rng(21)
+    M, N, K, E = 70, 24, 64, 3
+    a = rng.integers(0, 256, size=(M, K), dtype=np.uint8)
+    w = rng.integers(0, 256, size=(E, N, K), dtype=np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0
+    w[(w & 0x7F) == 0x7F] = 0
+    offs = np.array([20, 20, 64], dtype=np.int32)
+    got = oracle.mx_grouped_gemm(a, np.full((M, K // 32), 127, np.uint8), w, np.full((E, N, K // 32), 127, np.uint8),
+                                 offs)
+    ref = oracle.fp8_grouped_gemm_rowwise(a, np.ones(M, np.float32), w, np.ones((E, N), np.float32), offs)
+    assert np.array_equal(got, ref)
+    assert not got[64:].any()
+
+
+def test_mx_gemm_scale_bytes_act_per_32_block(oracle):
+    """Raising one A scale byte by one doubles exactly that 32-element block's
+    contribution, and one W byte by two quadruples its block's: the scale is
+    2^(byte - 127) and covers elements 32j .. 32j+31 along K."""
+    rng = np.random.default_rng(22)
+    M, N, K = 4, 3, 96
+    a = rng.integers(0, 0x7E, size=(M, K), dtype=np.uint8)
+    w = rng.integers(0, 0x7E, size=(1, N, K), dtype=np.uint8)
+    sa = rng.integers(120, 135, size=(M, K // 32), dtype=np.uint8)
+    sw = rng.integers(120, 135, size=(1, N, K // 32), dtype=np.uint8)
+    offs = np.array([M], np.int32)
+    base = oracle.mx_grouped_gemm(a, sa, w, sw, offs)
+
+    def block_only(j):  # the contribution of K block j alone
+        a2 = a.copy()
+        a2[:, [k for k in range(K) if k // 32 != j]] = 0
+        return oracle.mx_grouped_gemm(a2, sa, w, sw, offs)
+    sa2 = sa.copy()
+    sa2[1, 2] += 1
+    got = oracle.mx_grouped_gemm(a, sa2, w, sw, offs)
+    assert np.allclose(got[1], base[1] + block_only(2)[1], rtol=1e-14, atol=0)
+    assert np.array_equal(np.delete(got, 1, 0), np.delete(base, 1, 0))
+    sw2 = sw.copy()
+    sw2[0, 2, 0] += 2
+    got = oracle.mx_grouped_gemm(a, sa, w, sw2, offs)
+    assert np.allclose(got[:, 2], base[:, 2] + 3 * block_only(0)[:, 2], rtol=1e-14, atol=0)
+    assert np.array_equal(got[:, :2], base[:, :2])
+
+
+def test_mx_gemm_hand_example(oracle):
+    """One row, K = 64: a = 1.0 (0x38) in block 0 and 2.0 (0x40) in block 1
+    with scale bytes 128 (x2) and 126 (x0.5); w = 0.5 (0x30) everywhere with
+    bytes 127 and 129 (x1, x4): 32*(2*0.5) + 32*(1*2) = 96."""
+    a = np.array([[0x38] * 32 + [0x40] * 32], dtype=np.uint8)
+    w = np.array([[[0x30] * 64]], dtype=np.uint8)
+    got = oracle.mx_grouped_gemm(a, np.array([[128, 126]], np.uint8), w, np.array([[[127, 129]]], np.uint8),
+                                 np.array([1], np.int32))
+    assert got[0, 0] == 96.0
+
+
+def test_mx_pipeline_approximates_the_exact_product(oracle):
+    """MX rowwise quantization of both operands followed by the MX grouped
+    GEMM approximates the exact grouped product A W_g^T within the e4m3
+    rounding (a few percent in Frobenius norm); a scale applied with the wrong
+    sign of its exponent or to the wrong block is off by order one or more."""
+    M, N, K, E = 96, 64, 128, 2
+    a = synth.row_scaled_normal_bf16(M, K, seed=31)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=32, lo=-2.0, hi=2.0)
+    qa, sa = oracle.mx_quant_rowwise(a, oracle.FLOOR)
+    qw, sw = oracle.mx_quant_rowwise(w, oracle.FLOOR)
+    ends = [40, 96]
+    got = oracle.mx_grouped_gemm(qa, sa, qw.reshape(E, N, K), sw.reshape(E, N, K // 32), ends)
+    A, W = a.double().numpy(), w.double().numpy().reshape(E, N, K)
+    want = np.concatenate([A[:40] @ W[0].T, A[40:] @ W[1].T])
+    assert np.linalg.norm(got - want) <= 0.06 * np.linalg.norm(want)
