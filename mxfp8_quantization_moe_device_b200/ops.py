@@ -233,6 +233,24 @@ def _(a, inv_a, w, inv_w, offs):
     return a.new_empty((a.shape[0], w.shape[1]), dtype=torch.bfloat16)
 
 
+@torch.library.custom_op("mxq::mx_grouped_gemm", mutates_args=())
+def mx_grouped_gemm(a: torch.Tensor, sfa: torch.Tensor, w: torch.Tensor, sfw: torch.Tensor,
+                    offs: torch.Tensor) -> torch.Tensor:
+    """MXFP8 block-scaled grouped GEMM: (M, N) bf16, row m of group g = sum_k
+    a[m,k] 2^(sa-127) w[g,n,k] 2^(sw-127), scales in the blocked layouts;
+    rows past offs[-1] are zero."""
+    M = a.shape[0]
+    N = w.shape[1]
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device=a.device)
+    _b.mx_grouped_gemm(a.view(torch.uint8), sfa, w.view(torch.uint8), sfw, offs, out=out)
+    return out
+
+
+@mx_grouped_gemm.register_fake
+def _(a, sfa, w, sfw, offs):
+    return a.new_empty((a.shape[0], w.shape[1]), dtype=torch.bfloat16)
+
+
 @torch.library.custom_op("mxq::fp8_grouped_gemm_wgrad", mutates_args=())
 def fp8_grouped_gemm_wgrad(a: torch.Tensor, inv_a: torch.Tensor, b: torch.Tensor, inv_b: torch.Tensor,
                            offs: torch.Tensor) -> torch.Tensor:

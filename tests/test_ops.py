@@ -12,7 +12,7 @@ from mxfp8_quantization_moe_device_b200 import synth
 OPS = ["fp8_quant_jagged_rowwise", "fp8_quant_jagged_colwise", "fp8_quant_blockwise",
        "fp8_quant_blockwise_transposed", "mx_quant_3d_colwise", "mx_quant_rowwise", "mx_scales_to_blocked_grouped",
        "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped", "fp8_grouped_gemm_rowwise",
-       "fp8_grouped_gemm_wgrad"]
+       "fp8_grouped_gemm_wgrad", "mx_grouped_gemm"]
 
 
 def _cases(dev):
@@ -54,6 +54,15 @@ def test_gemm_fake_shape_on_meta_tensors():
     out = torch.ops.mxq.fp8_grouped_gemm_rowwise(a, torch.empty(300, device="meta"), w,
                                                  torch.empty((3, 128), device="meta"),
                                                  torch.empty(3, dtype=torch.int32, device="meta"))
+    assert tuple(out.shape) == (300, 128) and out.dtype == torch.bfloat16
+
+
+def test_mx_gemm_fake_shape_on_meta_tensors():
+    a = torch.empty((300, 256), dtype=torch.float8_e4m3fn, device="meta")
+    w = torch.empty((3, 128, 256), dtype=torch.float8_e4m3fn, device="meta")
+    out = torch.ops.mxq.mx_grouped_gemm(a, torch.empty(640 * 8, dtype=torch.uint8, device="meta"), w,
+                                        torch.empty(384 * 8, dtype=torch.uint8, device="meta"),
+                                        torch.empty(3, dtype=torch.int32, device="meta"))
     assert tuple(out.shape) == (300, 128) and out.dtype == torch.bfloat16
 
 
@@ -133,6 +142,20 @@ def test_gemm_op_matches_the_binding():
     mxq.fp8_grouped_gemm_rowwise(a.view(torch.uint8), ia.reshape(300).contiguous(),
                                  w.view(torch.uint8).reshape(3, 128, 256), iw.reshape(3, 128).contiguous(), offs,
                                  out=ref)
+    assert torch.equal(got, ref)
+
+
+@gpu
+def test_mx_gemm_op_matches_the_binding():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    offs = torch.tensor([100, 100, 290], dtype=torch.int32, device="cuda")
+    qa, sa, _ = mxq.mx_quant_rowwise_blocked_grouped(synth.normal_bf16((300, 256), 1.0, 1, device="cuda"), offs)
+    w = synth.normal_bf16((3 * 128, 256), 0.02, 2, device="cuda")
+    qw, sw, _ = mxq.mx_quant_rowwise_blocked_grouped(w, torch.tensor([384], dtype=torch.int32, device="cuda"))
+    got = torch.ops.mxq.mx_grouped_gemm(qa, sa, qw.reshape(3, 128, 256), sw, offs)
+    ref = torch.zeros_like(got)
+    mxq.mx_grouped_gemm(qa.view(torch.uint8), sa, qw.view(torch.uint8).reshape(3, 128, 256), sw, offs, out=ref)
     assert torch.equal(got, ref)
 
 
