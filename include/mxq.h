@@ -383,10 +383,13 @@ int mxq_version(void);
  *                              bounded waits on it expire and report
  *                              MXQ_ERR_TIMEOUT; 0 turns it off.
  *   MXQ_TESTING_FORCE_PATH     jagged ops: 0 automatic, 1 two-pass TMA
- *                              kernels (amax, then cast), 2 generic kernel. */
+ *                              kernels (amax, then cast), 2 generic kernel.
+ *   MXQ_TESTING_GEMM_TILE_N    mx_grouped_gemm tile width: 0 automatic (256
+ *                              when N % 256 == 0, else 128), 128 forced. */
 #define MXQ_TESTING_WAIT_LIMIT_NS 1
 #define MXQ_TESTING_SKIP_ARRIVAL 2
 #define MXQ_TESTING_FORCE_PATH 3
+#define MXQ_TESTING_GEMM_TILE_N 4
 int mxq_testing_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

@@ -17,10 +17,12 @@
 // viewed as one (E*N, K/32) matrix in the same layout (N % 128 == 0, so no
 // padding between experts). Rows past offs[G-1] are not written.
 //
-// The pipeline is the FP8 grouped GEMM's with 128 x 128 tiles; what changes:
+// The pipeline is the FP8 grouped GEMM's (128 x BN tiles, BN = 256 when N
+// allows, with one accumulator then: two would fill TMEM); what changes:
 //   - each stage also carries the 512-byte scale tile of A (the m-tile's index
 //     is its row tile in the blocked layout, since both pad every group to
-//     128 rows) and of W, fetched with bulk copies on the stage's barrier;
+//     128 rows) and the BN/128 tiles of W, fetched with bulk copies on the
+//     stage's barrier;
 //   - the MMA thread copies both into TMEM with tcgen05.cp 32x128b.warpx4
 //     (lane r % 32, column r / 32, byte = the K/32 block within the stage:
 //     exactly the blocked tile's order) and issues tcgen05.mma
@@ -34,33 +36,42 @@
 namespace mxq {
 namespace gmx {
 
-constexpr int BM = gm::BM, BK = gm::BK, BN = 128;
-constexpr int STAGES = gm::STAGES, ACC = gm::ACC, THREADS = gm::THREADS;
-constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK;
+constexpr int BM = gm::BM, BK = gm::BK;
+constexpr int STAGES = gm::STAGES, THREADS = gm::THREADS;
+constexpr int A_BYTES = BM * BK;
 constexpr int SF_BYTES = 512;           // one 128 x 4 blocked scale tile
-constexpr int SF_COL = ACC * BN;        // TMEM columns of the scales, after the accumulators
-constexpr int TMEM_COLS = 512;          // a power of two >= SF_COL + STAGES * 8
+constexpr int TMEM_COLS = 512;
+// per tile width: accumulators, TMEM column of the scales (after the
+// accumulators), scale columns per stage (4 for A, 4 per 128 rows of W)
+template <int BN> struct Cfg {
+    static constexpr int ACC = BN == 256 ? 1 : 2;
+    static constexpr int B_BYTES = BN * BK;
+    static constexpr int SF_COL = ACC * BN;
+    static constexpr int SF_STAGE_COLS = 4 + 4 * (BN / 128);
+    static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scales fit after the accumulators");
+};
 
-struct __align__(1024) Smem {
+template <int BN> struct __align__(1024) Smem {
     uint8_t a[STAGES][A_BYTES];
-    uint8_t b[STAGES][B_BYTES];
+    uint8_t b[STAGES][BN * BK];
     uint8_t sfa[STAGES][SF_BYTES];
-    uint8_t sfb[STAGES][SF_BYTES];
+    uint8_t sfb[STAGES][SF_BYTES * (BN / 128)];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t acc_full[ACC];
-    uint64_t acc_empty[ACC];
+    uint64_t acc_full[2];   // [0, Cfg<BN>::ACC) initialized and used
+    uint64_t acc_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort_flag;
     int Tend;
 };
-constexpr size_t smem_fixed() { return sizeof(Smem) + 1024; }
+template <int BN> constexpr size_t smem_fixed() { return sizeof(Smem<BN>) + 1024; }
 
 // instruction descriptor of kind::mxf8f6f4.block_scale: A and B e4m3
 // (format 0), both K-major, N, E8M0 scale factors (bit 23), M; the scale
 // bytes are picked per instruction by the ids in bits 4-5 (B) and 29-30 (A)
-constexpr uint32_t IDESC = ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+template <int BN>
+constexpr uint32_t idesc() { return ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24); }
 
 // shared-memory descriptor of a scale tile as tcgen05.cp reads it: 32 rows
 // of 16 bytes, no swizzle, 8-row core matrices 128 bytes apart; version 1
@@ -90,6 +101,7 @@ MXQ_DEV void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t
 
 } // namespace gmx
 
+template <int BN>
 __global__ void __launch_bounds__(gmx::THREADS, 1)
     k_mx_grouped_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                       const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfw, int64_t M, int64_t N,
@@ -97,8 +109,11 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
                       uint64_t wait_ns)
 {
     using namespace gmx;
+    constexpr int ACC = Cfg<BN>::ACC, B_BYTES = Cfg<BN>::B_BYTES;
+    constexpr int SF_COL = Cfg<BN>::SF_COL, SF_STAGE_COLS = Cfg<BN>::SF_STAGE_COLS;
+    constexpr uint32_t IDESC = idesc<BN>();
     extern __shared__ uint8_t smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<BN> &sm = *reinterpret_cast<Smem<BN> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     int *T = reinterpret_cast<int *>(&sm + 1); // G group m-tile starts, after the fixed part
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -151,20 +166,22 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
                 const int64_t mt = it / ntn, nt = it - mt * ntn;
                 const int g = tile_group(mt);
                 const int64_t m0 = (g ? offs[g - 1] : 0) + (mt - T[g]) * BM;
-                const int64_t wrow = (int64_t)g * N + nt * BN; // W row, and its row tile * 128
+                const int64_t wrow = (int64_t)g * N + nt * BN; // W row; its row tile is wrow / 128
                 const uint8_t *sa = sfa + mt * nkb * SF_BYTES;
-                const uint8_t *sw = sfw + (wrow / BN) * nkb * SF_BYTES;
+                const uint8_t *sw = sfw + (wrow / 128) * nkb * SF_BYTES;
                 for (int64_t kb = 0; kb < nkb; ++kb, ++seq) {
                     const int s = seq % STAGES;
                     if (seq >= STAGES && !mbar_wait(&sm.empty[s], ((uint32_t)(seq / STAGES) & 1u) ^ 1u, wait_ns)) {
                         *reinterpret_cast<volatile int *>(&sm.abort_flag) = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES + 2 * SF_BYTES);
+                    mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES + SF_BYTES * (1 + BN / 128));
                     tma_load_2d(sm.a[s], &tm_a, &sm.full[s], (int)(kb * BK), (int)m0);
                     tma_load_2d(sm.b[s], &tm_w, &sm.full[s], (int)(kb * BK), (int)wrow);
                     bulk_load(sm.sfa[s], sa + kb * SF_BYTES, SF_BYTES, &sm.full[s]);
-                    bulk_load(sm.sfb[s], sw + kb * SF_BYTES, SF_BYTES, &sm.full[s]);
+#pragma unroll
+                    for (int h = 0; h < BN / 128; ++h) // W row tiles wrow/128 + h: nkb tiles apart
+                        bulk_load(sm.sfb[s] + h * SF_BYTES, sw + (h * nkb + kb) * SF_BYTES, SF_BYTES, &sm.full[s]);
                 }
             }
             for (int j = seq - STAGES; j < seq; ++j)
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
             int seq = 0, t = 0;
             bool issued = false;
             for (int64_t it = blockIdx.x; it < total && !gm::aborted(&sm.abort_flag); it += gridDim.x, ++t) {
-                const int acc = t & 1;
+                const int acc = t % ACC; // one accumulator at BN 256: every tile waits for the last epilogue
                 if (t >= ACC && !mbar_wait(&sm.acc_empty[acc], ((uint32_t)(t / ACC) & 1u) ^ 1u, wait_ns)) {
                     *reinterpret_cast<volatile int *>(&sm.abort_flag) = 1;
                     break;
@@ -195,9 +212,11 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
                     // this stage's scales into its own TMEM columns; the copy and
                     // the MMAs below run in issue order, and the columns are
                     // rewritten only after this stage's MMAs have committed
-                    const uint32_t sft = tmem + (uint32_t)(SF_COL + s * 8);
+                    const uint32_t sft = tmem + (uint32_t)(SF_COL + s * SF_STAGE_COLS);
                     tc_cp_sf(sft, sf_desc(smem_u32(sm.sfa[s])));
-                    tc_cp_sf(sft + 4, sf_desc(smem_u32(sm.sfb[s])));
+#pragma unroll
+                    for (int h = 0; h < BN / 128; ++h) // W rows 128h.. of the tile: 4 columns each
+                        tc_cp_sf(sft + 4 + 4 * h, sf_desc(smem_u32(sm.sfb[s] + h * SF_BYTES)));
                     const uint64_t ad = gm::smem_desc_k128(smem_u32(sm.a[s]));
                     const uint64_t bd = gm::smem_desc_k128(smem_u32(sm.b[s]));
 #pragma unroll
@@ -226,7 +245,7 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
         // ------------------------------------------------ epilogue (warps 0-3, TMEM lanes 32w..32w+31)
         int t = 0;
         for (int64_t it = blockIdx.x; it < total; it += gridDim.x, ++t) {
-            const int acc = t & 1;
+            const int acc = t % ACC;
             bool ok = mbar_wait(&sm.acc_full[acc], (uint32_t)(t / ACC) & 1u, wait_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok || gm::aborted(&sm.abort_flag)) {

@@ -21,6 +21,7 @@ namespace {
 std::atomic<int64_t> g_wait_ns{1000000000LL};
 std::atomic<int> g_drop_load{0};
 std::atomic<int> g_force_path{0};
+std::atomic<int> g_mx_bn{0}; // MX grouped GEMM tile width: 0 automatic, 128 forced
 
 uint64_t wait_ns() { return (uint64_t)g_wait_ns.load(); }
 
@@ -103,8 +104,10 @@ int device_info(const DevInfo **out)
                                  (int)(gm::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(gm::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
-            cudaFuncSetAttribute(k_mx_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(gmx::smem_fixed() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mx_grouped_gemm<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gmx::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mx_grouped_gemm<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gmx::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::smem_fixed<128>()) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -451,17 +454,23 @@ int mx_grouped_gemm(const void *a, const void *sfa, const void *w, const void *s
     rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
+    // tiles 128 x 256 when N allows (one accumulator), else 128 x 128 (two)
+    const int bn = N % 256 == 0 && g_mx_bn.load() != 128 ? 256 : 128;
     const uint64_t dw[2] = {(uint64_t)K, (uint64_t)(num_groups * N)};
-    const uint32_t boxw[2] = {gmx::BK, (uint32_t)gmx::BN};
+    const uint32_t boxw[2] = {gmx::BK, (uint32_t)bn};
     rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, dw, sa, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
-    const int64_t items = (M / gmx::BM + num_groups) * (N / gmx::BN);
+    const int64_t items = (M / gmx::BM + num_groups) * (N / bn);
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, di->sms));
-    return launch(k_mx_grouped_gemm, dim3((unsigned)grid), dim3(gmx::THREADS),
-                  gmx::smem_fixed() + (size_t)num_groups * sizeof(int), stream, false, ta, tw,
-                  static_cast<const uint8_t *>(sfa), static_cast<const uint8_t *>(sfw), M, N, K, offs,
-                  (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+    const size_t smem_g = (size_t)num_groups * sizeof(int);
+    if (bn == 256)
+        return launch(k_mx_grouped_gemm<256>, dim3((unsigned)grid), dim3(gmx::THREADS), gmx::smem_fixed<256>() + smem_g,
+                      stream, false, ta, tw, static_cast<const uint8_t *>(sfa), static_cast<const uint8_t *>(sfw), M, N,
+                      K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+    return launch(k_mx_grouped_gemm<128>, dim3((unsigned)grid), dim3(gmx::THREADS), gmx::smem_fixed<128>() + smem_g,
+                  stream, false, ta, tw, static_cast<const uint8_t *>(sfa), static_cast<const uint8_t *>(sfw), M, N, K,
+                  offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
 }
 
 int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, const float *inv_b, int64_t N,
@@ -795,6 +804,11 @@ int mxq_testing_set(int32_t what, int64_t value)
         if (value < 0 || value > 2)
             return MXQ_ERR_UNSUPPORTED;
         g_force_path.store((int)value);
+        return MXQ_OK;
+    case MXQ_TESTING_GEMM_TILE_N:
+        if (value != 0 && value != 128)
+            return MXQ_ERR_UNSUPPORTED;
+        g_mx_bn.store((int)value);
         return MXQ_OK;
     default: return MXQ_ERR_UNSUPPORTED;
     }

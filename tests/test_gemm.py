@@ -180,15 +180,52 @@ def _check_mx(out, qa, sa, qw, sw, ends, K):
         start = e
 
 
+@pytest.mark.parametrize("tile", [0, 128], ids=["auto", "n128"])
 @pytest.mark.parametrize("M,N,K,ends,mode", [
     (300, 128, 256, [100, 100, 290], "floor"),     # an empty group; rows past the last group
-    (129, 256, 128, [1, 129], "rceil"),            # a one-row group; K of one stage
+    (129, 256, 128, [1, 129], "rceil"),            # a one-row group; K of one stage; 256-wide tiles
     (1000, 384, 1024, [250, 300, 700, 1000], "floor"),
+    (520, 512, 384, [7, 260, 260, 515], "rceil"),  # 256-wide tiles over two n-tiles, ragged groups
 ])
-def test_mx_grouped_gemm_vs_oracle(M, N, K, ends, mode):
+def test_mx_grouped_gemm_vs_oracle(M, N, K, ends, mode, tile):
     (qa, sa, qw, sw), (dqa, dsa, dqw, dsw, offs) = _mx_operands(M, N, K, len(ends), ends, mode, seed=M + K)
     out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
-    mxq.mx_grouped_gemm(dqa, dsa, dqw, dsw, offs, out=out)
+    mxq.testing_set(mxq.TESTING_GEMM_TILE_N, tile)
+    try:
+        mxq.mx_grouped_gemm(dqa, dsa, dqw, dsw, offs, out=out)
+    finally:
+        mxq.testing_set(mxq.TESTING_GEMM_TILE_N, 0)
     assert mxq.device_status() == 0
     _check_mx(out, qa, sa, qw, sw, ends, K)
     assert bool(torch.isnan(out[ends[-1]:]).all())  # rows past the last group untouched
+
+
+@pytest.mark.parametrize("tile", [0, 128], ids=["auto", "n128"])
+def test_mx_grouped_gemm_many_tiles_per_cta_sampled(tile):
+    """More work items than SMs, so every persistent CTA runs several tiles
+    and cycles its accumulators and barriers: (8192, 512) tokens in 8
+    Dirichlet groups x 8 experts (1024, 512); three rows of every group and
+    the last row of each checked against the oracle."""
+    M, N, K, E = 8192, 1024, 512, 8
+    a = synth.row_scaled_normal_bf16(M, K, seed=41, device=DEV)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=42, device=DEV, lo=-2.0, hi=2.0)
+    offs = synth.dirichlet_offsets(M, E, 0.5, 43).to(DEV)
+    dqa, dsa, _ = mxq.mx_quant_rowwise_blocked_grouped(a, offs, "floor")
+    dqw, dsw, _ = mxq.mx_quant_rowwise_blocked_grouped(w, torch.tensor([E * N], dtype=torch.int32, device=DEV),
+                                                       "floor")
+    mxq.testing_set(mxq.TESTING_GEMM_TILE_N, tile)
+    try:
+        out = mxq.mx_grouped_gemm(dqa.view(torch.uint8), dsa, dqw.view(torch.uint8).reshape(E, N, K), dsw, offs)
+    finally:
+        mxq.testing_set(mxq.TESTING_GEMM_TILE_N, 0)
+    assert mxq.device_status() == 0
+    o = offs.cpu().numpy()
+    sel = []
+    for g in range(E):
+        s0 = int(o[g - 1]) if g else 0
+        sel += sorted(set(list(range(s0, min(s0 + 3, int(o[g])))) + ([int(o[g]) - 1] if o[g] > s0 else [])))
+    qa, sa = oracle.mx_quant_rowwise(a[sel].cpu(), oracle.FLOOR)
+    qw, sw = oracle.mx_quant_rowwise(w.cpu(), oracle.FLOOR)
+    groups = np.searchsorted(o, np.array(sel), side="right")
+    ends = [int(np.sum(groups <= g)) for g in range(E)]
+    _check_mx(out[torch.tensor(sel, device=DEV)], qa, sa, qw.reshape(E, N, K), sw.reshape(E, N, K // 32), ends, K)
