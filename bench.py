@@ -82,6 +82,7 @@ KERNEL_FILES = {  # source files that define each kernel (plus common.cuh)
     "k_jagged_amax": "jagged.cuh", "k_jagged_cast": "jagged.cuh", "k_mx_3d_colwise": "mx3d.cuh",
     "k_blocked_grouped": "blocked.cuh", "k_blocked_grouped_k": "blocked.cuh", "k_mx_1x32_blocked": "blocked.cuh",
     "k_fp8_blockwise_t": "blockt.cuh", "k_fp8_grouped_gemm": "gemm.cuh", "k_fp8_grouped_gemm_wgrad": "gemm.cuh",
+    "k_mx_grouped_gemm": "gemm_mx.cuh",
 }
 
 
@@ -174,7 +175,7 @@ class Workload:
            "mx_rowwise", "blocked_grouped")
     # ops outside the step (the widened rows), built only when asked for by name
     EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked", "grouped_gemm",
-             "grouped_gemm_wgrad")
+             "grouped_gemm_wgrad", "mx_grouped_gemm")
 
     def __init__(self, dev, experts, mx3d_mode, only=None):
         import torch
@@ -285,6 +286,20 @@ class Workload:
             self.o.update(g_out=t.empty((T, N), dtype=t.bfloat16, device=dev))
             self.ops.append(("grouped_gemm", lambda: mxq.fp8_grouped_gemm_rowwise(
                 self.g_a, self.g_ia, self.g_w, self.g_iw, self.g_offs, out=self.o["g_out"]), 2 * T * N * K))
+
+        if "mx_grouped_gemm" in want:
+            # the same MoE shape in MXFP8: codes and blocked scales from the fused MX rowwise op
+            T, K, E, N = 16384, 7168, 16, 2048
+            self.x_offs = synth.dirichlet_offsets(T, E, 0.3, 8).to(dev)
+            x = synth.normal_bf16((T, K), 1.0, seed=7, device=dev)
+            w = synth.normal_bf16((E * N, K), 0.02, seed=12, device=dev)
+            qa, sa, _ = mxq.mx_quant_rowwise_blocked_grouped(x, self.x_offs, "floor")
+            qw, sw, _ = mxq.mx_quant_rowwise_blocked_grouped(w, t.tensor([E * N], dtype=t.int32, device=dev), "floor")
+            del x, w
+            self.x_a, self.x_sa, self.x_w, self.x_sw = qa.view(t.uint8), sa, qw.view(t.uint8).reshape(E, N, K), sw
+            self.o.update(x_out=t.empty((T, N), dtype=t.bfloat16, device=dev))
+            self.ops.append(("mx_grouped_gemm", lambda: mxq.mx_grouped_gemm(
+                self.x_a, self.x_sa, self.x_w, self.x_sw, self.x_offs, out=self.o["x_out"]), 2 * T * N * K))
 
         if "grouped_gemm_wgrad" in want:
             # the jagged backward config: grad_out^T (4096, 65536) and input (65536, 4096), G=16
@@ -520,7 +535,34 @@ def gemm_rows(wl, flush, reps):
     rows = [{"op": "fp8_grouped_gemm", "shape": f"({T},{K}) G=64 x (64,{N},{K})", "us": round(us, 3),
              "TFLOP/s": round(tf, 1), "frac_fp8_peak": round(tf / fp8_peak, 4), "peak_TFLOP/s": round(fp8_peak, 1),
              "peak_kind": kind}]
-    del aq, wq, out
+    del aq, wq
+    # the same shape in MXFP8: MX rowwise codes with blocked scales (one
+    # fused kernel per operand) into the block-scaled grouped GEMM
+    qa, sa, _ = mxq.mx_quant_rowwise_blocked_grouped(wl.tok, wl.offs64, "floor")
+    w = synth.normal_bf16((E * N, K), 0.02, seed=12, device=dev)
+    qw, sw, _ = mxq.mx_quant_rowwise_blocked_grouped(w, torch.tensor([E * N], dtype=torch.int32, device=dev), "floor")
+    del w
+    qa, qw = qa.view(torch.uint8), qw.view(torch.uint8).reshape(E, N, K)
+    fn = lambda: mxq.mx_grouped_gemm(qa, sa, qw, sw, wl.offs64, out=out)
+    for _ in range(5):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush_l2(torch, flush)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    us = statistics.median(ts)
+    tf = flops / (us * 1e-6) / 1e12
+    rows.append({"op": "mx_grouped_gemm", "shape": f"({T},{K}) G=64 x (64,{N},{K})", "us": round(us, 3),
+                 "TFLOP/s": round(tf, 1), "frac_fp8_peak": round(tf / fp8_peak, 4), "peak_TFLOP/s": round(fp8_peak, 1),
+                 "peak_kind": kind})
+    del qa, qw, out
     # weight gradient of the jagged backward config: grad_out^T (4096, 65536)
     # rowwise and input (65536, 4096) colwise, G=16, -> (16, 4096, 4096)
     if hasattr(wl, "grad_out"):

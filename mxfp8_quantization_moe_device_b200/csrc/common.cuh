@@ -129,15 +129,6 @@ MXQ_DEV void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y,
                  : "memory");
 }
 
-// untiled bulk copy of `bytes` from global to shared memory, counted on
-// `bar` (both addresses 16-byte aligned, bytes a multiple of 16)
-MXQ_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-
 MXQ_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 template <int N> MXQ_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }

@@ -81,6 +81,15 @@ MXQ_DEV uint64_t sf_desc(uint32_t addr)
            (uint64_t(1) << 46);
 }
 
+// untiled bulk copy of `bytes` from global to shared memory, counted on
+// `bar` (both addresses 16-byte aligned, bytes a multiple of 16)
+MXQ_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // 32 rows x 16 bytes of shared memory into TMEM lanes 0-31, columns
 // taddr .. taddr+3, repeated in the other three lane quadrants
 MXQ_DEV void tc_cp_sf(uint32_t taddr, uint64_t sdesc)
