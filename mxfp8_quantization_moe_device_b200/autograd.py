@@ -18,6 +18,14 @@ contracted dimension):
                              colwise ops)
 
 Rows of out and dA past offs[-1] (tokens routed to no expert) are zero.
+
+`mx_grouped_mm` is the MXFP8 variant: the forward and input-gradient GEMMs
+take e4m3 codes with one E8M0 scale per 32 elements along their contracted
+dimension (A and W along K by the MX rowwise op; dY along N by the same op, W
+along N by the MX 3-D colwise op, whose per-expert column-major output is
+W_e^T), the scales in the 128x4 blocked layout, through the block-scaled
+grouped GEMM; the weight gradient takes the FP8 jagged path above.
+
 Nothing here computes on the host or through torch kernels besides output
 allocation: quantization and GEMMs are the library's CUDA kernels, so a
 missing library raises instead of falling back.
@@ -105,6 +113,59 @@ class FP8GroupedMM(torch.autograd.Function):
         da = _grad_input(dy, w, offs) if ctx.needs_input_grad[0] else None
         dw = _grad_weight(dy, a, offs) if ctx.needs_input_grad[1] else None
         return da, dw, None
+
+
+def _mx_forward(a, w, offs, mode):
+    M, K = a.shape
+    E, N, _ = w.shape
+    qa, sa, _ = mxq.mx_quant_rowwise_blocked_grouped(a, offs, mode)
+    one = torch.tensor([E * N], dtype=torch.int32, device=w.device)
+    qw, sw, _ = mxq.mx_quant_rowwise_blocked_grouped(w.view(E * N, K), one, mode)
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device=a.device)
+    return mxq.mx_grouped_gemm(qa.view(torch.uint8), sa, qw.view(torch.uint8).view(E, N, K), sw, offs, out=out)
+
+
+def _mx_grad_input(dy, w, offs, mode):
+    M, N = dy.shape
+    E, _, K = w.shape
+    qdy, sdy, _ = mxq.mx_quant_rowwise_blocked_grouped(dy, offs, mode)
+    # W_e^T with 32-element blocks along N: the MX 3-D colwise op writes each
+    # expert column-major, i.e. (E, K, N) row-major, the dA GEMM's W operand
+    wt = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
+    _, sc = mxq.mx_quant_3d_colwise(w, mode, out=wt)
+    swt, _ = mxq.mx_scales_to_blocked_grouped(sc.view(E * K, N // 32),
+                                              torch.tensor([E * K], dtype=torch.int32, device=w.device))
+    da = torch.zeros((M, K), dtype=torch.bfloat16, device=dy.device)
+    return mxq.mx_grouped_gemm(qdy.view(torch.uint8), sdy, wt, swt, offs, out=da)
+
+
+class MXGroupedMM(torch.autograd.Function):
+    """MXFP8 forward and input gradient (one E8M0 scale per 32 elements along
+    each GEMM's contracted dimension: A and W along K, dY and W along N), FP8
+    jagged weight gradient (no MX weight-gradient GEMM is built)."""
+
+    @staticmethod
+    def forward(ctx, a, w, offs, mode):
+        _check(a, w, offs)
+        ctx.save_for_backward(a, w, offs)
+        ctx.mode = mode
+        return _mx_forward(a, w, offs, mode)
+
+    @staticmethod
+    def backward(ctx, dy):
+        a, w, offs = ctx.saved_tensors
+        dy = dy.to(torch.bfloat16).contiguous()
+        da = _mx_grad_input(dy, w, offs, ctx.mode) if ctx.needs_input_grad[0] else None
+        dw = _grad_weight(dy, a, offs) if ctx.needs_input_grad[1] else None
+        return da, dw, None, None
+
+
+def mx_grouped_mm(a, w, offs, mode="floor"):
+    """out (M, N) bf16 = the MXFP8 grouped product of a (M, K) bf16 tokens
+    sorted by expert and w (E, N, K) bf16 expert weights (E8M0 scales by the
+    floor or rceil rule); differentiable in a (MXFP8 input gradient) and w
+    (FP8 jagged weight gradient)."""
+    return MXGroupedMM.apply(a, w, offs, mode)
 
 
 def fp8_grouped_mm(a, w, offs):

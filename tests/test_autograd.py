@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from mxfp8_quantization_moe_device_b200 import synth
-from mxfp8_quantization_moe_device_b200.autograd import fp8_grouped_mm
+from mxfp8_quantization_moe_device_b200.autograd import fp8_grouped_mm, mx_grouped_mm
 
 DEC = np.abs(np.array([oracle.e4m3_value(c) for c in range(256)]))
 
@@ -141,5 +141,89 @@ def test_weight_only_gradient():
     wd = w.cuda().requires_grad_(True)
     out = fp8_grouped_mm(a.cuda(), wd, torch.tensor(ends, dtype=torch.int32, device="cuda"))
     out.backward(dy.cuda())
+    r, dytq, idyt, acq, iac = _oracle_pipeline(a, w, dy, ends)["dw"]
+    _check_wgrad(wd.grad, r, dytq, idyt, acq, iac, ends)
+
+
+# ---------------------------------------------------------------- MXFP8 variant
+
+def _mx_values(codes, scales, axis):
+    """e4m3 values times 2^(e-127) of their 32-element block along `axis`."""
+    return DEC_SIGNED[codes] * np.repeat(2.0 ** (scales.astype(np.float64) - 127), 32, axis=axis)
+
+
+DEC_SIGNED = np.array([oracle.e4m3_value(c) for c in range(256)])
+
+
+def _mx_oracle_pipeline(a, w, dy, offs, mode):
+    M, K = a.shape
+    E, N, _ = w.shape
+    o = np.asarray(offs, dtype=np.int32)
+    qa, sa = oracle.mx_quant_rowwise(a, mode)
+    qw, sw = oracle.mx_quant_rowwise(w.reshape(E * N, K), mode)
+    qw, sw = qw.reshape(E, N, K), sw.reshape(E, N, K // 32)
+    out = oracle.mx_grouped_gemm(qa, sa, qw, sw, o)
+    qd, sd = oracle.mx_quant_rowwise(dy, mode)
+    wt, swt = oracle.mx_quant_3d_colwise(w, mode)   # (E, K, N) codes, (E, K, N/32) scales
+    da = oracle.mx_grouped_gemm(qd, sd, wt, swt, o)
+    return dict(out=(out, qa, sa, qw, sw), da=(da, qd, sd, wt, swt))
+
+
+def _check_mx_grouped(got, ref, qa, sa, qw, sw, offs, K):
+    xa = np.abs(_mx_values(qa, sa, 1))
+    xw = np.abs(_mx_values(qw, sw, 2))
+    end, start = int(offs[-1]), 0
+    g64 = got.float().cpu().numpy().astype(np.float64)
+    for g, e in enumerate(offs):
+        if e > start:
+            S = xa[start:e] @ xw[g].T
+            bound = 2.0 ** -8 * np.abs(ref[start:e]) + K * 2.0 ** -23 * S
+            assert np.max(np.abs(g64[start:e] - ref[start:e]) - bound) <= 0, g
+        start = e
+    assert np.all(g64[end:] == 0)
+
+
+def test_mx_oracle_pipeline_approximates_the_exact_products():
+    """The MX oracle pipeline's out and dA are the exact grouped products
+    A W_g^T and dY W_g up to the e4m3 rounding of the operands; W quantized
+    along N by the 3-D colwise op is W_g^T, so a transposed operand or a
+    scale on the wrong axis is off by order one."""
+    M, N, K, ends = 256, 128, 256, [64, 64, 240]
+    E = len(ends)
+    a = synth.row_scaled_normal_bf16(M, K, seed=51)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=52, lo=-2.0, hi=2.0).reshape(E, N, K)
+    dy = synth.row_scaled_normal_bf16(M, N, seed=53, lo=-3.0, hi=1.0)
+    r = _mx_oracle_pipeline(a, w, dy, ends, oracle.FLOOR)
+    A, W, D = a.double().numpy(), w.double().numpy(), dy.double().numpy()
+    out, da, s = np.zeros((M, N)), np.zeros((M, K)), 0
+    for g, e in enumerate(ends):
+        out[s:e], da[s:e] = A[s:e] @ W[g].T, D[s:e] @ W[g]
+        s = e
+    end = ends[-1]
+    for got, want in ((r["out"][0][:end], out[:end]), (r["da"][0][:end], da[:end])):
+        assert np.linalg.norm(got - want) <= 0.08 * np.linalg.norm(want)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", ["floor", "rceil"])
+def test_mx_forward_and_backward_vs_oracle(mode):
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    M, N, K, ends = 384, 256, 128, [5, 200, 384]
+    E = len(ends)
+    a = synth.row_scaled_normal_bf16(M, K, seed=61)
+    w = synth.row_scaled_normal_bf16(E * N, K, seed=62, lo=-2.0, hi=2.0).reshape(E, N, K)
+    dy = synth.row_scaled_normal_bf16(M, N, seed=63, lo=-3.0, hi=1.0)
+    m = oracle.FLOOR if mode == "floor" else oracle.RCEIL
+    ref = _mx_oracle_pipeline(a, w, dy, ends, m)
+    offs = torch.tensor(ends, dtype=torch.int32, device="cuda")
+    ad = a.cuda().requires_grad_(True)
+    wd = w.cuda().requires_grad_(True)
+    out = mx_grouped_mm(ad, wd, offs, mode)
+    out.backward(dy.cuda())
+    r, qa, sa, qw, sw = ref["out"]
+    _check_mx_grouped(out.detach(), r, qa, sa, qw, sw, ends, K)
+    r, qd, sd, wt, swt = ref["da"]
+    _check_mx_grouped(ad.grad, r, qd, sd, wt, swt, ends, N)
     r, dytq, idyt, acq, iac = _oracle_pipeline(a, w, dy, ends)["dw"]
     _check_wgrad(wd.grad, r, dytq, idyt, acq, iac, ends)
