@@ -93,6 +93,13 @@ def test_host_checks_return_before_any_cuda_call(lib):
         binding.ERR_UNSUPPORTED
     assert lib.fp8_grouped_gemm_rowwise(fake, null, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_NULL
     assert lib.fp8_grouped_gemm_rowwise(odd, fake, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_ALIGN
+    assert lib.mx_grouped_gemm(fake, fake, fake, fake, 128, 100, 128, fake, 1, fake, null) == binding.ERR_SHAPE
+    assert lib.mx_grouped_gemm(fake, fake, fake, fake, 128, 128, 96, fake, 1, fake, null) == binding.ERR_SHAPE
+    assert lib.mx_grouped_gemm(fake, fake, fake, fake, 128, 128, 128, fake, 5000, fake, null) == \
+        binding.ERR_UNSUPPORTED
+    assert lib.mx_grouped_gemm(fake, null, fake, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_NULL
+    assert lib.mx_grouped_gemm(fake, fake, fake, odd, 128, 128, 128, fake, 1, fake, null) == binding.ERR_ALIGN
+    assert lib.mx_grouped_gemm(null, null, null, null, 0, 128, 128, null, 1, null, null) == binding.OK  # M == 0
     assert lib.fp8_grouped_gemm_wgrad(fake, fake, fake, fake, 100, 128, 128, fake, 1, fake, null) == binding.ERR_SHAPE
     assert lib.fp8_grouped_gemm_wgrad(fake, fake, fake, fake, 128, 128, 120, fake, 1, fake, null) == binding.ERR_SHAPE
     assert lib.fp8_grouped_gemm_wgrad(fake, fake, null, fake, 128, 128, 128, fake, 1, fake, null) == binding.ERR_NULL
@@ -130,3 +137,15 @@ def test_binding_refuses_cpu_tensors():
         binding.fp8_quant_blockwise(x)
     with pytest.raises(TypeError):
         binding.mx_quant_rowwise(x)
+
+
+def test_testing_hooks_accept_only_their_documented_values(lib):
+    """mxq_testing_set: unknown hooks and out-of-range values are refused;
+    every accepted value is put back to its default."""
+    assert lib.mxq_testing_set(99, 0) == binding.ERR_UNSUPPORTED
+    assert lib.mxq_testing_set(binding.TESTING_FORCE_PATH, 3) == binding.ERR_UNSUPPORTED
+    assert lib.mxq_testing_set(binding.TESTING_GEMM_TILE_N, 64) == binding.ERR_UNSUPPORTED
+    for hook, value in ((binding.TESTING_FORCE_PATH, 2), (binding.TESTING_GEMM_TILE_N, 128),
+                        (binding.TESTING_WAIT_LIMIT_NS, 5_000_000), (binding.TESTING_SKIP_ARRIVAL, 1)):
+        assert lib.mxq_testing_set(hook, value) == binding.OK
+        assert lib.mxq_testing_set(hook, 0) == binding.OK
