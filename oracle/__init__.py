@@ -53,6 +53,11 @@ def lib():
                                                              _i32, ctypes.POINTER(ctypes.c_double)]),
             "oracle_mx_grouped_gemm": (ctypes.c_int, [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i32p, _i32,
                                                       ctypes.POINTER(ctypes.c_double)]),
+            "oracle_mx_jagged_blocks": (_i64, [_i32p, _i32]),
+            "oracle_mx_quant_jagged_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _i64, _i32p, _i32, ctypes.c_int,
+                                                              _u8p, _u8p]),
+            "oracle_mx_grouped_gemm_wgrad": (ctypes.c_int, [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i32p, _i32,
+                                                            ctypes.POINTER(ctypes.c_double)]),
             "oracle_mx_quant_3d_colwise": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_quant_rowwise": (ctypes.c_int, [_u16p, _i64, _i64, ctypes.c_int, _u8p, _u8p]),
             "oracle_mx_scales_to_blocked_grouped": (ctypes.c_int, [_u8p, _i64, _i64, _i32p, _i32, _u8p, _i64, _i32p]),
@@ -213,6 +218,44 @@ def mx_grouped_gemm(a, sa, w, sw, offs):
     res = np.zeros((M, N), dtype=np.float64)
     _check(lib().oracle_mx_grouped_gemm(_p(a, _u8p), _p(sa, _u8p), _p(w, _u8p), _p(sw, _u8p), M, N, K,
                                         _p(o, _i32p), E, res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return res
+
+
+def mx_jagged_blocks(offs):
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    return lib().oracle_mx_jagged_blocks(_p(o, _i32p), len(o))
+
+
+def mx_quant_jagged_colwise(words, rows, cols, stride_row, stride_col, offs, mode):
+    """MX quantization of a (rows, cols) bf16 matrix along its rows, groups of
+    rows from offs, 32-element blocks from each group's first row. Returns
+    (out (cols, rows) codes = the column-major buffer, scales (cols, nblk))."""
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    nblk = mx_jagged_blocks(o)
+    out = np.zeros((cols, rows), dtype=np.uint8)
+    sc = np.zeros((cols, nblk), dtype=np.uint8)
+    _check(lib().oracle_mx_quant_jagged_colwise(_p(w, _u16p), rows, cols, stride_row, stride_col, _p(o, _i32p),
+                                                len(o), mode, _p(out, _u8p), _p(sc, _u8p)))
+    return out, sc
+
+
+def mx_grouped_gemm_wgrad(a, sa, b, sb, offs):
+    """a (N, M), b (K, M) e4m3 codes with per-group-block E8M0 scales sa (N,
+    nblk), sb (K, nblk); offs (G,) ends along M. Returns (G, N, K) float64."""
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.uint8)
+    sb = np.ascontiguousarray(sb, dtype=np.uint8)
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    N, M = a.shape
+    K, M2 = b.shape
+    nblk = mx_jagged_blocks(o)
+    assert M2 == M and sa.shape == (N, nblk) and sb.shape == (K, nblk)
+    res = np.zeros((len(o), N, K), dtype=np.float64)
+    _check(lib().oracle_mx_grouped_gemm_wgrad(_p(a, _u8p), _p(sa, _u8p), _p(b, _u8p), _p(sb, _u8p), N, K, M,
+                                              _p(o, _i32p), len(o),
+                                              res.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
     return res
 
 

@@ -600,6 +600,99 @@ int oracle_mx_grouped_gemm(const uint8_t *a, const uint8_t *sa, const uint8_t *w
 }
 
 /* ------------------------------------------------------------------ */
+/* MX quantization along the grouped dimension, for the weight gradient */
+/* of the MXFP8 grouped GEMM (reading R19: #3505 "integrate new cuda    */
+/* kernel for blocked layout for groups along K" implies scales grouped */
+/* along the contracted token dimension; here each group's tokens are   */
+/* cut into 32-element MX blocks starting at the group's first token,   */
+/* the last block of a group holding the remainder). Element (r, c) of  */
+/* a (rows, cols) bf16 matrix with rows grouped by offs; per column c   */
+/* and block j of group g (rows s_g + 32j .. min(s_g + 32j + 32, e_g)): */
+/* byte = E8M0(amax over the block) by `mode`, out[c * rows + r] =      */
+/* mx_element(x, byte) (column-major), scales[c * nblk + B_g + j] with  */
+/* B_g = sum_{h<g} ceil(size_h / 32) and nblk = B_G. Rows past          */
+/* offs[G-1] are not written.                                            */
+/* ------------------------------------------------------------------ */
+int64_t oracle_mx_jagged_blocks(const int32_t *offs, int32_t groups)
+{
+    int64_t n = 0, start = 0;
+    for (int32_t g = 0; g < groups; ++g) {
+        n += (offs[g] - start + 31) / 32;
+        start = offs[g];
+    }
+    return n;
+}
+
+int oracle_mx_quant_jagged_colwise(const uint16_t *in, int64_t rows, int64_t cols, int64_t stride_row,
+                                   int64_t stride_col, const int32_t *offs, int32_t groups, int mode, uint8_t *out,
+                                   uint8_t *scales)
+{
+    int64_t nblk;
+    if (rows < 0 || cols < 0 || groups <= 0)
+        return ORACLE_ERR_ARG;
+    if (!offsets_valid(offs, groups, rows))
+        return ORACLE_ERR_OFFSETS;
+    nblk = oracle_mx_jagged_blocks(offs, groups);
+    for (int64_t c = 0; c < cols; ++c) {
+        int64_t start = 0, base = 0;
+        for (int32_t g = 0; g < groups; ++g) {
+            const int64_t end = offs[g];
+            for (int64_t j = 0; start + 32 * j < end; ++j) {
+                const int64_t r0 = start + 32 * j, r1 = r0 + 32 < end ? r0 + 32 : end;
+                float amax = 0.0f;
+                uint8_t byte;
+                for (int64_t r = r0; r < r1; ++r) {
+                    float a = absf(bf16_value(in[r * stride_row + c * stride_col]));
+                    if (a > amax)
+                        amax = a;
+                }
+                byte = oracle_e8m0(amax, mode);
+                scales[c * nblk + base + j] = byte;
+                for (int64_t r = r0; r < r1; ++r)
+                    out[c * rows + r] = oracle_mx_element(bf16_value(in[r * stride_row + c * stride_col]), byte);
+            }
+            base += (end - start + 31) / 32;
+            start = end;
+        }
+    }
+    return 0;
+}
+
+/* The MXFP8 weight-gradient product over each group's tokens (R19):    */
+/*   out[g][n][k] = sum_{m in group g} x(a[n][m], sa[n][B_g + (m-s_g)/32]) */
+/*                                    * x(b[k][m], sb[k][B_g + (m-s_g)/32]) */
+/* with x(c, e) = e4m3(c) * 2^(e-127); a (N, M) and b (K, M) keep M      */
+/* contiguous (the column-major buffers above, of grad_out and of the    */
+/* input), sa (N, nblk) and sb (K, nblk). Empty groups give zeros. In    */
+/* double.                                                                */
+int oracle_mx_grouped_gemm_wgrad(const uint8_t *a, const uint8_t *sa, const uint8_t *b, const uint8_t *sb,
+                                 int64_t N, int64_t K, int64_t M, const int32_t *offs, int32_t groups, double *out)
+{
+    int64_t start = 0, base = 0, nblk;
+    if (N < 0 || K < 0 || M < 0 || groups <= 0)
+        return ORACLE_ERR_ARG;
+    if (!offsets_valid(offs, groups, M))
+        return ORACLE_ERR_OFFSETS;
+    nblk = oracle_mx_jagged_blocks(offs, groups);
+    for (int32_t g = 0; g < groups; ++g) {
+        const int64_t end = offs[g];
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t k = 0; k < K; ++k) {
+                double acc = 0.0;
+                for (int64_t m = start; m < end; ++m) {
+                    const int64_t j = base + (m - start) / 32;
+                    acc += oracle_e4m3_value(a[n * M + m]) * e8m0_value(sa[n * nblk + j]) *
+                           (oracle_e4m3_value(b[k * M + m]) * e8m0_value(sb[k * nblk + j]));
+                }
+                out[((int64_t)g * N + n) * K + k] = acc;
+            }
+        base += (end - start + 31) / 32;
+        start = end;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Weight-gradient grouped GEMM, the backward consumer of the jagged    */
 /* ops (#2064 Summary: the per-group scaled operands of the grad_weight */
 /* grouped GEMM). The contraction runs over each group's own positions: */

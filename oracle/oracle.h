@@ -49,6 +49,12 @@ int oracle_fp8_grouped_gemm_rowwise(const uint8_t *a, const float *inv_a, const 
                                     double *out);
 int oracle_mx_grouped_gemm(const uint8_t *a, const uint8_t *sa, const uint8_t *w, const uint8_t *sw,
                            int64_t M, int64_t N, int64_t K, const int32_t *offs, int32_t groups, double *out);
+int64_t oracle_mx_jagged_blocks(const int32_t *offs, int32_t groups);
+int oracle_mx_quant_jagged_colwise(const uint16_t *in, int64_t rows, int64_t cols, int64_t stride_row,
+                                   int64_t stride_col, const int32_t *offs, int32_t groups, int mode, uint8_t *out,
+                                   uint8_t *scales);
+int oracle_mx_grouped_gemm_wgrad(const uint8_t *a, const uint8_t *sa, const uint8_t *b, const uint8_t *sb,
+                                 int64_t N, int64_t K, int64_t M, const int32_t *offs, int32_t groups, double *out);
 int oracle_fp8_grouped_gemm_wgrad(const uint8_t *a, const float *inv_a, const uint8_t *b, const float *inv_b,
                                   int64_t N, int64_t K, int64_t M, const int32_t *offs, int32_t groups,
                                   double *out);

@@ -746,3 +746,84 @@ def test_mx_pipeline_approximates_the_exact_product(oracle):
     A, W = a.double().numpy(), w.double().numpy().reshape(E, N, K)
     want = np.concatenate([A[:40] @ W[0].T, A[40:] @ W[1].T])
     assert np.linalg.norm(got - want) <= 0.06 * np.linalg.norm(want)
+
+
+# ---------------------------------------------------------------- MX along the grouped dimension (R19)
+
+def _bf16_words(x):
+    return x.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def test_mx_jagged_colwise_is_rowwise_on_each_zero_padded_group(oracle):
+    """Each group's rows, transposed and padded with zeros to a multiple of
+    32, quantized by the MX rowwise routine give the same codes and scales:
+    blocks start at the group's first row, the last one holds the remainder
+    (zeros do not change an amax)."""
+    x = synth.row_scaled_normal_bf16(200, 12, seed=71)
+    offs = [0, 37, 37, 64, 190]   # an empty first group, unaligned ends, rows 190.. in no group
+    for mode in (oracle.FLOOR, oracle.RCEIL):
+        q, sc = oracle.mx_quant_jagged_colwise(_bf16_words(x).reshape(-1), 200, 12, 12, 1, offs, mode)
+        assert sc.shape == (12, oracle.mx_jagged_blocks(offs))
+        start, base = 0, 0
+        for end in offs:
+            size = end - start
+            if size:
+                nb = (size + 31) // 32
+                pad = torch.zeros((12, 32 * nb), dtype=torch.bfloat16)
+                pad[:, :size] = x[start:end].t()
+                rq, rs = oracle.mx_quant_rowwise(pad, mode)
+                assert np.array_equal(q[:, start:end], rq[:, :size])
+                assert np.array_equal(sc[:, base:base + nb], rs)
+                base += nb
+            start = end
+        assert not q[:, 190:].any()
+
+
+def test_mx_jagged_colwise_hand_example(oracle):
+    """One column, one group of 40 rows: block 0 = rows 0-31 (1.0 and one
+    448: floor byte 127, codes 0x38 and 0x7E), block 1 = rows 32-39 (all 3.0:
+    floor(log2 3) - 8 = -7, byte 120, 3 / 2^-7 = 384 = code 0x7C)."""
+    col = torch.ones(40, dtype=torch.bfloat16)
+    col[5] = 448.0
+    col[32:] = 3.0
+    q, sc = oracle.mx_quant_jagged_colwise(_bf16_words(col).reshape(-1), 40, 1, 1, 1, [40], oracle.FLOOR)
+    assert list(sc[0]) == [127, 120]
+    assert q[0, 0] == 0x38 and q[0, 5] == 0x7E and all(q[0, 32:] == 0x7C)
+
+
+def test_mx_wgrad_unit_scales_equal_the_fp8_wgrad(oracle):
+    """With every scale byte 127 the MX weight-gradient product is the FP8
+    weight-gradient GEMM with unit inverse scales (groups, empty groups and
+    the contraction over each group's own columns pinned through it)."""
+    rng = np.random.default_rng(23)
+    N, K, M = 20, 12, 90
+    a = rng.integers(0, 256, size=(N, M), dtype=np.uint8)
+    b = rng.integers(0, 256, size=(K, M), dtype=np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0
+    b[(b & 0x7F) == 0x7F] = 0
+    offs = np.array([17, 17, 60, 85], dtype=np.int32)
+    nblk = oracle.mx_jagged_blocks(offs)
+    got = oracle.mx_grouped_gemm_wgrad(a, np.full((N, nblk), 127, np.uint8), b, np.full((K, nblk), 127, np.uint8),
+                                       offs)
+    ref = oracle.fp8_grouped_gemm_wgrad(a, np.ones((4, N), np.float32), b, np.ones((4, K), np.float32), offs)
+    assert np.array_equal(got, ref)
+
+
+def test_mx_wgrad_pipeline_approximates_the_exact_product(oracle):
+    """MX quantization of dY and A along the tokens (per-group blocks) and
+    the MX weight-gradient product approximate the exact dY_g^T A_g within
+    the e4m3 rounding; a block indexed from the global row instead of the
+    group's first row, or a transposed operand, is off by far more."""
+    M, N, K = 200, 24, 16
+    dy = synth.row_scaled_normal_bf16(M, N, seed=81, lo=-3.0, hi=1.0)
+    a = synth.row_scaled_normal_bf16(M, K, seed=82)
+    offs = [45, 45, 130, 200]
+    qd, sd = oracle.mx_quant_jagged_colwise(_bf16_words(dy).reshape(-1), M, N, N, 1, offs, oracle.FLOOR)
+    qa, sa = oracle.mx_quant_jagged_colwise(_bf16_words(a).reshape(-1), M, K, K, 1, offs, oracle.FLOOR)
+    got = oracle.mx_grouped_gemm_wgrad(qd, sd, qa, sa, offs)
+    D, A = dy.double().numpy(), a.double().numpy()
+    start = 0
+    for g, end in enumerate(offs):
+        want = D[start:end].T @ A[start:end]
+        assert np.linalg.norm(got[g] - want) <= 0.08 * max(np.linalg.norm(want), 1e-300)
+        start = end
