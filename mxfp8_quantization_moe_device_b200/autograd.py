@@ -26,9 +26,10 @@ along N by the MX 3-D colwise op, whose per-expert column-major output is
 W_e^T), the scales in the 128x4 blocked layout, through the block-scaled
 grouped GEMM; the weight gradient takes the FP8 jagged path above.
 
-Nothing here computes on the host or through torch kernels besides output
-allocation: quantization and GEMMs are the library's CUDA kernels, so a
-missing library raises instead of falling back.
+Nothing here computes on the host: quantization and GEMMs are the library's
+CUDA kernels (torch only allocates and zero-fills outputs, and makes an
+incoming gradient contiguous bf16), so a missing library raises instead of
+falling back.
 """
 import torch
 
