@@ -97,6 +97,29 @@ def kernel_source_hash(kernel):
     return h.hexdigest()[:16]
 
 
+def load_traffic_capture(kernel):
+    """The capture behind load_traffic(kernel), unscaled: its workload, its
+    measured DRAM bytes and that workload's algorithmic bytes (None when the
+    capture predates the kernel's current sources)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        parts = []
+        for k in kernel.split("+"):
+            e = d["kernels"][k]
+            if e.get("source_hash") != kernel_source_hash(k):
+                return None
+            parts.append(e)
+        dram = sum(e["capture_dram_bytes"] for e in parts)
+        alg = sum(e["capture_algorithmic_bytes"] for e in parts[-1:])
+        return {"workload": parts[-1]["capture_workload"], "dram_bytes": dram, "algorithmic_bytes": alg,
+                "dram_over_algorithmic": round(dram / alg, 4), "scaled_by": parts[-1]["scaled_by"],
+                "summary": parts[-1]["captured_on"]}
+    except Exception:
+        return None
+
+
 def load_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the kernel's current sources (else None)."""
@@ -375,15 +398,27 @@ def flush_l2(torch, buf):
     buf.zero_()
 
 
+def flush_l2_clean(torch, buf, sink):
+    """Write `buf` (larger than L2), then read it back: L2 ends holding clean
+    lines of `buf` only, so the next kernel starts cold without first having
+    to write back the flush's own dirty lines."""
+    buf.zero_()
+    torch.sum(buf.view(torch.int32), dtype=torch.int64, out=sink)
+
+
 def per_shape_sweep(wl, reps):
     """us/call and GB/s per config shape after 5 warm-up calls: the median of
-    `reps` calls with the L2 flushed (256 MB write) before each, the median of
-    `reps` back-to-back calls with a hot L2 ("us_hot", labelled as such), and
-    the median host time to enqueue one call ("enqueue_us")."""
+    `reps` calls with the L2 flushed (256 MB write) before each ("us"); the
+    median of `reps` calls after the same write followed by a read of the
+    flush buffer, so that the L2 is cold but holds no dirty lines the call
+    would first have to write back ("us_clean"); the median of `reps`
+    back-to-back calls with a hot L2 ("us_hot", labelled as such); and the
+    median host time to enqueue one call ("enqueue_us")."""
     torch, mxq = wl.torch, wl.mxq
     from mxfp8_quantization_moe_device_b200 import synth
     dev = wl.dev
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
     peak, _ = load_peaks()
     rows = []
 
@@ -391,11 +426,13 @@ def per_shape_sweep(wl, reps):
         for _ in range(5):
             fn()
         torch.cuda.synchronize()
-        ts, hot, enq = [], [], []
-        for cold in (True, False):
+        ts, clean, hot, enq = [], [], [], []
+        for mode in ("cold", "clean", "hot"):
             for _ in range(reps):
-                if cold:
+                if mode == "cold":
                     flush_l2(torch, flush)
+                elif mode == "clean":
+                    flush_l2_clean(torch, flush, sink)
                 else:
                     # keep the GPU busy (~100 us, no memory traffic) while the
                     # host enqueues, so that the events time the call alone
@@ -408,12 +445,14 @@ def per_shape_sweep(wl, reps):
                 h1 = time.perf_counter()
                 b.record()
                 b.synchronize()
-                (ts if cold else hot).append(a.elapsed_time(b) * 1e3)
+                {"cold": ts, "clean": clean, "hot": hot}[mode].append(a.elapsed_time(b) * 1e3)
                 enq.append((h1 - h0) * 1e6)
         us = statistics.median(ts)
         gbs = nbytes / (us * 1e-6) / 1e9
+        usc = statistics.median(clean)
         rows.append({"op": name, "shape": shape, "us": round(us, 3), "GB/s": round(gbs, 1),
                      "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4),
+                     "us_clean": round(usc, 3), "frac_measured_clean": round(nbytes / (usc * 1e-6) / 1e9 / peak, 4),
                      "us_hot": round(statistics.median(hot), 3), "enqueue_us": round(statistics.median(enq), 1)})
 
     # tiny jagged
@@ -635,6 +674,24 @@ def oracle_samples(wl):
     ]
 
 
+def host_description():
+    """The host the oracle runs on: core count and CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count()
+    return {"nproc": usable, "cpu_count": os.cpu_count(), "cpu_model": model}
+
+
 def run_oracle_samples(samples):
     """Time each sample once; estimate the oracle's time for the full step
     from each op's per-byte rate. Returns (GB/s, seconds spent, per-op)."""
@@ -825,7 +882,8 @@ def main():
     achieved = per_op[dom]["GB/s"]
     roofline = {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "op": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                "algorithmic_bytes_per_launch": dom_bytes, "traffic": load_traffic(KERNEL_NAMES[dom])}
+                "algorithmic_bytes_per_launch": dom_bytes, "traffic": load_traffic(KERNEL_NAMES[dom]),
+                "traffic_capture": load_traffic_capture(KERNEL_NAMES[dom])}
 
     out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -847,7 +905,8 @@ def main():
         samples = oracle_samples(wl)
         gbs, spent, per_o = run_oracle_samples(samples)
         out["cpu_baseline"] = {"value": round(gbs, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                               "sample": SAMPLE_DESC, "seconds": round(spent, 2), "per_op_GB/s": per_o}
+                               "sample": SAMPLE_DESC, "seconds": round(spent, 2), "per_op_GB/s": per_o,
+                               "extrapolated_from_sample": True, "host": host_description()}
     if not args.no_e2e:
         ms, bi, bo, ok = run_e2e(wl, max(1, args.e2e_steps))
         ms = max_over_ranks(ms, dev, world)
@@ -886,13 +945,18 @@ def main_reference(args, world, rank):
         times.append(spent)
     value = statistics.median(vals)
     total = sum(fb for _, _, _, fb in samples)
+    # the oracle runs a bounded slice per step; ms_per_step is the full
+    # step's bytes at the rate measured on that slice (flagged as such), and
+    # sample_ms_per_step is the slice's own measured time
     out = {"metric": METRIC, "impl": "reference", "value": round(value, 5), "unit": "GB/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / (value * 1e9) * 1e3, 1),
+           "extrapolated_from_sample": True, "sample_ms_per_step": round(statistics.median(times) * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3 (fp32 scale math)",
            "data": "synthetic (seeded)",
            "config": {"workload": WORKLOAD, "step_bytes": total, "parallelism": "single-threaded CPU oracle"},
            "cpu_baseline": {"value": round(value, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                            "sample": REF_SAMPLE_DESC},
+                            "sample": REF_SAMPLE_DESC, "extrapolated_from_sample": True,
+                            "host": host_description()},
            "e2e": {"value": round(value, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
            "wall_s": round(time.perf_counter() - t0, 1)}
     print(json.dumps(out))

@@ -342,11 +342,16 @@ int mx_quant_rowwise_blocked_grouped(const void *in, int64_t rows, int64_t cols,
  * fp8_quant_jagged_colwise, without the workspace: the scratch is a fixed
  * array of fp8_quant_jagged_colwise_noalloc_max_scratch_bytes() bytes
  * (1 MiB) inside the library, held by every GPU that loads it until exit.
- *   - A problem whose workspace would exceed that size (see
- *     fp8_quant_jagged_workspace_bytes with is_colwise = 1) returns
- *     MXQ_ERR_WORKSPACE and launches nothing.
- *   - The first call on a device looks up the array's device address with
- *     that device current; make it before any stream capture.
+ *   - The scratch this call needs is decided by the kernels it picks for
+ *     these very arguments: the kernels that keep a per-(group, column)
+ *     amax table use G * cols * 4 bytes of it (rounded up to 256), the
+ *     single-kernel path of small or strided problems none. A call that
+ *     would need more than the array holds returns MXQ_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - `stream` must belong to the current device (MXQ_ERR_UNSUPPORTED
+ *     otherwise). The first call on a device that needs scratch looks up
+ *     the array's device address with that device current; make it before
+ *     any stream capture.
  *   - The call allocates nothing. All calls on a device share the array
  *     (each clears what it uses first), so calls that overlap on the GPU
  *     race; serialize them.

@@ -83,6 +83,13 @@ def _check(fn, rc):
         raise MXQError(fn, rc)
 
 
+def _call(name, dev, *args):
+    """One library call with `dev` current (the kernels launch on the current
+    device) on that device's current torch stream; raises on a non-OK status."""
+    with torch.cuda.device(dev):
+        _check(name, getattr(lib(), name)(*args, _stream(dev)))
+
+
 def _cuda(t, name):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
@@ -103,6 +110,18 @@ def _mode(mode):
     if mode in (RCEIL, "rceil"):
         return RCEIL
     raise ValueError(f"unknown scale mode {mode!r}")
+
+
+def _out_buffer(t, name, shape, esize, dev, dtype=None):
+    """A caller-provided output: the library writes it through its data
+    pointer with the op's own layout, so shape, element size, contiguity and
+    device are checked here, before any write can go astray."""
+    _cuda(t, name)
+    if (tuple(t.shape) != tuple(shape) or t.element_size() != esize or not t.is_contiguous()
+            or t.device != dev or (dtype is not None and t.dtype != dtype)):
+        want = f"{dtype}" if dtype is not None else f"{esize}-byte"
+        raise TypeError(f"{name} must be a contiguous {want} tensor of shape {tuple(shape)} on {dev}")
+    return t
 
 
 def _offsets(offs, dev):
@@ -127,17 +146,20 @@ def _jagged(name, x, offs, colwise, out, inv_scales, workspace):
     rows, cols = x.shape
     sr, sc = x.stride()
     G = offs.numel()
+    oshape = (cols, rows) if colwise else (rows, cols)
+    ishape = (G, cols if colwise else rows)
     if out is None:
-        out = torch.empty((cols, rows) if colwise else (rows, cols), dtype=torch.uint8, device=dev)
+        out = torch.empty(oshape, dtype=torch.uint8, device=dev)
     if inv_scales is None:
-        inv_scales = torch.empty((G, cols if colwise else rows), dtype=torch.float32, device=dev)
+        inv_scales = torch.empty(ishape, dtype=torch.float32, device=dev)
+    _out_buffer(out, "out", oshape, 1, dev)
+    _out_buffer(inv_scales, "inv_scales", ishape, 4, dev, torch.float32)
     need = jagged_workspace_bytes(rows, cols, sr, sc, G, colwise)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     # the library reads x through its data pointer and element strides
-    rc = getattr(lib(), name)(_ptr(x), rows, cols, sr, sc, _ptr(offs), G, _ptr(out), _ptr(inv_scales),
-                              _ptr(workspace), workspace.numel() if workspace is not None else 0, _stream(dev))
-    _check(name, rc)
+    _call(name, dev, _ptr(x), rows, cols, sr, sc, _ptr(offs), G, _ptr(out), _ptr(inv_scales),
+          _ptr(workspace), workspace.numel() if workspace is not None else 0)
     q = out.view(torch.float8_e4m3fn)
     return (q.t() if colwise else q), inv_scales
 
@@ -167,9 +189,10 @@ def fp8_quant_jagged_colwise_noalloc(x, offs, *, out, inv_scales):
     _offsets(offs, dev)
     rows, cols = x.shape
     sr, sc = x.stride()
-    rc = lib().fp8_quant_jagged_colwise_noalloc(_ptr(x), rows, cols, sr, sc, _ptr(offs), offs.numel(), _ptr(out),
-                                                _ptr(inv_scales), _stream(dev))
-    _check("fp8_quant_jagged_colwise_noalloc", rc)
+    _out_buffer(out, "out", (cols, rows), 1, dev)
+    _out_buffer(inv_scales, "inv_scales", (offs.numel(), cols), 4, dev, torch.float32)
+    _call("fp8_quant_jagged_colwise_noalloc", dev, _ptr(x), rows, cols, sr, sc, _ptr(offs), offs.numel(), _ptr(out),
+          _ptr(inv_scales))
     return out.view(torch.float8_e4m3fn).t(), inv_scales
 
 
@@ -186,9 +209,7 @@ def fp8_quant_blockwise(x, block_rows=1, block_cols=128, *, out=None, inv_scales
         out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     if inv_scales is None:
         inv_scales = torch.empty((rows // block_rows, cols // block_cols), dtype=torch.float32, device=x.device)
-    rc = lib().fp8_quant_blockwise(_ptr(x), rows, cols, block_rows, block_cols, _ptr(out), _ptr(inv_scales),
-                                   _stream(x.device))
-    _check("fp8_quant_blockwise", rc)
+    _call("fp8_quant_blockwise", x.device, _ptr(x), rows, cols, block_rows, block_cols, _ptr(out), _ptr(inv_scales))
     return out.view(torch.float8_e4m3fn), inv_scales
 
 
@@ -206,9 +227,7 @@ def fp8_quant_blockwise_transposed(x, block_cols=1, *, out=None, inv_scales=None
         out = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
     if inv_scales is None:
         inv_scales = torch.empty((cols // block_cols, rows // 128), dtype=torch.float32, device=x.device)
-    rc = lib().fp8_quant_blockwise_transposed(_ptr(x), rows, cols, 128, block_cols, _ptr(out), _ptr(inv_scales),
-                                              _stream(x.device))
-    _check("fp8_quant_blockwise_transposed", rc)
+    _call("fp8_quant_blockwise_transposed", x.device, _ptr(x), rows, cols, 128, block_cols, _ptr(out), _ptr(inv_scales))
     return out.view(torch.float8_e4m3fn), inv_scales
 
 
@@ -223,8 +242,7 @@ def mx_quant_3d_colwise(w, mode="floor", *, out=None, scales=None):
         out = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
     if scales is None:
         scales = torch.empty((E, K, N // 32), dtype=torch.uint8, device=w.device)
-    rc = lib().mx_quant_3d_colwise(_ptr(w), E, N, K, _mode(mode), _ptr(out), _ptr(scales), _stream(w.device))
-    _check("mx_quant_3d_colwise", rc)
+    _call("mx_quant_3d_colwise", w.device, _ptr(w), E, N, K, _mode(mode), _ptr(out), _ptr(scales))
     return out.view(torch.float8_e4m3fn).transpose(1, 2), scales
 
 
@@ -239,8 +257,7 @@ def mx_quant_rowwise(x, mode="floor", *, out=None, scales=None):
         out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
-    rc = lib().mx_quant_rowwise(_ptr(x), rows, cols, _mode(mode), _ptr(out), _ptr(scales), _stream(x.device))
-    _check("mx_quant_rowwise", rc)
+    _call("mx_quant_rowwise", x.device, _ptr(x), rows, cols, _mode(mode), _ptr(out), _ptr(scales))
     return out.view(torch.float8_e4m3fn), scales
 
 
@@ -267,9 +284,8 @@ def mx_scales_to_blocked_grouped(scales, offs, *, capacity_rows=None, out=None, 
         out = torch.empty(capacity_rows * cols4, dtype=torch.uint8, device=dev)
     if group_row_starts is None and with_starts:
         group_row_starts = torch.empty(G, dtype=torch.int32, device=dev)
-    rc = lib().mx_scales_to_blocked_grouped(_ptr(scales), rows, cols, _ptr(offs), G, _ptr(out), capacity_rows,
-                                            _ptr(group_row_starts), _stream(dev))
-    _check("mx_scales_to_blocked_grouped", rc)
+    _call("mx_scales_to_blocked_grouped", dev, _ptr(scales), rows, cols, _ptr(offs), G, _ptr(out), capacity_rows,
+          _ptr(group_row_starts))
     return out, group_row_starts
 
 
@@ -296,9 +312,8 @@ def mx_scales_to_blocked_grouped_k(scales, offs, *, capacity_cols=None, out=None
         out = torch.empty(rows_p * capacity_cols, dtype=torch.uint8, device=dev)
     if group_col_starts is None and with_starts:
         group_col_starts = torch.empty(G, dtype=torch.int32, device=dev)
-    rc = lib().mx_scales_to_blocked_grouped_k(_ptr(scales), rows, cols, _ptr(offs), G, _ptr(out), capacity_cols,
-                                              _ptr(group_col_starts), _stream(dev))
-    _check("mx_scales_to_blocked_grouped_k", rc)
+    _call("mx_scales_to_blocked_grouped_k", dev, _ptr(scales), rows, cols, _ptr(offs), G, _ptr(out), capacity_cols,
+          _ptr(group_col_starts))
     return out, group_col_starts
 
 
@@ -323,9 +338,8 @@ def mx_quant_rowwise_blocked_grouped(x, offs, mode="floor", *, capacity_rows=Non
         scales = torch.empty(capacity_rows * ((cols + 127) // 128) * 4, dtype=torch.uint8, device=dev)
     if group_row_starts is None and with_starts:
         group_row_starts = torch.empty(G, dtype=torch.int32, device=dev)
-    rc = lib().mx_quant_rowwise_blocked_grouped(_ptr(x), rows, cols, _mode(mode), _ptr(offs), G, _ptr(out),
-                                                _ptr(scales), capacity_rows, _ptr(group_row_starts), _stream(dev))
-    _check("mx_quant_rowwise_blocked_grouped", rc)
+    _call("mx_quant_rowwise_blocked_grouped", dev, _ptr(x), rows, cols, _mode(mode), _ptr(offs), G, _ptr(out),
+          _ptr(scales), capacity_rows, _ptr(group_row_starts))
     return out.view(torch.float8_e4m3fn), scales, group_row_starts
 
 
@@ -352,9 +366,8 @@ def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, *, out=None):
         raise TypeError("shape mismatch between a, w, inv_a, inv_w and offs")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    rc = lib().fp8_grouped_gemm_rowwise(_ptr(a), _ptr(inv_a), _ptr(w), _ptr(inv_w), M, N, K, _ptr(offs), E,
-                                        _ptr(out), _stream(dev))
-    _check("fp8_grouped_gemm_rowwise", rc)
+    _call("fp8_grouped_gemm_rowwise", dev, _ptr(a), _ptr(inv_a), _ptr(w), _ptr(inv_w), M, N, K, _ptr(offs), E,
+          _ptr(out))
     return out
 
 
@@ -385,9 +398,7 @@ def mx_grouped_gemm(a, sfa, w, sfw, offs, *, out=None):
         raise TypeError("scale buffers smaller than the blocked layout needs")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    rc = lib().mx_grouped_gemm(_ptr(a), _ptr(sfa), _ptr(w), _ptr(sfw), M, N, K, _ptr(offs), E, _ptr(out),
-                               _stream(dev))
-    _check("mx_grouped_gemm", rc)
+    _call("mx_grouped_gemm", dev, _ptr(a), _ptr(sfa), _ptr(w), _ptr(sfw), M, N, K, _ptr(offs), E, _ptr(out))
     return out
 
 
@@ -415,9 +426,7 @@ def fp8_grouped_gemm_wgrad(a, inv_a, b, inv_b, offs, *, out=None):
         raise TypeError("shape mismatch between a, b, inv_a, inv_b and offs")
     if out is None:
         out = torch.empty((G, N, K), dtype=torch.bfloat16, device=dev)
-    rc = lib().fp8_grouped_gemm_wgrad(_ptr(a), _ptr(inv_a), _ptr(b), _ptr(inv_b), N, K, M, _ptr(offs), G, _ptr(out),
-                                      _stream(dev))
-    _check("fp8_grouped_gemm_wgrad", rc)
+    _call("fp8_grouped_gemm_wgrad", dev, _ptr(a), _ptr(inv_a), _ptr(b), _ptr(inv_b), N, K, M, _ptr(offs), G, _ptr(out))
     return out
 
 

@@ -723,11 +723,15 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 void *g_noalloc_ptr[128];
 std::mutex g_noalloc_mu;
 
-int noalloc_scratch(void **out)
+int noalloc_scratch(cudaStream_t stream, void **out)
 {
-    int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 128)
+    // the array of the stream's device; the kernels launch on the current
+    // device, so the two must agree
+    int d = 0, sd = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 128 || cudaStreamGetDevice(stream, &sd) != cudaSuccess)
         return MXQ_ERR_CUDA;
+    if (sd != d)
+        return MXQ_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
     if (!g_noalloc_ptr[d]) {
         void *p = nullptr;
@@ -745,17 +749,24 @@ extern "C" int fp8_quant_jagged_colwise_noalloc(const void *in, int64_t rows, in
                                                 int64_t stride_col, const int32_t *offs, int32_t num_groups,
                                                 void *out, float *inv_scales, cudaStream_t stream)
 {
-    const size_t need = fp8_quant_jagged_workspace_bytes(rows, cols, stride_row, stride_col, num_groups, 1);
-    if (need > kNoAllocScratchBytes)
-        return MXQ_ERR_WORKSPACE;
+    if (rows < 0 || cols < 0 || num_groups < 1)
+        return MXQ_ERR_SHAPE;
+    // the plan of this very call (real pointers): only the kernels that keep
+    // a table need scratch, and only they are limited by the array's size
+    JaggedPlan pl;
+    int rc = plan_jagged(in, cols, rows, stride_col, stride_row, num_groups, out, &pl);
+    if (rc != MXQ_OK)
+        return rc;
     void *scratch = nullptr;
-    if (need > 0) {
-        const int rc = noalloc_scratch(&scratch);
+    if (pl.ws > 0) {
+        if (pl.ws > kNoAllocScratchBytes)
+            return MXQ_ERR_WORKSPACE;
+        rc = noalloc_scratch(stream, &scratch);
         if (rc != MXQ_OK)
             return rc;
     }
     return fp8_quant_jagged_colwise(in, rows, cols, stride_row, stride_col, offs, num_groups, out, inv_scales,
-                                    scratch, need > 0 ? kNoAllocScratchBytes : 0, stream);
+                                    scratch, scratch ? kNoAllocScratchBytes : 0, stream);
 }
 
 extern "C" size_t fp8_quant_jagged_colwise_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
