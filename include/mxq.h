@@ -334,6 +334,63 @@ int mx_quant_rowwise_blocked_grouped(const void *in, int64_t rows, int64_t cols,
                                      cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * mx_quant_jagged_colwise_padded / mx_quant_jagged_rowwise_padded - the
+ * left and right operands of the MXFP8 weight-gradient grouped GEMM
+ * (#3504's stack: "integrate new cuda kernel for blocked layout for groups
+ * along K"): MX quantization along the grouped dimension (the tokens).
+ *   colwise     groups are row ranges of (rows, cols); one line per column.
+ *   rowwise     groups are column ranges of (rows, cols); one line per row.
+ *   in          bf16 with element strides; lines must be contiguous
+ *               (colwise: stride_col == 1, a row-major input; rowwise:
+ *               stride_row == 1, the transposed view of a row-major
+ *               tensor), the other stride a multiple of 8 and >= the line
+ *               count, else MXQ_ERR_UNSUPPORTED. The line count must be a
+ *               multiple of 128 (MXQ_ERR_SHAPE).
+ *   mode        MXQ_E8M0_FLOOR or MXQ_E8M0_RCEIL.
+ *   Each group's positions are cut into 32-element blocks from the group's
+ *   first position (the last block holds the remainder); every block gets
+ *   an E8M0 scale over its own elements and e4m3 codes.
+ *   out         e4m3, line-major (lines, out_cols_capacity): group g's
+ *               positions start at padded position 128 * T[g], T[g] =
+ *               sum_{h<g} ceil(size_h / 128); pad positions and the capacity
+ *               past the last group are zero codes.
+ *               out_cols_capacity is a multiple of 128 and >=
+ *               mx_blocked_grouped_rows_bound(positions, num_groups).
+ *   scales_blocked  E8M0 bytes of the (lines, out_cols_capacity / 32) scale
+ *               matrix in the 128x4 blocked layout (16-byte aligned,
+ *               lines * out_cols_capacity / 32 bytes): group g's scale
+ *               columns start at 4 * T[g] (the groups-along-K layout of
+ *               mx_scales_to_blocked_grouped_k); every byte not covered by
+ *               a block is 0.
+ * ------------------------------------------------------------------------ */
+int mx_quant_jagged_colwise_padded(const void *in, int64_t rows, int64_t cols,
+                                   int64_t stride_row, int64_t stride_col,
+                                   const int32_t *offs, int32_t num_groups, int32_t mode,
+                                   void *out, int64_t out_cols_capacity, uint8_t *scales_blocked,
+                                   cudaStream_t stream);
+int mx_quant_jagged_rowwise_padded(const void *in, int64_t rows, int64_t cols,
+                                   int64_t stride_row, int64_t stride_col,
+                                   const int32_t *offs, int32_t num_groups, int32_t mode,
+                                   void *out, int64_t out_cols_capacity, uint8_t *scales_blocked,
+                                   cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * mx_grouped_gemm_wgrad - the MXFP8 weight gradient of a grouped matmul on
+ * the tensor cores: for every group g (token range [offs[g-1], offs[g])),
+ *   out[g][n][k] = sum over the group's padded positions p of
+ *                  a[n][p] 2^(sa[n][p/32] - 127) * b[k][p] 2^(sb[k][p/32] - 127)
+ * with a (N, capacity) and b (K, capacity) the padded codes and sfa, sfb the
+ * blocked scales written by mx_quant_jagged_*_padded (a from grad_out^T,
+ * rowwise; b from the input, colwise) with the same offsets and capacity.
+ * M is the token count the offsets index. N % 128 == 0, K % 128 == 0,
+ * capacity % 128 == 0 and >= mx_blocked_grouped_rows_bound(M, num_groups).
+ * out: bf16 (num_groups, N, K); empty groups give zeros.
+ * ------------------------------------------------------------------------ */
+int mx_grouped_gemm_wgrad(const void *a, const uint8_t *sfa, const void *b, const uint8_t *sfb,
+                          int64_t N, int64_t K, int64_t M, int64_t capacity,
+                          const int32_t *offs, int32_t num_groups, void *out, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * fp8_quant_jagged_colwise_noalloc - the source pages have no counterpart to
  * this entry point; it exists for callers that cannot allocate device memory
  * (a plugin inside a framework that owns all device memory and passes no
@@ -382,14 +439,17 @@ int mxq_version(void);
 /* Test hooks (host-side settings read at launch time):
  *   MXQ_TESTING_WAIT_LIMIT_NS  bound of every device-side wait, nanoseconds
  *                              (default 1e9; 0 restores the default).
- *   MXQ_TESTING_SKIP_ARRIVAL   when 1, CTA 0 of the jagged cast pass never
- *                              issues its first TMA load, so the transaction
+ *   MXQ_TESTING_SKIP_ARRIVAL   when 1, CTA 0 of the jagged cast pass (or
+ *                              of the single-read kernel) never issues its
+ *                              first TMA load, so the transaction
  *                              arrival on that ring slot never comes, the
  *                              bounded waits on it expire and report
  *                              MXQ_ERR_TIMEOUT; 0 turns it off.
  *   MXQ_TESTING_FORCE_PATH     jagged ops: 0 automatic, 1 two-pass TMA
- *                              kernels (amax, then cast), 2 generic kernel.
- *   MXQ_TESTING_GEMM_TILE_N    mx_grouped_gemm tile width: 0 automatic (256
+ *                              kernels (amax, then cast), 2 generic kernel,
+ *                              3 single-read kernel (cooperative launch).
+ *   MXQ_TESTING_GEMM_TILE_N    mx_grouped_gemm (and mx_grouped_gemm_wgrad)
+ *                              tile width: 0 automatic (256
  *                              when N % 256 == 0, else 128), 128 forced. */
 #define MXQ_TESTING_WAIT_LIMIT_NS 1
 #define MXQ_TESTING_SKIP_ARRIVAL 2

@@ -24,7 +24,10 @@ take e4m3 codes with one E8M0 scale per 32 elements along their contracted
 dimension (A and W along K by the MX rowwise op; dY along N by the same op, W
 along N by the MX 3-D colwise op, whose per-expert column-major output is
 W_e^T), the scales in the 128x4 blocked layout, through the block-scaled
-grouped GEMM; the weight gradient takes the FP8 jagged path above.
+grouped GEMM; its weight gradient quantizes dY^T and A in 32-token blocks
+that restart at every group, each group padded to 128 tokens with its scales
+in the groups-along-K blocked layout, into the block-scaled weight-gradient
+grouped GEMM.
 
 Nothing here computes on the host: quantization and GEMMs are the library's
 CUDA kernels (torch only allocates and zero-fills outputs, and makes an
@@ -140,10 +143,19 @@ def _mx_grad_input(dy, w, offs, mode):
     return mxq.mx_grouped_gemm(qdy.view(torch.uint8), sdy, wt, swt, offs, out=da)
 
 
+def _mx_grad_weight(dy, a, offs, mode):
+    M, N = dy.shape
+    # dY^T and A in MX blocks along each group's tokens, every group padded
+    # to 128 tokens, scales in the groups-along-K blocked layout
+    qdy, sdy = mxq.mx_quant_jagged_rowwise_padded(dy.t(), offs, mode)
+    qa, sa = mxq.mx_quant_jagged_colwise_padded(a, offs, mode)
+    return mxq.mx_grouped_gemm_wgrad(qdy.view(torch.uint8), sdy, qa.view(torch.uint8), sa, offs, M)
+
+
 class MXGroupedMM(torch.autograd.Function):
-    """MXFP8 forward and input gradient (one E8M0 scale per 32 elements along
-    each GEMM's contracted dimension: A and W along K, dY and W along N), FP8
-    jagged weight gradient (no MX weight-gradient GEMM is built)."""
+    """MXFP8 forward, input gradient and weight gradient: one E8M0 scale per
+    32 elements along each GEMM's contracted dimension (A and W along K, dY
+    and W along N, dY and A along each group's tokens)."""
 
     @staticmethod
     def forward(ctx, a, w, offs, mode):
@@ -157,15 +169,15 @@ class MXGroupedMM(torch.autograd.Function):
         a, w, offs = ctx.saved_tensors
         dy = dy.to(torch.bfloat16).contiguous()
         da = _mx_grad_input(dy, w, offs, ctx.mode) if ctx.needs_input_grad[0] else None
-        dw = _grad_weight(dy, a, offs) if ctx.needs_input_grad[1] else None
+        dw = _mx_grad_weight(dy, a, offs, ctx.mode) if ctx.needs_input_grad[1] else None
         return da, dw, None, None
 
 
 def mx_grouped_mm(a, w, offs, mode="floor"):
     """out (M, N) bf16 = the MXFP8 grouped product of a (M, K) bf16 tokens
     sorted by expert and w (E, N, K) bf16 expert weights (E8M0 scales by the
-    floor or rceil rule); differentiable in a (MXFP8 input gradient) and w
-    (FP8 jagged weight gradient)."""
+    floor or rceil rule); differentiable in a and w, both gradients in
+    MXFP8."""
     return MXGroupedMM.apply(a, w, offs, mode)
 
 

@@ -47,6 +47,11 @@ SIGNATURES = {
     "mx_blocked_grouped_k_cols_bound": (_i64, [_i64, _i32]),
     "mx_quant_rowwise_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _i64, _vp,
                                                         _vp]),
+    "mx_quant_jagged_colwise_padded": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _i64,
+                                                      _vp, _vp]),
+    "mx_quant_jagged_rowwise_padded": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _i64,
+                                                      _vp, _vp]),
+    "mx_grouped_gemm_wgrad": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "mxq_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(_i32)]),
     "mxq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mxq_version": (ctypes.c_int, []),
@@ -343,6 +348,45 @@ def mx_quant_rowwise_blocked_grouped(x, offs, mode="floor", *, capacity_rows=Non
     return out.view(torch.float8_e4m3fn), scales, group_row_starts
 
 
+def _mx_jagged_padded(name, x, offs, mode, colwise, capacity, out, scales):
+    _cuda(x, "x")
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    dev = x.device
+    _offsets(offs, dev)
+    rows, cols = x.shape
+    sr, sc = x.stride()
+    G = offs.numel()
+    lines, positions = (cols, rows) if colwise else (rows, cols)
+    if capacity is None:
+        capacity = blocked_grouped_rows_bound(positions, G)
+    if out is None:
+        out = torch.empty((lines, capacity), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(lines * capacity // 32, dtype=torch.uint8, device=dev)
+    _out_buffer(out, "out", (lines, capacity), 1, dev)
+    _out_buffer(scales, "scales", (lines * capacity // 32,), 1, dev)
+    _call(name, dev, _ptr(x), rows, cols, sr, sc, _ptr(offs), G, _mode(mode), _ptr(out), capacity, _ptr(scales))
+    return out.view(torch.float8_e4m3fn), scales
+
+
+def mx_quant_jagged_colwise_padded(x, offs, mode="floor", *, capacity=None, out=None, scales=None):
+    """MXFP8 quantization of x (rows, cols) along its rows, in 32-row blocks
+    that restart at every group (groups = row ranges). Returns (q (cols,
+    capacity) e4m3, each group's rows at its 128-padded position, zeros
+    elsewhere; flat blocked E8M0 scales of the (cols, capacity/32) matrix,
+    groups along its columns)."""
+    return _mx_jagged_padded("mx_quant_jagged_colwise_padded", x, offs, mode, True, capacity, out, scales)
+
+
+def mx_quant_jagged_rowwise_padded(x, offs, mode="floor", *, capacity=None, out=None, scales=None):
+    """MXFP8 quantization of x (rows, cols) along its columns in 32-column
+    blocks that restart at every group (groups = column ranges); x is
+    typically the transposed view of a row-major tensor. Returns (q (rows,
+    capacity), flat blocked scales of the (rows, capacity/32) matrix)."""
+    return _mx_jagged_padded("mx_quant_jagged_rowwise_padded", x, offs, mode, False, capacity, out, scales)
+
+
 # ---------------------------------------------------------------- GEMM
 
 def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, *, out=None):
@@ -427,6 +471,37 @@ def fp8_grouped_gemm_wgrad(a, inv_a, b, inv_b, offs, *, out=None):
     if out is None:
         out = torch.empty((G, N, K), dtype=torch.bfloat16, device=dev)
     _call("fp8_grouped_gemm_wgrad", dev, _ptr(a), _ptr(inv_a), _ptr(b), _ptr(inv_b), N, K, M, _ptr(offs), G, _ptr(out))
+    return out
+
+
+def mx_grouped_gemm_wgrad(a, sfa, b, sfb, offs, tokens, *, out=None):
+    """MXFP8 weight-gradient grouped GEMM on the tensor cores: out[g][n][k] =
+    sum over group g's padded positions of a[n][p] 2^(sa-127) * b[k][p]
+    2^(sb-127). a (N, capacity) and b (K, capacity) e4m3 with their flat
+    blocked scales sfa, sfb, as mx_quant_jagged_rowwise_padded (grad_out^T)
+    and mx_quant_jagged_colwise_padded (input) return them for the same
+    offsets; offs (G,) int32 group ends over `tokens` tokens. Returns out
+    (G, N, K) bf16."""
+    for t, n in ((a, "a"), (sfa, "sfa"), (b, "b"), (sfb, "sfb")):
+        _cuda(t, n)
+        if not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous")
+    if a.element_size() != 1 or b.element_size() != 1 or a.dim() != 2 or b.dim() != 2:
+        raise TypeError("a must be (N, capacity) and b (K, capacity), one byte per element (e4m3)")
+    if sfa.element_size() != 1 or sfb.element_size() != 1:
+        raise TypeError("sfa and sfb must be byte (E8M0) tensors")
+    dev = a.device
+    _offsets(offs, dev)
+    N, cap = a.shape
+    K, cap2 = b.shape
+    G = offs.numel()
+    if cap2 != cap or sfa.numel() < N * cap // 32 or sfb.numel() < K * cap // 32:
+        raise TypeError("shape mismatch between a, b and their scales")
+    if out is None:
+        out = torch.empty((G, N, K), dtype=torch.bfloat16, device=dev)
+    _out_buffer(out, "out", (G, N, K), 2, dev, torch.bfloat16)
+    _call("mx_grouped_gemm_wgrad", dev, _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), N, K, int(tokens), cap, _ptr(offs),
+          G, _ptr(out))
     return out
 
 

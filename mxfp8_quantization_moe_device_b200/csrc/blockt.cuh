@@ -195,8 +195,7 @@ __global__ void __launch_bounds__(bt::THREADS, bt::CTAS_PER_SM)
             }
         }
         fence_proxy_async_smem();
-        named_barrier(1, CWARPS * 32);
-        if (sm.abort_flag)
+        if (barrier_or(1, CWARPS * 32, sm.abort_flag != 0))
             break;
         if (threadIdx.x == 0) {
             tma_store_2d(&tm_out, sm.out[ob][0], (int)(rt * TR), (int)(ct * 2 * TH));

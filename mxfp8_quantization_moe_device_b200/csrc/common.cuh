@@ -144,6 +144,22 @@ MXQ_DEV void named_barrier(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Named barrier over `n` threads that also ORs `pred` across them: every
+// participant gets the same answer, so a stop decision taken at it is
+// uniform and no thread is left waiting at a later barrier.
+MXQ_DEV bool barrier_or(int id, int n, bool pred)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.or.pred q, %2, %3, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"((uint32_t)pred), "r"(id), "r"(n)
+                 : "memory");
+    return r != 0;
+}
+
 // ---------------------------------------------------------------- memory
 MXQ_DEV uint4 ld_stream_v4(const void *p)
 {

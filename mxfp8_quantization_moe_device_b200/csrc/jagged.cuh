@@ -530,8 +530,7 @@ __global__ void __launch_bounds__(jag::cst::THREADS, jag::cst::CTAS_PER_SM)
                 }
             }
         }
-        named_barrier(1, CWARPS * 32);
-        if (sm.abort_flag)
+        if (barrier_or(1, CWARPS * 32, sm.abort_flag != 0))
             break;
         if (threadIdx.x == 0 && full_tile) {
             tma_store_2d(&tm_out, sm.out[ob], (int)(pt * TP), (int)(lt * TL));

@@ -157,8 +157,7 @@ __global__ void __launch_bounds__(THREADS, CTAS_PER_SM)
         sm.sc[ob][2 * lane][w] = (uint8_t)b0;
         sm.sc[ob][2 * lane + 1][w] = (uint8_t)b1;
         fence_proxy_async_smem();
-        named_barrier(1, CWARPS * 32);
-        if (sm.abort_flag)
+        if (barrier_or(1, CWARPS * 32, sm.abort_flag != 0))
             break;
 
         if (threadIdx.x == 0) {

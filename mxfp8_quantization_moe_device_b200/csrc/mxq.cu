@@ -10,9 +10,11 @@
 #include "blockt.cuh"
 #include "mx3d.cuh"
 #include "jagged.cuh"
+#include "jagged1.cuh"
 #include "blocked.cuh"
 #include "gemm.cuh"
 #include "gemm_mx.cuh"
+#include "mxj.cuh"
 
 using namespace mxq;
 
@@ -76,9 +78,11 @@ struct DevInfo {
     int coop = 0;
     int amx_per_sm = 0;   // resident CTAs of the jagged amax pass
     int cst_per_sm = 0;   // resident CTAs of the jagged cast pass
+    int sg_per_sm = 0;    // resident CTAs of the single-read jagged kernel
     int rb_per_sm = 0;    // resident CTAs of the 1x128 kernel
     int mx32_per_sm = 0;  // resident CTAs of the 1x32 kernel
     int mxb_per_sm = 0;   // resident CTAs of the 1x32 kernel with blocked scales
+    int mxj_per_sm = 0;   // resident CTAs of the padded MX jagged kernel (at MAX_G groups)
 };
 
 DevInfo g_dev[128];
@@ -113,15 +117,27 @@ int device_info(const DevInfo **out)
             cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::smem_fixed<256>()) != cudaSuccess ||
             cudaFuncSetAttribute(k_jagged_cast, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)jag::cst::SMEM_BYTES) != cudaSuccess)
+                                 (int)jag::cst::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(k_jagged_single, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)jg1::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mx_jagged_colwise_padded, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(mxj::SMEM_FIXED + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mx_grouped_gemm_wgrad<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gmx::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_mx_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(gmx::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess)
             return MXQ_ERR_CUDA;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.amx_per_sm, k_jagged_amax, jag::amx::THREADS, 0) !=
                 cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.cst_per_sm, k_jagged_cast, jag::cst::THREADS,
                                                           jag::cst::SMEM_BYTES) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.sg_per_sm, k_jagged_single, jg1::THREADS,
+                                                          jg1::SMEM_BYTES) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.rb_per_sm, k_fp8_1x128, RB_THREADS, 0) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mx32_per_sm, k_mx_1x32, RB_THREADS, 0) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mxb_per_sm, k_mx_1x32_blocked, 256, 0) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mxb_per_sm, k_mx_1x32_blocked, 256, 0) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.mxj_per_sm, k_mx_jagged_colwise_padded, mxj::THREADS,
+                                                          mxj::SMEM_FIXED + blk::MAX_G * sizeof(int)) != cudaSuccess)
             return MXQ_ERR_CUDA;
         di.ready = true;
     }
@@ -157,9 +173,11 @@ int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_
 
 // ------------------------------------------------------------ jagged plan
 struct JaggedPlan {
-    bool twopass = false;
+    bool twopass = false;     // k_jagged_amax + k_jagged_cast
+    bool single = false;      // k_jagged_single
     int wpc = 0;              // amax pass: warps per 256-line chunk
     int grid_a = 0, grid_c = 0;
+    int grid_s = 0;           // single-read kernel: grid (all resident)
     size_t ws = 0;
 };
 
@@ -175,7 +193,18 @@ bool twopass_layout_ok(const void *in, int64_t L, int64_t P, int64_t s_line, int
            P < (int64_t(1) << 31) && L < (int64_t(1) << 31);
 }
 
-size_t twopass_workspace(int64_t L, int G) { return round_up((size_t)G * (size_t)L * 4, 256); }
+// scratch of the table kernels: the (G, L) fp32 amax table, then the
+// (G, strips of 64 lines) merge counters of the single-read kernel
+size_t table_bytes(int64_t L, int G) { return round_up((size_t)G * (size_t)L * 4, 256); }
+size_t counter_bytes(int64_t L, int G) { return round_up((size_t)G * (size_t)((L + 63) / 64) * 4, 256); }
+size_t twopass_workspace(int64_t L, int G) { return table_bytes(L, G) + counter_bytes(L, G); }
+
+// partial-maximum slots of the single-read kernel: (strips, units + G, 64) fp32
+int64_t single_units(int64_t P, int64_t grid) { return std::min<int64_t>((P + 127) / 128, grid); }
+size_t partial_bytes(int64_t L, int64_t P, int G, int64_t grid)
+{
+    return round_up((size_t)((L + 63) / 64) * (size_t)(single_units(P, grid) + G) * 64 * 4, 256);
+}
 
 int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, int G, const void *out,
                 JaggedPlan *pl)
@@ -192,6 +221,22 @@ int plan_jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_
     int rc = device_info(&di);
     if (rc != MXQ_OK)
         return rc;
+    // the single-read kernel runs only when asked for: on B200 it is still
+    // slower than the two passes (its cross-CTA merges serialize)
+    if (force == 3 && di->coop && di->sg_per_sm >= 1) {
+        // single read: a strip's 128-position blocks fall into at most
+        // `grid` units (the grid is all resident) of at most MAX_UT blocks
+        const int64_t grid = (int64_t)di->sms * di->sg_per_sm;
+        const int64_t blocks = (P + jg1::TP - 1) / jg1::TP;
+        if (blocks <= grid * jg1::MAX_UT) {
+            pl->single = true;
+            pl->grid_s = (int)grid;
+            pl->ws = twopass_workspace(L, G) + partial_bytes(L, P, G, grid);
+            return MXQ_OK;
+        }
+    }
+    if (force == 3)
+        return MXQ_OK; // not eligible: the caller reports MXQ_ERR_UNSUPPORTED
     if (di->amx_per_sm < 1 || di->cst_per_sm < 1)
         return MXQ_OK;
     pl->twopass = true;
@@ -223,8 +268,38 @@ int jagged(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, 
     int rc = plan_jagged(in, L, P, s_line, s_pos, G, out, &pl);
     if (rc != MXQ_OK)
         return rc;
-    if (g_force_path.load() == 1 && !pl.twopass)
+    if ((g_force_path.load() == 1 && !pl.twopass) || (g_force_path.load() == 3 && !pl.single))
         return MXQ_ERR_UNSUPPORTED;
+    if (pl.single) {
+        if (!ws || ws_bytes < pl.ws)
+            return MXQ_ERR_WORKSPACE;
+        if (!aligned(ws, 256))
+            return MXQ_ERR_ALIGN;
+        CUtensorMap tc, to;
+        const uint64_t din[2] = {(uint64_t)L, (uint64_t)P};
+        const uint64_t sin[1] = {(uint64_t)s_pos * 2};
+        const uint32_t bc[2] = {jg1::TL, jg1::TP};
+        rc = make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, din, sin, bc, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc != MXQ_OK)
+            return rc;
+        const uint64_t dout[2] = {(uint64_t)P, (uint64_t)L};
+        const uint64_t sout[1] = {(uint64_t)P};
+        const uint32_t bo[2] = {jg1::TP, jg1::TL};
+        rc = make_map(&to, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bo, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc != MXQ_OK)
+            return rc;
+        unsigned *amax = static_cast<unsigned *>(ws);
+        int *counters = reinterpret_cast<int *>(static_cast<uint8_t *>(ws) + table_bytes(L, G));
+        unsigned *partials = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(ws) + twopass_workspace(L, G));
+        // the table and the counters start at zero; the partial slots are
+        // always written before they are read
+        if (cudaMemsetAsync(ws, 0, twopass_workspace(L, G), stream) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        const int pstride = (int)(single_units(P, pl.grid_s) + G);
+        return launch(k_jagged_single, dim3(pl.grid_s), dim3(jg1::THREADS), jg1::SMEM_BYTES, stream, true,
+                      tc, to, (int)L, (int)P, offs, G, amax, counters, partials, pstride, static_cast<uint8_t *>(out), inv,
+                      wait_ns(), g_drop_load.load());
+    }
     if (pl.twopass) {
         if (!ws || ws_bytes < pl.ws)
             return MXQ_ERR_WORKSPACE;
@@ -302,7 +377,11 @@ size_t fp8_quant_jagged_workspace_bytes(int64_t rows, int64_t cols, int64_t stri
     const int64_t sl = is_colwise ? stride_col : stride_row, sp = is_colwise ? stride_row : stride_col;
     if (!twopass_layout_ok(nullptr, L, P, sl, sp, num_groups, nullptr))
         return 0;
-    return twopass_workspace(L, num_groups);
+    // the single-read kernel's partial slots depend on the current device's
+    // resident grid; without device information, size for 1024 CTAs
+    const DevInfo *di = nullptr;
+    const int64_t grid = device_info(&di) == MXQ_OK ? (int64_t)di->sms * std::max(di->sg_per_sm, 1) : 1024;
+    return twopass_workspace(L, num_groups) + partial_bytes(L, P, num_groups, grid);
 }
 
 int fp8_quant_blockwise(const void *in, int64_t rows, int64_t cols, int32_t block_rows, int32_t block_cols,
@@ -695,6 +774,135 @@ int mx_quant_rowwise_blocked_grouped(const void *in, int64_t rows, int64_t cols,
 
 } // extern "C"
 
+namespace {
+
+// MX quantization along grouped positions, groups padded to 128 positions:
+// lines contiguous (s_line == 1), L a multiple of 128
+int mx_jagged_padded(const void *in, int64_t L, int64_t P, int64_t s_line, int64_t s_pos, const int32_t *offs, int G,
+                     int mode, void *out, int64_t cap, uint8_t *scales, cudaStream_t stream)
+{
+    if (L < 0 || P < 0 || G < 1 || cap < 0 || cap % 128)
+        return MXQ_ERR_SHAPE;
+    if (mode != MXQ_E8M0_FLOOR && mode != MXQ_E8M0_RCEIL)
+        return MXQ_ERR_UNSUPPORTED;
+    if (cap < mx_blocked_grouped_rows_bound(P, G))
+        return MXQ_ERR_SHAPE;
+    if (G > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if (L == 0 || cap == 0)
+        return MXQ_OK;
+    if (!offs || !out || !scales || (P > 0 && !in))
+        return MXQ_ERR_NULL;
+    if (L % 128)
+        return MXQ_ERR_SHAPE;
+    // the TMA path: lines contiguous, 16-byte aligned rows of positions
+    if (s_line != 1 || s_pos % 8 || s_pos < L)
+        return MXQ_ERR_UNSUPPORTED;
+    if ((in && !aligned(in, 16)) || !aligned(out, 16) || !aligned(scales, 16))
+        return MXQ_ERR_ALIGN;
+    if (P >= (int64_t(1) << 31) || L >= (int64_t(1) << 31) || cap >= (int64_t(1) << 31) ||
+        (cap / 128) * (L / 64) >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    CUtensorMap tin, tout;
+    // a map needs a non-zero extent: with P == 0 every tile is padding and
+    // the map is never read
+    const uint64_t din[2] = {(uint64_t)L, (uint64_t)std::max<int64_t>(P, 1)};
+    const uint64_t sin[1] = {(uint64_t)s_pos * 2};
+    const uint32_t bin[2] = {mxj::TL, mxj::TP};
+    rc = make_map(&tin, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, P > 0 ? in : out, din, sin, bin,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t dout[2] = {(uint64_t)cap, (uint64_t)L};
+    const uint64_t sout[1] = {(uint64_t)cap};
+    const uint32_t bout[2] = {mxj::TP, mxj::TL};
+    rc = make_map(&tout, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, out, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t items = (cap / 128) * (L / 64);
+    const int64_t grid = std::min<int64_t>(items, (int64_t)di->sms * std::max(di->mxj_per_sm, 1));
+    return launch(k_mx_jagged_colwise_padded, dim3((unsigned)grid), dim3(mxj::THREADS),
+                  mxj::SMEM_FIXED + (size_t)G * sizeof(int), stream, false, tin, tout, (int)L, (int)P, offs, G,
+                  (int)(cap / 128), scales, mode, wait_ns());
+}
+
+} // namespace
+
+extern "C" {
+
+int mx_quant_jagged_colwise_padded(const void *in, int64_t rows, int64_t cols, int64_t stride_row,
+                                   int64_t stride_col, const int32_t *offs, int32_t num_groups, int32_t mode,
+                                   void *out, int64_t out_cols_capacity, uint8_t *scales_blocked, cudaStream_t stream)
+{
+    // line = column, position = row
+    return mx_jagged_padded(in, cols, rows, stride_col, stride_row, offs, num_groups, mode, out, out_cols_capacity,
+                            scales_blocked, stream);
+}
+
+int mx_quant_jagged_rowwise_padded(const void *in, int64_t rows, int64_t cols, int64_t stride_row,
+                                   int64_t stride_col, const int32_t *offs, int32_t num_groups, int32_t mode,
+                                   void *out, int64_t out_cols_capacity, uint8_t *scales_blocked, cudaStream_t stream)
+{
+    // line = row, position = column
+    return mx_jagged_padded(in, rows, cols, stride_row, stride_col, offs, num_groups, mode, out, out_cols_capacity,
+                            scales_blocked, stream);
+}
+
+int mx_grouped_gemm_wgrad(const void *a, const uint8_t *sfa, const void *b, const uint8_t *sfb, int64_t N, int64_t K,
+                          int64_t M, int64_t capacity, const int32_t *offs, int32_t num_groups, void *out,
+                          cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || capacity < 0 || num_groups < 1 || N % gmx::BM || K % 128 || capacity % 128)
+        return MXQ_ERR_SHAPE;
+    if (capacity < mx_blocked_grouped_rows_bound(M, num_groups))
+        return MXQ_ERR_SHAPE;
+    if (num_groups > blk::MAX_G)
+        return MXQ_ERR_UNSUPPORTED;
+    if (N == 0 || K == 0)
+        return MXQ_OK;
+    if (!a || !sfa || !b || !sfb || !offs || !out)
+        return MXQ_ERR_NULL;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(sfa, 16) || !aligned(sfb, 16))
+        return MXQ_ERR_ALIGN;
+    if (capacity >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
+        M >= (int64_t(1) << 31))
+        return MXQ_ERR_UNSUPPORTED;
+    const DevInfo *di = nullptr;
+    int rc = device_info(&di);
+    if (rc != MXQ_OK)
+        return rc;
+    const int bn = K % 256 == 0 && g_mx_bn.load() != 128 ? 256 : 128;
+    CUtensorMap ta, tb;
+    const uint64_t cc = (uint64_t)std::max<int64_t>(capacity, 128); // a map needs a non-zero extent
+    const uint64_t da[2] = {cc, (uint64_t)N};
+    const uint64_t sa[1] = {cc};
+    const uint32_t boxa[2] = {gmx::BK, gmx::BM};
+    rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, boxa, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const uint64_t db[2] = {cc, (uint64_t)K};
+    const uint32_t boxb[2] = {gmx::BK, (uint32_t)bn};
+    rc = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, db, sa, boxb, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != MXQ_OK)
+        return rc;
+    const int64_t items = (int64_t)num_groups * (N / gmx::BM) * (K / bn);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(items, di->sms));
+    const size_t smem_g = (size_t)num_groups * sizeof(int);
+    if (bn == 256)
+        return launch(k_mx_grouped_gemm_wgrad<256>, dim3((unsigned)grid), dim3(gmx::THREADS),
+                      gmx::smem_fixed<256>() + smem_g, stream, false, ta, tb, sfa, sfb, N, K, M,
+                      (int)(capacity / 128), offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+    return launch(k_mx_grouped_gemm_wgrad<128>, dim3((unsigned)grid), dim3(gmx::THREADS),
+                  gmx::smem_fixed<128>() + smem_g, stream, false, ta, tb, sfa, sfb, N, K, M, (int)(capacity / 128),
+                  offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+}
+
+} // extern "C"
+
 // ---------------------------------------------------------------------------
 // Allocation-free variant of fp8_quant_jagged_colwise.
 //
@@ -812,7 +1020,7 @@ int mxq_testing_set(int32_t what, int64_t value)
     case MXQ_TESTING_WAIT_LIMIT_NS: g_wait_ns.store(value > 0 ? value : 1000000000LL); return MXQ_OK;
     case MXQ_TESTING_SKIP_ARRIVAL: g_drop_load.store(value ? 1 : 0); return MXQ_OK;
     case MXQ_TESTING_FORCE_PATH:
-        if (value < 0 || value > 2)
+        if (value < 0 || value > 3)
             return MXQ_ERR_UNSUPPORTED;
         g_force_path.store((int)value);
         return MXQ_OK;

@@ -143,9 +143,11 @@ def test_testing_hooks_accept_only_their_documented_values(lib):
     """mxq_testing_set: unknown hooks and out-of-range values are refused;
     every accepted value is put back to its default."""
     assert lib.mxq_testing_set(99, 0) == binding.ERR_UNSUPPORTED
-    assert lib.mxq_testing_set(binding.TESTING_FORCE_PATH, 3) == binding.ERR_UNSUPPORTED
+    assert lib.mxq_testing_set(binding.TESTING_FORCE_PATH, 4) == binding.ERR_UNSUPPORTED
+    assert lib.mxq_testing_set(binding.TESTING_FORCE_PATH, -1) == binding.ERR_UNSUPPORTED
     assert lib.mxq_testing_set(binding.TESTING_GEMM_TILE_N, 64) == binding.ERR_UNSUPPORTED
-    for hook, value in ((binding.TESTING_FORCE_PATH, 2), (binding.TESTING_GEMM_TILE_N, 128),
+    for hook, value in ((binding.TESTING_FORCE_PATH, 2), (binding.TESTING_FORCE_PATH, 3),
+                        (binding.TESTING_GEMM_TILE_N, 128),
                         (binding.TESTING_WAIT_LIMIT_NS, 5_000_000), (binding.TESTING_SKIP_ARRIVAL, 1)):
         assert lib.mxq_testing_set(hook, value) == binding.OK
         assert lib.mxq_testing_set(hook, 0) == binding.OK

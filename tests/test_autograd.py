@@ -166,7 +166,38 @@ def _mx_oracle_pipeline(a, w, dy, offs, mode):
     qd, sd = oracle.mx_quant_rowwise(dy, mode)
     wt, swt = oracle.mx_quant_3d_colwise(w, mode)   # (E, K, N) codes, (E, K, N/32) scales
     da = oracle.mx_grouped_gemm(qd, sd, wt, swt, o)
-    return dict(out=(out, qa, sa, qw, sw), da=(da, qd, sd, wt, swt))
+    # dW: dY^T and A in 32-token blocks from each group's first token
+    qdt, sdt = oracle.mx_quant_jagged_colwise(_words(dy).reshape(-1), M, N, N, 1, o, mode)   # (N, M)
+    qac, sac = oracle.mx_quant_jagged_colwise(_words(a).reshape(-1), M, K, K, 1, o, mode)   # (K, M)
+    dw = oracle.mx_grouped_gemm_wgrad(qdt, sdt, qac, sac, o)
+    return dict(out=(out, qa, sa, qw, sw), da=(da, qd, sd, wt, swt), dw=(dw, qdt, sdt, qac, sac))
+
+
+def _mx_token_values(codes, scales, offs):
+    """Values of codes (L, M) with scales (L, nblk) of 32-token blocks from
+    each group's first token."""
+    L, M = codes.shape
+    f = np.zeros((L, M))
+    s, base = 0, 0
+    for e in offs:
+        n = int(e) - s
+        for j in range((n + 31) // 32):
+            f[:, s + 32 * j:min(s + 32 * j + 32, s + n)] = 2.0 ** (scales[:, base + j:base + j + 1] - 127.0)
+        base += (n + 31) // 32
+        s = int(e)
+    return DEC_SIGNED[codes] * f
+
+
+def _check_mx_wgrad(got, ref, qa, sa, qb, sb, offs):
+    xa, xb = np.abs(_mx_token_values(qa, sa, offs)), np.abs(_mx_token_values(qb, sb, offs))
+    g64 = got.float().cpu().numpy().astype(np.float64)
+    s = 0
+    for g, e in enumerate(offs):
+        n = int(e) - s
+        S = xa[:, s:e] @ xb[:, s:e].T
+        bound = 2.0 ** -8 * np.abs(ref[g]) + ((n + 127) // 128 * 128) * 2.0 ** -23 * S
+        assert np.max(np.abs(g64[g] - ref[g]) - bound) <= 0, g
+        s = int(e)
 
 
 def _check_mx_grouped(got, ref, qa, sa, qw, sw, offs, K):
@@ -199,9 +230,14 @@ def test_mx_oracle_pipeline_approximates_the_exact_products():
     for g, e in enumerate(ends):
         out[s:e], da[s:e] = A[s:e] @ W[g].T, D[s:e] @ W[g]
         s = e
+    dw = np.stack([D[(ends[g - 1] if g else 0):ends[g]].T @ A[(ends[g - 1] if g else 0):ends[g]] for g in range(E)])
     end = ends[-1]
-    for got, want in ((r["out"][0][:end], out[:end]), (r["da"][0][:end], da[:end])):
+    for got, want in ((r["out"][0][:end], out[:end]), (r["da"][0][:end], da[:end]), (r["dw"][0], dw)):
         assert np.linalg.norm(got - want) <= 0.08 * np.linalg.norm(want)
+    # dW of a group is its own tokens' product: moving one token across a
+    # group end changes both groups by order one
+    moved = _mx_oracle_pipeline(a, w, dy, [65, 65, 240], oracle.FLOOR)["dw"][0]
+    assert np.linalg.norm(moved[0] - dw[0]) > 0.01 * np.linalg.norm(dw[0])
 
 
 @pytest.mark.gpu
@@ -225,5 +261,5 @@ def test_mx_forward_and_backward_vs_oracle(mode):
     _check_mx_grouped(out.detach(), r, qa, sa, qw, sw, ends, K)
     r, qd, sd, wt, swt = ref["da"]
     _check_mx_grouped(ad.grad, r, qd, sd, wt, swt, ends, N)
-    r, dytq, idyt, acq, iac = _oracle_pipeline(a, w, dy, ends)["dw"]
-    _check_wgrad(wd.grad, r, dytq, idyt, acq, iac, ends)
+    r, qdt, sdt, qac, sac = ref["dw"]
+    _check_mx_wgrad(wd.grad, r, qdt, sdt, qac, sac, ends)

@@ -80,10 +80,14 @@ JAGGED = [
     (9600, 72, [17, 4000, 4001, 9583]),  # several position chunks per CTA range
     (256, 64, [0, 0, 0]),                # every group empty: only inverse scales written
     (1024, 4104, [100, 700, 1024]),      # 17 line chunks, the last one 8 lines wide
+    # eleven groups in the first 128 rows, the last of them running on: the
+    # single-read kernel keeps 8 groups of a unit in shared memory and the
+    # rest (here also one spanning two units) in the global table
+    (1024, 136, [10, 20, 30, 40, 50, 60, 70, 80, 90, 100, 200, 300, 1024]),
 ]
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["two_pass", "generic"])
+@pytest.mark.parametrize("path", [1, 2, 3], ids=["two_pass", "generic", "single_read"])
 @pytest.mark.parametrize("M,D,spec", JAGGED)
 def test_jagged_colwise_and_rowwise_vs_oracle(M, D, spec, path):
     mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
@@ -190,7 +194,7 @@ def test_jagged_colwise_strided_view_generic():
     assert np.array_equal(f32bits(inv.cpu().numpy()), f32bits(ref_inv))
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["two_pass", "generic"])
+@pytest.mark.parametrize("path", [1, 2, 3], ids=["two_pass", "generic", "single_read"])
 def test_jagged_colwise_padded_rows_partial_lane(path):
     """Row stride 208 elements, 203 columns: the last lane of the two-pass
     amax pass holds 3 of its 8 lines, and the TMA maps see a padded stride."""
@@ -659,7 +663,7 @@ def test_mx_rowwise_blocked_full_size_is_rowwise_then_conversion():
 
 def test_bad_offsets_are_reported_and_nothing_is_written():
     x = synth.row_scaled_normal_bf16(256, 64, seed=1, device=DEV)
-    for path in (1, 2):
+    for path in (1, 2, 3):
         mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
         for bad in ([64, 32, 256], [-16, 256], [64, 272]):
             out = torch.full((64, 256), SENT, dtype=torch.uint8, device=DEV)
@@ -675,14 +679,16 @@ def test_bad_offsets_are_reported_and_nothing_is_written():
     assert mxq.device_status() == 0  # cleared by the read
 
 
-def test_barrier_timeout_is_reported_and_context_survives():
-    """One CTA of the cast pass leaves its first TMA load unissued: the bounded
-    waits on that ring slot expire, the kernels return, the status reads
-    TIMEOUT and the next call on the same context is correct."""
+@pytest.mark.parametrize("path", [1, 3], ids=["two_pass", "single_read"])
+def test_barrier_timeout_is_reported_and_context_survives(path):
+    """CTA 0 leaves its first TMA load unissued: the bounded waits on that
+    ring slot expire (and, on the single-read kernel, the other CTAs' waits
+    for that unit's share of the group maxima), the kernels return, the
+    status reads TIMEOUT and the next call on the same context is correct."""
     x = synth.row_scaled_normal_bf16(4096, 128, seed=2, device=DEV)
     offs = torch.tensor([1000, 4096], dtype=torch.int32)
     try:
-        mxq.testing_set(mxq.TESTING_FORCE_PATH, 1)
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
         mxq.testing_set(mxq.TESTING_WAIT_LIMIT_NS, 20_000_000)
         mxq.testing_set(mxq.TESTING_SKIP_ARRIVAL, 1)
         mxq.fp8_quant_jagged_colwise(x, offs.to(DEV))

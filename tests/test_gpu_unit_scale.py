@@ -8,8 +8,8 @@ PR 2827 "[fp8 blockwise] load 2d chunks ...").
 * Every non-negative finite bf16 value (+0 and the subnormals below the 1e-12
   floor included, up to the largest finite bf16) is the amax of one unit,
   with unit mates at fixed fractions of it. Each unit goes through the
-  jagged ops on all three of their kernels (two-pass TMA kernels, the
-  contiguous-rows kernel, the generic kernel) and through blockwise 1x128 and
+  jagged ops on all four of their kernels (single-read and two-pass TMA
+  kernels, the contiguous-rows kernel, the generic kernel) and through blockwise 1x128 and
   the transposed 128x1 op; every inverse-scale bit and every code is compared
   with the oracle.
 * The hand-worked fixtures of tests/golden/ (unit scales and e4m3 codes) run
@@ -91,7 +91,7 @@ def _jagged_input():
     return _bf16(np.concatenate([g0.T, g1.T], axis=0)), n
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["two_pass", "generic"])
+@pytest.mark.parametrize("path", [1, 2, 3], ids=["two_pass", "generic", "single_read"])
 def test_jagged_unit_scale_every_bf16_amax(path):
     x, n = _jagged_input()
     M = x.shape[0]
@@ -169,7 +169,7 @@ def _fp8_units():
     return units
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["two_pass", "generic"])
+@pytest.mark.parametrize("path", [1, 2, 3], ids=["two_pass", "generic", "single_read"])
 def test_golden_fp8_units_through_jagged(path):
     units = _fp8_units()
     # each unit is one column of a single row group of 16 (zero padded); 8

@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 # jagged paths whose kernels keep the amax table in scratch memory
-SCRATCH_PATHS = [1]
+SCRATCH_PATHS = [1, 3]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -91,14 +91,15 @@ def test_noalloc_small_problem_needs_no_scratch():
     assert torch.equal(inv.view(torch.int32), want_inv.view(torch.int32))
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+@pytest.mark.parametrize("path", SCRATCH_PATHS)
+def test_noalloc_rejects_problems_beyond_its_scratch(path):
     # forced onto the table kernels, 64 groups x 8192 columns of fp32 amax
     # need 2 MiB > 1 MiB: refused, nothing launched
     x = torch.zeros((64, 8192), dtype=torch.bfloat16, device=DEV)
     offs = torch.arange(1, 65, dtype=torch.int32, device=DEV)
     out = torch.empty((8192, 64), dtype=torch.uint8, device=DEV)
     inv = torch.empty((64, 8192), dtype=torch.float32, device=DEV)
-    mxq.testing_set(mxq.TESTING_FORCE_PATH, 1)
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, path)
     try:
         with pytest.raises(mxq.MXQError) as ei:
             mxq.fp8_quant_jagged_colwise_noalloc(x, offs, out=out, inv_scales=inv)
