@@ -403,7 +403,7 @@ def flush_l2_clean(torch, buf, sink):
     lines of `buf` only, so the next kernel starts cold without first having
     to write back the flush's own dirty lines."""
     buf.zero_()
-    torch.sum(buf.view(torch.int32), dtype=torch.int64, out=sink)
+    torch.sum(buf.view(torch.int64), dim=0, out=sink)
 
 
 def per_shape_sweep(wl, reps):
@@ -454,6 +454,8 @@ def per_shape_sweep(wl, reps):
                      "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4),
                      "us_clean": round(usc, 3), "frac_measured_clean": round(nbytes / (usc * 1e-6) / 1e9 / peak, 4),
                      "us_hot": round(statistics.median(hot), 3), "enqueue_us": round(statistics.median(enq), 1)})
+
+    run.rows = rows
 
     # tiny jagged
     a, offs = synth.tiny_jagged(device=dev)
@@ -526,7 +528,126 @@ def per_shape_sweep(wl, reps):
     # grouped GEMM on the tensor cores, fed by the rowwise quantization:
     # tokens (65536, 7168) in the 64 Dirichlet(0.3) groups x 64 experts (2048, 7168)
     rows += gemm_rows(wl, flush, reps)
+    rows += jagged_extra_rows(wl, run)
+    rows += mx_wgrad_rows(wl, run, flush, reps)
+    rows += grouped_mm_rows(wl, flush, max(reps // 5, 5))
     del flush
+    return rows
+
+
+def jagged_extra_rows(wl, run):
+    """The jagged colwise op on its single-read kernel (forced; the automatic
+    choice is the two-pass kernels), labelled as such."""
+    mxq = wl.mxq
+    if not hasattr(wl, "inp"):
+        return []
+    rows = []
+    M, D = wl.inp.shape
+    mxq.testing_set(mxq.TESTING_FORCE_PATH, 3)
+    try:
+        before = len(run.rows)
+        run("jagged_colwise_single_read", "(65536,4096) G=16",
+            lambda: mxq.fp8_quant_jagged_colwise(wl.inp, wl.offs16), M * D * 3 + 16 * D * 4)
+        rows = run.rows[before:]
+        del run.rows[before:]
+    finally:
+        mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+    return rows
+
+
+def mx_wgrad_rows(wl, run, flush, reps):
+    """The MXFP8 weight gradient on the jagged backward config: MX
+    quantization of grad_out^T and of the input along each group's tokens
+    (groups padded to 128 tokens, blocked scales), then the block-scaled
+    weight-gradient GEMM (16, 4096, 4096) against the FP8 dense peak."""
+    torch, mxq = wl.torch, wl.mxq
+    if not hasattr(wl, "inp"):
+        return []
+    M, D = wl.inp.shape
+    G = 16
+    cap = mxq.blocked_grouped_rows_bound(M, G)
+    qa = torch.empty((D, cap), dtype=torch.uint8, device=wl.dev)
+    sa = torch.empty(D * cap // 32, dtype=torch.uint8, device=wl.dev)
+    qb = torch.empty((D, cap), dtype=torch.uint8, device=wl.dev)
+    sb = torch.empty(D * cap // 32, dtype=torch.uint8, device=wl.dev)
+    nbytes = M * D * 2 + D * cap + D * cap // 32
+    before = len(run.rows)
+    run("mx_jagged_rowwise_padded", "(4096,65536)^T G=16 floor",
+        lambda: mxq.mx_quant_jagged_rowwise_padded(wl.grad_out.t(), wl.offs16, "floor", capacity=cap, out=qa,
+                                                   scales=sa), nbytes)
+    run("mx_jagged_colwise_padded", "(65536,4096) G=16 floor",
+        lambda: mxq.mx_quant_jagged_colwise_padded(wl.inp, wl.offs16, "floor", capacity=cap, out=qb, scales=sb),
+        nbytes)
+    rows = run.rows[before:]
+    del run.rows[before:]
+    out = torch.empty((G, D, D), dtype=torch.bfloat16, device=wl.dev)
+    fn = lambda: mxq.mx_grouped_gemm_wgrad(qa, sa, qb, sb, wl.offs16, M, out=out)
+    us = _median_us(torch, fn, max(reps // 5, 3), flush)
+    tf = 2.0 * M * D * D / (us * 1e-6) / 1e12
+    peak, kind = _fp8_peak()
+    rows.append({"op": "mx_grouped_gemm_wgrad", "shape": f"({D},{cap})x({D},{cap}) G=16 -> (16,{D},{D})",
+                 "us": round(us, 3), "TFLOP/s": round(tf, 1), "frac_fp8_peak": round(tf / peak, 4),
+                 "peak_TFLOP/s": round(peak, 1), "peak_kind": kind})
+    del qa, qb, out
+    return rows
+
+
+def _fp8_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 2"
+    except Exception:
+        return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
+def _median_us(torch, fn, reps, flush):
+    """Median device time of `fn` over `reps` calls, L2 flushed before each."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush_l2(torch, flush)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    return statistics.median(ts)
+
+
+def grouped_mm_rows(wl, flush, reps):
+    """One forward + backward of the differentiable grouped matmuls at the
+    shapes of the page "[scaled grouped mm] integrate triton kernels into
+    differentiable scaled grouped mm" (Performance): tokens A (M, 4096) with
+    M in {256, 4096, 65536} x experts B (E, 4096, 4096) with E in {4, 8, 16},
+    the tokens split equally among the experts (the page does not give its
+    group sizes). Device time of out = mm(a, w, offs); out.backward(dy), and
+    its TFLOP/s over the three GEMMs (6 M N K)."""
+    torch = wl.torch
+    from mxfp8_quantization_moe_device_b200 import synth
+    from mxfp8_quantization_moe_device_b200.autograd import fp8_grouped_mm, mx_grouped_mm
+    dev = wl.dev
+    rows = []
+    K = N = 4096
+    for M in (256, 4096, 65536):
+        a = synth.row_scaled_normal_bf16(M, K, seed=81, device=dev).requires_grad_(True)
+        dy = synth.row_scaled_normal_bf16(M, N, seed=82, device=dev)
+        for E in (4, 8, 16):
+            w = synth.normal_bf16((E, N, K), 0.02, 83, device=dev).requires_grad_(True)
+            offs = torch.arange(M // E, M + 1, M // E, dtype=torch.int32).to(dev)
+            for name, mm in (("fp8_grouped_mm", lambda: fp8_grouped_mm(a, w, offs)),
+                             ("mx_grouped_mm", lambda: mx_grouped_mm(a, w, offs, "floor"))):
+                def step(mm=mm):
+                    a.grad, w.grad = None, None
+                    mm().backward(dy)
+                us = _median_us(torch, step, reps, flush)
+                rows.append({"op": name + "_fwd_bwd", "shape": f"A ({M},{K}) x B ({E},{N},{K})", "us": round(us, 1),
+                             "TFLOP/s": round(6.0 * M * N * K / (us * 1e-6) / 1e12, 1)})
+            del w
+        del a, dy
     return rows
 
 

@@ -180,6 +180,20 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
                              const int32_t *offs, int32_t num_groups, void *out,
                              cudaStream_t stream);
 
+/* fp8_grouped_gemm_rowwise with W at any row and group strides (bytes):
+ * w[g][n][k] at w + g * w_group_stride + n * w_row_stride + k. Both strides
+ * multiples of 16, w_row_stride >= K (MXQ_ERR_ALIGN otherwise). The plain
+ * call is w_row_stride = K, w_group_stride = N * K. A row-major (K', G * N')
+ * matrix holding every expert's W_e^T side by side (the column-major output
+ * of fp8_quant_jagged_colwise on W viewed as (G * N', K') with one group per
+ * expert) is read with N = K', K = N', w_row_stride = G * N',
+ * w_group_stride = N'. */
+int fp8_grouped_gemm_rowwise_strided(const void *a, const float *inv_a, const void *w, const float *inv_w,
+                                     int64_t M, int64_t N, int64_t K,
+                                     int64_t w_row_stride, int64_t w_group_stride,
+                                     const int32_t *offs, int32_t num_groups, void *out,
+                                     cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ *
  * mx_grouped_gemm - the MXFP8 consumer of the MX rowwise quantization and of
  * the per-group 128x4 blocked scale layout (#3504 title: per-group blocked

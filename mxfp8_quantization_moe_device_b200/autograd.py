@@ -12,7 +12,8 @@ tokens, so its operands need one scale per (expert group, row) and per
 Scale granularity of each GEMM (one e4m3 scale per listed unit, amax over the
 contracted dimension):
   forward   out = A W^T      A per token (over K), W per (expert, n) (over K)
-  input     dA  = dY W       dY per token (over N), W per (expert, k) (over N)
+  input     dA  = dY W       dY per token (over N), W per (expert, k) (over N:
+                             one jagged colwise launch for all experts)
   weight    dW  = dY^T A     dY per (group, n) and A per (group, k), both over
                              the group's tokens (the jagged rowwise and
                              colwise ops)
@@ -30,9 +31,10 @@ in the groups-along-K blocked layout, into the block-scaled weight-gradient
 grouped GEMM.
 
 Nothing here computes on the host: quantization and GEMMs are the library's
-CUDA kernels (torch only allocates and zero-fills outputs, and makes an
-incoming gradient contiguous bf16), so a missing library raises instead of
-falling back.
+CUDA kernels (torch only allocates and zero-fills outputs, makes an incoming
+gradient contiguous bf16, and copies the expert boundaries of W viewed as
+(E*N, K) to the device), so a missing library raises instead of falling
+back.
 """
 import torch
 
@@ -76,16 +78,14 @@ def _grad_input(dy, w, offs):
     M, N = dy.shape
     E, _, K = w.shape
     dyq, idy = _rowwise(dy, N)
-    # W_e^T per expert: the colwise op on W_e (N, K) with one group over all
-    # N rows writes the column-major buffer, i.e. W_e^T (K, N) row-major, with
-    # one scale per (expert, k)
-    wt = torch.empty((E, K, N), dtype=torch.uint8, device=w.device)
-    iwt = torch.empty((E, K), dtype=torch.float32, device=w.device)
-    nn = torch.tensor([N], dtype=torch.int32, device=w.device)
-    for e in range(E):
-        mxq.fp8_quant_jagged_colwise(w[e], nn, out=wt[e], inv_scales=iwt[e].view(1, K))
+    # every W_e^T in one launch: the colwise op on W viewed as (E*N, K) with
+    # one group of N rows per expert writes the (K, E*N) buffer whose row k
+    # holds W_e[:, k] of every expert side by side, one scale per (expert, k);
+    # the GEMM reads it through its strided weight operand
+    ends = torch.arange(N, E * N + 1, N, dtype=torch.int32).to(w.device)
+    wtq, iwt = mxq.fp8_quant_jagged_colwise(w.reshape(E * N, K), ends)
     da = torch.zeros((M, K), dtype=torch.bfloat16, device=dy.device)
-    return mxq.fp8_grouped_gemm_rowwise(dyq, idy, wt, iwt, offs, out=da)
+    return mxq.fp8_grouped_gemm_rowwise_wt(dyq, idy, wtq.t().view(torch.uint8), iwt, offs, out=da)
 
 
 def _grad_weight(dy, a, offs):

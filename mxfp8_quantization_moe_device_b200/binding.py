@@ -39,6 +39,8 @@ SIGNATURES = {
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "fp8_grouped_gemm_rowwise": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
+    "fp8_grouped_gemm_rowwise_strided": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i32,
+                                                        _vp, _vp]),
     "mx_grouped_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "mx_quant_rowwise": (ctypes.c_int, [_vp, _i64, _i64, _i32, _vp, _vp, _vp]),
     "mx_scales_to_blocked_grouped": (ctypes.c_int, [_vp, _i64, _i64, _vp, _i32, _vp, _i64, _vp, _vp]),
@@ -412,6 +414,37 @@ def fp8_grouped_gemm_rowwise(a, inv_a, w, inv_w, offs, *, out=None):
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     _call("fp8_grouped_gemm_rowwise", dev, _ptr(a), _ptr(inv_a), _ptr(w), _ptr(inv_w), M, N, K, _ptr(offs), E,
           _ptr(out))
+    return out
+
+
+def fp8_grouped_gemm_rowwise_wt(a, inv_a, wt, inv_w, offs, *, out=None):
+    """fp8_grouped_gemm_rowwise with every expert's weight given transposed
+    and side by side: wt (K_w, E * N_w) e4m3 row-major, row k holding
+    W_e[:, k] of every expert e (the column-major buffer of
+    fp8_quant_jagged_colwise on W viewed as (E * N_w, K_w) with one group of
+    N_w rows per expert), inv_w (E, K_w). Computes out[m] = (a[m] .
+    W_e[:, :]^T-as-read) * inv_a[m] * inv_w[e] with contraction over N_w:
+    out (M, K_w) bf16, a (M, N_w) e4m3, inv_a (M,)."""
+    for t, n in ((a, "a"), (inv_a, "inv_a"), (wt, "wt"), (inv_w, "inv_w")):
+        _cuda(t, n)
+        if not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous")
+    if a.element_size() != 1 or wt.element_size() != 1 or a.dim() != 2 or wt.dim() != 2:
+        raise TypeError("a must be (M, N_w) and wt (K_w, E * N_w), one byte per element (e4m3)")
+    if inv_a.dtype != torch.float32 or inv_w.dtype != torch.float32:
+        raise TypeError("inv_a and inv_w must be float32")
+    dev = a.device
+    _offsets(offs, dev)
+    M, Nw = a.shape
+    Kw, EN = wt.shape
+    E = offs.numel()
+    if EN != E * Nw or inv_a.numel() != M or inv_w.numel() != E * Kw:
+        raise TypeError("shape mismatch between a, wt, inv_a, inv_w and offs")
+    if out is None:
+        out = torch.empty((M, Kw), dtype=torch.bfloat16, device=dev)
+    _out_buffer(out, "out", (M, Kw), 2, dev, torch.bfloat16)
+    _call("fp8_grouped_gemm_rowwise_strided", dev, _ptr(a), _ptr(inv_a), _ptr(wt), _ptr(inv_w), M, Kw, Nw, E * Nw,
+          Nw, _ptr(offs), E, _ptr(out))
     return out
 
 

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
     k_fp8_grouped_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                        const float *__restrict__ inv_a, const float *__restrict__ inv_w, int64_t M, int64_t N,
                        int64_t K, const int32_t *__restrict__ offs, int G, uint16_t *__restrict__ out,
-                       uint64_t wait_ns)
+                       uint64_t wait_ns, int w_group_inner)
 {
     using namespace gm;
     constexpr int B_BYTES = BN * BK;
@@ -192,7 +192,12 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
                     tma_load_2d(sm.a[s], &tm_a, &sm.full[s], (int)(kb * BK), (int)m0);
-                    tma_load_2d(sm.b[s], &tm_w, &sm.full[s], (int)(kb * BK), (int)((int64_t)g * N + nt * BN));
+                    // W's map is (k, n, group), or (k, group, n) when the
+                    // group stride is the smaller one
+                    if (w_group_inner)
+                        tma_load_3d(sm.b[s], &tm_w, &sm.full[s], (int)(kb * BK), g, (int)(nt * BN));
+                    else
+                        tma_load_3d(sm.b[s], &tm_w, &sm.full[s], (int)(kb * BK), (int)(nt * BN), g);
                 }
             }
             // drain: every issued fill lands before the CTA exits

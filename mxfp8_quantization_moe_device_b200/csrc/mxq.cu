@@ -457,9 +457,9 @@ int fp8_quant_blockwise_transposed(const void *in, int64_t rows, int64_t cols, i
                   tout, inv_scales, rows, cols, (int)block_cols, wait_ns());
 }
 
-int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, const float *inv_w, int64_t M,
-                             int64_t N, int64_t K, const int32_t *offs, int32_t num_groups, void *out,
-                             cudaStream_t stream)
+int fp8_grouped_gemm_rowwise_strided(const void *a, const float *inv_a, const void *w, const float *inv_w, int64_t M,
+                                     int64_t N, int64_t K, int64_t w_row_stride, int64_t w_group_stride,
+                                     const int32_t *offs, int32_t num_groups, void *out, cudaStream_t stream)
 {
     if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % 128 || K % gm::BK)
         return MXQ_ERR_SHAPE;
@@ -473,7 +473,12 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
         return MXQ_ERR_NULL;
     if (!aligned(a, 16) || !aligned(w, 16) || !aligned(out, 16) || !aligned(inv_a, 4) || !aligned(inv_w, 4))
         return MXQ_ERR_ALIGN;
-    if (M >= (int64_t(1) << 31) || (int64_t)num_groups * N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    // W rows must not overlap and start on 16-byte boundaries (TMA strides)
+    if (w_row_stride < K || w_row_stride % 16 || w_group_stride < 0 || w_group_stride % 16 ||
+        (num_groups > 1 && w_group_stride == 0))
+        return MXQ_ERR_ALIGN;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) ||
+        num_groups >= (int64_t(1) << 31))
         return MXQ_ERR_UNSUPPORTED;
     const DevInfo *di = nullptr;
     int rc = device_info(&di);
@@ -486,11 +491,17 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
     rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
-    // tiles 128 x 256 when N allows, else 128 x 128
+    // tiles 128 x 256 when N allows, else 128 x 128; W through a rank-3 map
+    // with its dimensions in increasing stride order: (k, n, group), or
+    // (k, group, n) when the groups sit side by side within a row
     const int bn = N % 256 == 0 ? 256 : 128;
-    const uint64_t dw[2] = {(uint64_t)K, (uint64_t)(num_groups * N)};
-    const uint32_t boxw[2] = {gm::BK, (uint32_t)bn};
-    rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w, dw, sa, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
+    const int group_inner = num_groups > 1 && w_group_stride < w_row_stride ? 1 : 0;
+    const uint64_t gs = (uint64_t)std::max<int64_t>(w_group_stride, 16);
+    const uint64_t dw[3] = {(uint64_t)K, group_inner ? (uint64_t)num_groups : (uint64_t)N,
+                            group_inner ? (uint64_t)N : (uint64_t)num_groups};
+    const uint64_t sw[2] = {group_inner ? gs : (uint64_t)w_row_stride, group_inner ? (uint64_t)w_row_stride : gs};
+    const uint32_t boxw[3] = {gm::BK, group_inner ? 1u : (uint32_t)bn, group_inner ? (uint32_t)bn : 1u};
+    rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w, dw, sw, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
     // work items: at most (M / 128 + G) m-tiles times N / bn n-tiles
@@ -499,10 +510,18 @@ int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, c
     if (bn == 256)
         return launch(k_fp8_grouped_gemm<256>, dim3((unsigned)grid), dim3(gm::THREADS),
                       gm::smem_fixed<256>() + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M,
-                      N, K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+                      N, K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns(), group_inner);
     return launch(k_fp8_grouped_gemm<128>, dim3((unsigned)grid), dim3(gm::THREADS),
                   gm::smem_fixed<128>() + (size_t)num_groups * sizeof(int), stream, false, ta, tw, inv_a, inv_w, M, N,
-                  K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
+                  K, offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns(), group_inner);
+}
+
+int fp8_grouped_gemm_rowwise(const void *a, const float *inv_a, const void *w, const float *inv_w, int64_t M,
+                             int64_t N, int64_t K, const int32_t *offs, int32_t num_groups, void *out,
+                             cudaStream_t stream)
+{
+    // W (num_groups, N, K) row-major
+    return fp8_grouped_gemm_rowwise_strided(a, inv_a, w, inv_w, M, N, K, K, N * K, offs, num_groups, out, stream);
 }
 
 int mx_grouped_gemm(const void *a, const void *sfa, const void *w, const void *sfw, int64_t M, int64_t N, int64_t K,
