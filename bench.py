@@ -82,7 +82,8 @@ KERNEL_FILES = {  # source files that define each kernel (plus common.cuh)
     "k_jagged_amax": "jagged.cuh", "k_jagged_cast": "jagged.cuh", "k_mx_3d_colwise": "mx3d.cuh",
     "k_blocked_grouped": "blocked.cuh", "k_blocked_grouped_k": "blocked.cuh", "k_mx_1x32_blocked": "blocked.cuh",
     "k_fp8_blockwise_t": "blockt.cuh", "k_fp8_grouped_gemm": "gemm.cuh", "k_fp8_grouped_gemm_wgrad": "gemm.cuh",
-    "k_mx_grouped_gemm": "gemm_mx.cuh",
+    "k_mx_grouped_gemm": "gemm_mx.cuh", "k_jagged_single": "jagged1.cuh", "k_mx_jagged_colwise_padded": "mxj.cuh",
+    "k_mx_grouped_gemm_wgrad": "mxj.cuh",
 }
 
 
@@ -198,7 +199,8 @@ class Workload:
            "mx_rowwise", "blocked_grouped")
     # ops outside the step (the widened rows), built only when asked for by name
     EXTRA = ("blockwise_128x1_t", "blockwise_128x128_t", "blocked_grouped_k", "mx_rowwise_blocked", "grouped_gemm",
-             "grouped_gemm_wgrad", "mx_grouped_gemm")
+             "grouped_gemm_wgrad", "mx_grouped_gemm", "mx_jagged_colwise_padded", "mx_grouped_gemm_wgrad",
+             "jagged_colwise_single_read")
 
     def __init__(self, dev, experts, mx3d_mode, only=None):
         import torch
@@ -323,6 +325,41 @@ class Workload:
             self.o.update(x_out=t.empty((T, N), dtype=t.bfloat16, device=dev))
             self.ops.append(("mx_grouped_gemm", lambda: mxq.mx_grouped_gemm(
                 self.x_a, self.x_sa, self.x_w, self.x_sw, self.x_offs, out=self.o["x_out"]), 2 * T * N * K))
+
+        if want & {"mx_jagged_colwise_padded", "mx_grouped_gemm_wgrad", "jagged_colwise_single_read"}:
+            # the jagged backward config: grad_out^T (4096, 65536) and input (65536, 4096), G=16
+            go, x, offs16 = synth.jagged_bwd(device=dev)
+            self.offs16 = offs16.to(dev)
+            M, D = x.shape
+            cap = mxq.blocked_grouped_rows_bound(M, 16)
+            if "jagged_colwise_single_read" in want:
+                self.inp = x
+                self.o.update(in_q=t.empty((D, M), **u8), in_s=t.empty((16, D), **f32))
+
+                def single():
+                    mxq.testing_set(mxq.TESTING_FORCE_PATH, 3)
+                    try:
+                        mxq.fp8_quant_jagged_colwise(self.inp, self.offs16, out=self.o["in_q"],
+                                                     inv_scales=self.o["in_s"])
+                    finally:
+                        mxq.testing_set(mxq.TESTING_FORCE_PATH, 0)
+                self.ops.append(("jagged_colwise_single_read", single, M * D * 3 + 16 * D * 4))
+            if want & {"mx_jagged_colwise_padded", "mx_grouped_gemm_wgrad"}:
+                self.inp = x
+                self.o.update(mq=t.empty((D, cap), **u8), ms=t.empty(D * cap // 32, **u8))
+                if "mx_jagged_colwise_padded" in want:
+                    self.ops.append(("mx_jagged_colwise_padded", lambda: mxq.mx_quant_jagged_colwise_padded(
+                        self.inp, self.offs16, "floor", capacity=cap, out=self.o["mq"], scales=self.o["ms"]),
+                        M * D * 2 + D * cap + D * cap // 32))
+                else:
+                    qa, sa = mxq.mx_quant_jagged_rowwise_padded(go.t(), self.offs16, "floor", capacity=cap)
+                    mxq.mx_quant_jagged_colwise_padded(x, self.offs16, "floor", capacity=cap, out=self.o["mq"],
+                                                       scales=self.o["ms"])
+                    self.mw = (qa.view(t.uint8), sa, self.o["mq"], self.o["ms"], M)
+                    self.o.update(mw_out=t.empty((16, D, D), dtype=t.bfloat16, device=dev))
+                    self.ops.append(("mx_grouped_gemm_wgrad", lambda: mxq.mx_grouped_gemm_wgrad(
+                        *self.mw[:4], self.offs16, self.mw[4], out=self.o["mw_out"]), 2 * M * D * D))
+            del go
 
         if "grouped_gemm_wgrad" in want:
             # the jagged backward config: grad_out^T (4096, 65536) and input (65536, 4096), G=16

@@ -266,3 +266,73 @@ def fp8_grouped_gemm_wgrad(a: torch.Tensor, inv_a: torch.Tensor, b: torch.Tensor
 def _(a, inv_a, b, inv_b, offs):
     return a.new_empty((offs.shape[0], a.shape[0], b.shape[0]), dtype=torch.bfloat16)
 
+
+@torch.library.custom_op("mxq::mx_quant_jagged_colwise_padded", mutates_args=())
+def mx_quant_jagged_colwise_padded(x: torch.Tensor, offs: torch.Tensor, mode: str) -> tuple[torch.Tensor, torch.Tensor]:
+    """MXFP8 along the rows of x (rows, cols) in 32-row blocks from each
+    group's first row, each group padded to 128 rows: (q (cols, capacity)
+    e4m3, blocked scales of the (cols, capacity / 32) matrix, flat uint8)."""
+    rows, cols = x.shape
+    cap = _rows_cap(rows, offs.shape[0])
+    q = torch.empty((cols, cap), dtype=torch.uint8, device=x.device)
+    sc = torch.empty((cols * cap // 32,), dtype=torch.uint8, device=x.device)
+    _b.mx_quant_jagged_colwise_padded(x, offs, _mode(mode), capacity=cap, out=q, scales=sc)
+    return q.view(_F8), sc
+
+
+@mx_quant_jagged_colwise_padded.register_fake
+def _(x, offs, mode):
+    rows, cols = x.shape
+    cap = _rows_cap(rows, offs.shape[0])
+    return x.new_empty((cols, cap), dtype=_F8), x.new_empty((cols * cap // 32,), dtype=torch.uint8)
+
+
+@torch.library.custom_op("mxq::mx_quant_jagged_rowwise_padded", mutates_args=())
+def mx_quant_jagged_rowwise_padded(x: torch.Tensor, offs: torch.Tensor, mode: str) -> tuple[torch.Tensor, torch.Tensor]:
+    """MXFP8 along the columns of x (rows, cols) in 32-column blocks from each
+    group's first column, each group padded to 128 columns: (q (rows,
+    capacity) e4m3, blocked scales of the (rows, capacity / 32) matrix)."""
+    rows, cols = x.shape
+    cap = _rows_cap(cols, offs.shape[0])
+    q = torch.empty((rows, cap), dtype=torch.uint8, device=x.device)
+    sc = torch.empty((rows * cap // 32,), dtype=torch.uint8, device=x.device)
+    _b.mx_quant_jagged_rowwise_padded(x, offs, _mode(mode), capacity=cap, out=q, scales=sc)
+    return q.view(_F8), sc
+
+
+@mx_quant_jagged_rowwise_padded.register_fake
+def _(x, offs, mode):
+    rows, cols = x.shape
+    cap = _rows_cap(cols, offs.shape[0])
+    return x.new_empty((rows, cap), dtype=_F8), x.new_empty((rows * cap // 32,), dtype=torch.uint8)
+
+
+@torch.library.custom_op("mxq::mx_grouped_gemm_wgrad", mutates_args=())
+def mx_grouped_gemm_wgrad(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor, offs: torch.Tensor,
+                          tokens: int) -> torch.Tensor:
+    """MXFP8 weight-gradient grouped GEMM over each group's padded tokens:
+    (G, N, K) bf16 from the padded codes a (N, capacity), b (K, capacity)
+    and their blocked scales."""
+    out = torch.empty((offs.shape[0], a.shape[0], b.shape[0]), dtype=torch.bfloat16, device=a.device)
+    _b.mx_grouped_gemm_wgrad(a.view(torch.uint8), sfa, b.view(torch.uint8), sfb, offs, tokens, out=out)
+    return out
+
+
+@mx_grouped_gemm_wgrad.register_fake
+def _(a, sfa, b, sfb, offs, tokens):
+    return a.new_empty((offs.shape[0], a.shape[0], b.shape[0]), dtype=torch.bfloat16)
+
+
+@torch.library.custom_op("mxq::fp8_grouped_gemm_rowwise_wt", mutates_args=())
+def fp8_grouped_gemm_rowwise_wt(a: torch.Tensor, inv_a: torch.Tensor, wt: torch.Tensor, inv_w: torch.Tensor,
+                                offs: torch.Tensor) -> torch.Tensor:
+    """The FP8 grouped GEMM with every expert's weight given transposed side
+    by side, wt (K_w, E * N_w): (M, K_w) bf16; rows past offs[-1] are zero."""
+    out = torch.zeros((a.shape[0], wt.shape[0]), dtype=torch.bfloat16, device=a.device)
+    _b.fp8_grouped_gemm_rowwise_wt(a.view(torch.uint8), inv_a, wt.view(torch.uint8), inv_w, offs, out=out)
+    return out
+
+
+@fp8_grouped_gemm_rowwise_wt.register_fake
+def _(a, inv_a, wt, inv_w, offs):
+    return a.new_empty((a.shape[0], wt.shape[0]), dtype=torch.bfloat16)

@@ -12,7 +12,8 @@ from mxfp8_quantization_moe_device_b200 import synth
 OPS = ["fp8_quant_jagged_rowwise", "fp8_quant_jagged_colwise", "fp8_quant_blockwise",
        "fp8_quant_blockwise_transposed", "mx_quant_3d_colwise", "mx_quant_rowwise", "mx_scales_to_blocked_grouped",
        "mx_scales_to_blocked_grouped_k", "mx_quant_rowwise_blocked_grouped", "fp8_grouped_gemm_rowwise",
-       "fp8_grouped_gemm_wgrad", "mx_grouped_gemm"]
+       "fp8_grouped_gemm_wgrad", "mx_grouped_gemm", "mx_quant_jagged_colwise_padded", "mx_quant_jagged_rowwise_padded",
+       "mx_grouped_gemm_wgrad", "fp8_grouped_gemm_rowwise_wt"]
 
 
 def _cases(dev):
@@ -36,6 +37,8 @@ def _cases(dev):
         ("mx_scales_to_blocked_grouped", (s, offs_s)),
         ("mx_scales_to_blocked_grouped_k", (s, offs_k)),
         ("mx_quant_rowwise_blocked_grouped", (x, offs, "floor")),
+        ("mx_quant_jagged_colwise_padded", (x, offs, "rceil")),
+        ("mx_quant_jagged_rowwise_padded", (x.t(), offs, "floor")),
     ]
 
 
@@ -75,6 +78,19 @@ def test_wgrad_fake_shape_on_meta_tensors():
     assert tuple(out.shape) == (3, 256, 384) and out.dtype == torch.bfloat16
 
 
+def test_new_gemm_fake_shapes_on_meta_tensors():
+    a = torch.empty((256, 640), dtype=torch.float8_e4m3fn, device="meta")
+    b = torch.empty((384, 640), dtype=torch.float8_e4m3fn, device="meta")
+    sc = torch.empty((256 * 20,), dtype=torch.uint8, device="meta")
+    offs = torch.empty(4, dtype=torch.int32, device="meta")
+    out = torch.ops.mxq.mx_grouped_gemm_wgrad(a, sc, b, sc, offs, 300)
+    assert tuple(out.shape) == (4, 256, 384) and out.dtype == torch.bfloat16
+    wt = torch.empty((512, 4 * 256), dtype=torch.float8_e4m3fn, device="meta")
+    out = torch.ops.mxq.fp8_grouped_gemm_rowwise_wt(a[:, :256], torch.empty(256, device="meta"), wt,
+                                                    torch.empty((4, 512), device="meta"), offs)
+    assert tuple(out.shape) == (256, 512) and out.dtype == torch.bfloat16
+
+
 def test_fake_shapes_on_meta_tensors():
     want = {  # (shapes, dtypes) of each case's outputs
         0: ([(512, 256), (4, 512)], [torch.float8_e4m3fn, torch.float32]),
@@ -90,6 +106,9 @@ def test_fake_shapes_on_meta_tensors():
         10: ([(384 * 4 * ((7 + 9) // 4),), (3,)], [torch.uint8, torch.int32]),
         11: ([(256, 512), (128 * ((256 + 127 * 4) // 128) * 16,), (4,)],
              [torch.float8_e4m3fn, torch.uint8, torch.int32]),
+        # tokens padded per group: capacity 128 * floor((256 + 127 * 4) / 128) = 640
+        12: ([(512, 640), (512 * 640 // 32,)], [torch.float8_e4m3fn, torch.uint8]),
+        13: ([(512, 640), (512 * 640 // 32,)], [torch.float8_e4m3fn, torch.uint8]),
     }
     for i, (name, args) in enumerate(_cases("cpu")):
         out = getattr(torch.ops.mxq, name)(*[_meta(a) for a in args])
