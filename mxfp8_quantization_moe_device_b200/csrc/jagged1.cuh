@@ -18,8 +18,11 @@
 // exactly one strip; otherwise every block is a unit. A persistent
 // cooperative grid (one CTA per SM) takes units in ticket order
 // (strip-major): CTA c owns tickets c, c + grid, c + 2 grid...
-// Each CTA loads a unit once (TMA, 128 x 64 tiles) and keeps it in shared
-// memory until the amax of every group it touches is known:
+// Each CTA loads a unit (TMA, 128 x 64 tiles) into its amax ring, reduces
+// it and hands the slots straight back; once the amax of every group the
+// unit touches is known, a second producer loads the unit again into the
+// cast ring. The second load finds the tiles in L2: the units between their
+// two loads are a few tens of MB across the GPU. Group maxima:
 //   * a group that lies inside one unit is reduced locally;
 //   * a group spanning several units of the strip: every unit stores its
 //     64 partial maxima in a slot of its own (plain stores: units never
@@ -38,22 +41,22 @@
 // therefore completes (no deadlock) as long as all CTAs are resident, which
 // the cooperative launch guarantees.
 //
-// Warp roles in a CTA (480 threads):
-//   warps 0-7   cast: two quads, quad q takes the unit's tiles of parity q
-//               (at most two); one warp = 32 rows x 64 lines of a tile, a
-//               lane two lines. A quad copies its tiles into registers as
-//               soon as they land and hands the ring slots back, so the
-//               ring keeps loading while the unit waits for its scales;
-//               codes leave through a 128B-swizzled staging tile and a TMA
-//               store of the 64 x 128 transpose (plain stores for the tile
-//               that holds offs[G-1]).
-//   warps 8-11  amax: the same 32-row blocks, packed bf16 max, partial maxima
-//               per group merged in a per-unit shared table.
-//   warp 14     publisher: stores the unit's maxima of the groups it shares
-//               with other units in its global slots and counts them in.
-//   warp 12     merge: waits for the spanning groups' counters, turns amax
-//               into scales in the shared table, writes inverse scales.
-//   warp 13     producer: the TMA loads of the ring.
+// Warp roles in a CTA (512 threads):
+//   warps 0-7   cast: two quads, quad q takes the cast ring's tiles of
+//               parity q; one warp = 32 rows x 64 lines of a tile, a lane
+//               two lines; codes leave through a 128B-swizzled staging tile
+//               and a TMA store of the 64 x 128 transpose (plain stores for
+//               the tile that holds offs[G-1]).
+//   warps 8-9   amax: two 32-row blocks of every tile each, packed bf16 max,
+//               partial maxima per group merged in a per-unit shared table.
+//   warp 10     amax producer: the TMA loads of the amax ring.
+//   warp 11     cast producer: a unit's TMA loads into the cast ring, once
+//               its scales are ready.
+//   warps 12-15 publish and merge, unit ku on warp 12 + ku % 4 (so four
+//               units' exchanges overlap): store the maxima of the groups
+//               the unit shares with other units in their global slots and
+//               count them in; wait for those groups' counters, turn amax
+//               into scales in the shared table, write inverse scales.
 // Every wait is bounded by %globaltimer; on expiry the kernel records
 // MXQ_ERR_TIMEOUT, stops, and drains its own copies in flight.
 #pragma once
@@ -66,28 +69,33 @@ namespace jg1 {
 
 constexpr int TP = 128;       // positions per tile
 constexpr int TL = 64;        // lines per tile (one strip)
-constexpr int RING = 10;      // input tiles in shared memory (held or in flight)
+constexpr int RA = 7;         // amax ring (tiles)
+constexpr int RC = 4;         // cast ring (tiles; even: slot parity = quad)
 constexpr int MAX_UT = 4;     // tiles per unit (the host keeps units within this)
-constexpr int UQ = 8;         // units in flight (per-unit scale tables)
+constexpr int UQ = 4;         // units between their two loads (per-unit scale tables)
 constexpr int MAXG_U = 8;     // groups of a unit kept in the shared table
 constexpr int CAST_WARPS = 8;
-constexpr int AMAX_WARP0 = 8;
-constexpr int MERGE_WARP = 12;
-constexpr int PROD_WARP = 13;
-constexpr int PUB_WARP = 14;
-constexpr int THREADS = 15 * 32;
+constexpr int AMAX_WARP0 = 8;   // two amax warps
+constexpr int AMAX_WARPS = 2;
+constexpr int PROD_WARP = 10;
+constexpr int CPROD_WARP = 11;
+constexpr int PM_WARP0 = 12;    // four publish-and-merge warps, unit ku to warp ku % 4
+constexpr int PM_WARPS = 4;
+constexpr int THREADS = 16 * 32;
 constexpr int IN_BYTES = TP * TL * 2;  // 16 KB
 constexpr int OUT_BYTES = TP * TL;     // 8 KB
 
 struct __align__(1024) Smem {
-    uint8_t in[RING][IN_BYTES];
+    uint8_t in[RA][IN_BYTES];           // amax ring
+    uint8_t cin[RC][IN_BYTES];          // cast ring
     uint8_t out[2][2][OUT_BYTES];       // [quad][buffer]
     uint32_t tab[UQ][MAXG_U][TL];       // amax bits, then fp32 scale bits
-    uint32_t red[8][TL];                // merge warp: partial maxima of 8 slot subsets
-    uint64_t full[RING];
-    uint64_t empty[RING];
+    uint32_t red[PM_WARPS][8][TL];      // merge: partial maxima of 8 slot subsets, per warp
+    uint64_t full[RA];
+    uint64_t empty[RA];
+    uint64_t cfull[RC];
+    uint64_t cempty[RC];
     uint64_t amax_computed[UQ];
-    uint64_t amax_done[UQ];
     uint64_t scales_ready[UQ];
     uint64_t scales_free[UQ];
     int offs[jag::MAX_SEG];
@@ -157,13 +165,16 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
     const int ups = min(blocks, (int)gridDim.x); // units per strip (<= grid)
     const uint32_t total = (uint32_t)nstrips * (uint32_t)ups;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < RING; ++i) {
+        for (int i = 0; i < RA; ++i) {
             mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], 8); // 4 amax warps + the 4 warps of one cast quad
+            mbar_init(&sm.empty[i], AMAX_WARPS);
+        }
+        for (int i = 0; i < RC; ++i) {
+            mbar_init(&sm.cfull[i], 1);
+            mbar_init(&sm.cempty[i], 4); // the warps of one cast quad
         }
         for (int i = 0; i < UQ; ++i) {
             mbar_init(&sm.amax_computed[i], 1);
-            mbar_init(&sm.amax_done[i], 1);
             mbar_init(&sm.scales_ready[i], 1);
             mbar_init(&sm.scales_free[i], CAST_WARPS);
         }
@@ -184,16 +195,27 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
     __syncthreads();
     const int *soffs = sm.offs;
 
-    if (warp == PROD_WARP) {
-        // ------------------------------------------------------ producer
+    if (warp == PROD_WARP || warp == CPROD_WARP) {
+        // ------------------------------------------------------ producers
+        // amax producer: every unit's tiles, as slots free up; cast
+        // producer: a unit's tiles again once its scales are ready
+        const bool cast = warp == CPROD_WARP;
+        const int R = cast ? RC : RA;
+        uint8_t(*ring)[IN_BYTES] = cast ? sm.cin : sm.in;
+        uint64_t *fullb = cast ? sm.cfull : sm.full;
+        uint64_t *emptyb = cast ? sm.cempty : sm.empty;
         if (lane == 0) {
-            int i = 0;
+            int i = 0, ku = 0;
             bool stop = false;
-            for (uint32_t t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+            for (uint32_t t = blockIdx.x; t < total && !stop; t += gridDim.x, ++ku) {
                 const Unit u = unit_of(t, ups, blocks, end, soffs, G);
+                if (cast && !mbar_wait(&sm.scales_ready[ku % UQ], (uint32_t)(ku / UQ) & 1u, wait_ns)) {
+                    set_abort(sm);
+                    break;
+                }
                 for (int k = 0; k < u.ntiles; ++k, ++i) {
-                    const int slot = i % RING;
-                    if (i >= RING && !mbar_wait(&sm.empty[slot], ((uint32_t)(i / RING) & 1u) ^ 1u, wait_ns)) {
+                    const int slot = i % R;
+                    if (i >= R && !mbar_wait(&emptyb[slot], ((uint32_t)(i / R) & 1u) ^ 1u, wait_ns)) {
                         set_abort(sm);
                         stop = true;
                         break;
@@ -202,21 +224,21 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                         stop = true;
                         break;
                     }
-                    if (drop_load && blockIdx.x == 0 && i == 0)
+                    if (!cast && drop_load && blockIdx.x == 0 && i == 0)
                         continue; // test hook: this tile never arrives
-                    mbar_arrive_expect_tx(&sm.full[slot], IN_BYTES);
-                    tma_load_2d(sm.in[slot], &tm_in, &sm.full[slot], u.s * TL, u.r0 + k * TP);
+                    mbar_arrive_expect_tx(&fullb[slot], IN_BYTES);
+                    tma_load_2d(ring[slot], &tm_in, &fullb[slot], u.s * TL, u.r0 + k * TP);
                 }
             }
             // drain: every issued fill lands before the CTA exits
-            for (int j = i - RING; j < i; ++j)
-                if (j >= 0 && !(drop_load && blockIdx.x == 0 && j == 0))
-                    mbar_wait(&sm.full[j % RING], (uint32_t)(j / RING) & 1u, wait_ns);
+            for (int j = i - R; j < i; ++j)
+                if (j >= 0 && !(!cast && drop_load && blockIdx.x == 0 && j == 0))
+                    mbar_wait(&fullb[j % R], (uint32_t)(j / R) & 1u, wait_ns);
         }
         return;
     }
 
-    if (warp >= AMAX_WARP0 && warp < MERGE_WARP) {
+    if (warp >= AMAX_WARP0 && warp < AMAX_WARP0 + AMAX_WARPS) {
         // ------------------------------------------------------ amax warps
         const int aw = warp - AMAX_WARP0;
         int i = 0, ku = 0;
@@ -224,14 +246,14 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
             const Unit u = unit_of(t, ups, blocks, end, soffs, G);
             const int uq = ku % UQ;
             const bool ok = ku < UQ || mbar_wait(&sm.scales_free[uq], (uint32_t)(ku / UQ - 1) & 1u, wait_ns);
-            if (barrier_or(3, 4 * 32, !ok || abort_set(sm))) {
+            if (barrier_or(3, AMAX_WARPS * 32, !ok || abort_set(sm))) {
                 set_abort(sm);
                 break;
             }
             uint32_t *tab = &sm.tab[uq][0][0];
-            for (int x = aw * 32 + lane; x < MAXG_U * TL; x += 4 * 32)
+            for (int x = aw * 32 + lane; x < MAXG_U * TL; x += AMAX_WARPS * 32)
                 tab[x] = 0u;
-            named_barrier(3, 4 * 32);
+            named_barrier(3, AMAX_WARPS * 32);
             const int l0 = u.s * TL + 2 * lane;
             int g = u.gf;
             int gend = soffs[g];
@@ -252,15 +274,19 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                 acc = 0u;
             };
             for (int kt = 0; kt < u.ntiles; ++kt, ++i) {
-                const int slot = i % RING;
-                if (fail || !__all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (uint32_t)(i / RING) & 1u, wait_ns))) {
+                const int slot = i % RA;
+                if (fail || !__all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (uint32_t)(i / RA) & 1u, wait_ns))) {
                     fail = true; // stop at the end-of-unit barrier, together
                     continue;
                 }
-                const int row0 = u.r0 + kt * TP + 32 * aw;
-                const uint32_t *tile = reinterpret_cast<const uint32_t *>(sm.in[slot]) + (32 * aw) * (TL / 2) + lane;
                 uint32_t dep = 0u;
-                if (row0 < u.r1) {
+#pragma unroll 1
+                for (int bb = 0; bb < 4 / AMAX_WARPS; ++bb) {
+                    const int blk = (4 / AMAX_WARPS) * aw + bb; // 32-row block of the tile
+                    const int row0 = u.r0 + kt * TP + 32 * blk;
+                    const uint32_t *tile = reinterpret_cast<const uint32_t *>(sm.in[slot]) + (32 * blk) * (TL / 2) + lane;
+                    if (row0 >= u.r1)
+                        break;
                     const int nrows = min(32, u.r1 - row0);
                     if (row0 + nrows <= gend) {
                         if (nrows == 32) {
@@ -284,13 +310,13 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                             }
                             const int re = min(nrows, gend - row0);
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (i >= r && i < re)
-                                    acc = absmax_bf16x2(acc, tile[i * (TL / 2)]);
+                            for (int ii = 0; ii < 32; ++ii)
+                                if (ii >= r && ii < re)
+                                    acc = absmax_bf16x2(acc, tile[ii * (TL / 2)]);
                             r = re;
                         }
                     }
-                    dep = acc;
+                    dep ^= acc;
                 }
                 // these reads end before the slot's next TMA fill
                 release_slot_after(&sm.empty[slot], dep);
@@ -299,7 +325,7 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                 flush();
             if (__any_sync(0xffffffffu, spilled))
                 __threadfence(); // global atomics of spilled groups before the counters
-            if (barrier_or(3, 4 * 32, fail)) {
+            if (barrier_or(3, AMAX_WARPS * 32, fail)) {
                 set_abort(sm);
                 break;
             }
@@ -312,10 +338,13 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
         return;
     }
 
-    if (warp == PUB_WARP) {
-        // ------------------------------------------------------ publisher
+    if (warp >= PM_WARP0) {
+        // ---------------------------------------- publish and merge warps
+        const int pm = warp - PM_WARP0;
         int ku = 0;
         for (uint32_t t = blockIdx.x; t < total; t += gridDim.x, ++ku) {
+            if (ku % PM_WARPS != pm)
+                continue;
             const Unit u = unit_of(t, ups, blocks, end, soffs, G);
             const int uq = ku % UQ;
             const bool ok = mbar_wait(&sm.amax_computed[uq], (uint32_t)(ku / UQ) & 1u, wait_ns);
@@ -346,25 +375,6 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                         if (en > st && unit_of_pos(st, ups, blocks) != unit_of_pos(en - 1, ups, blocks))
                             red_release_gpu_add(counters + (int64_t)gg * nstrips + u.s, 1);
                     }
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.amax_done[uq]);
-            __syncwarp();
-        }
-        return;
-    }
-
-    if (warp == MERGE_WARP) {
-        // ------------------------------------------------------ merge warp
-        int ku = 0;
-        for (uint32_t t = blockIdx.x; t < total; t += gridDim.x, ++ku) {
-            const Unit u = unit_of(t, ups, blocks, end, soffs, G);
-            const int uq = ku % UQ;
-            bool ok = mbar_wait(&sm.amax_done[uq], (uint32_t)(ku / UQ) & 1u, wait_ns);
-            if (!__all_sync(0xffffffffu, ok) || abort_set(sm)) {
-                set_abort(sm);
-                break;
             }
             const int l0 = u.s * TL + 2 * lane;
             bool fail = false;
@@ -430,7 +440,7 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                     }
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4 *>(&sm.red[k][16 * qq + 4 * c]) =
+                        *reinterpret_cast<uint4 *>(&sm.red[pm][k][16 * qq + 4 * c]) =
                             make_uint4(m[4 * c], m[4 * c + 1], m[4 * c + 2], m[4 * c + 3]);
                     __syncwarp();
                     const unsigned *row = amax + (int64_t)gg * L;
@@ -438,8 +448,8 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                     a1 = l0 + 1 < L ? ld_relaxed_gpu(row + l0 + 1) : 0u;
 #pragma unroll
                     for (int x = 0; x < 8; ++x) {
-                        a0 = max(a0, sm.red[x][2 * lane]);
-                        a1 = max(a1, sm.red[x][2 * lane + 1]);
+                        a0 = max(a0, sm.red[pm][x][2 * lane]);
+                        a1 = max(a1, sm.red[pm][x][2 * lane + 1]);
                     }
                     __syncwarp();
                     if (slot >= MAXG_U) {
@@ -485,35 +495,12 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
     const int qbar = 1 + q;
     const bool store_thread = threadIdx.x == 128 * q;
     bool prev_stored = true;
-    int i0 = 0, ku = 0, nq = 0; // i0: ring sequence number of the unit's first tile
+    int i0 = 0, ku = 0, nq = 0; // i0: cast-ring sequence number of the unit's first tile
     for (uint32_t t = blockIdx.x; t < total; t += gridDim.x, ++ku) {
         const Unit u = unit_of(t, ups, blocks, end, soffs, G);
         const int uq = ku % UQ;
-        // this quad's tiles of the unit: kt0 and kt0 + 2 (units hold <= 4)
-        const int kt0 = (q - i0) & 1;
-        const int mine = u.ntiles > kt0 ? (u.ntiles - kt0 + 1) / 2 : 0;
-        uint32_t v[2][32];
-        bool fail = false;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            if (j < mine && !fail) {
-                const int i = i0 + kt0 + 2 * j, slot = i % RING;
-                if (__all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (uint32_t)(i / RING) & 1u, wait_ns))) {
-                    const uint32_t *tile = reinterpret_cast<const uint32_t *>(sm.in[slot]) + (w * 32) * (TL / 2) + lane;
-                    uint32_t dep = 0u;
-#pragma unroll
-                    for (int r = 0; r < 32; ++r) {
-                        v[j][r] = tile[r * (TL / 2)];
-                        dep ^= v[j][r];
-                    }
-                    release_slot_after(&sm.empty[slot], dep);
-                } else {
-                    fail = true;
-                }
-            }
-        }
-        const bool ok = fail || mbar_wait(&sm.scales_ready[uq], (uint32_t)(ku / UQ) & 1u, wait_ns);
-        if (barrier_or(qbar, 4 * 32, fail || !ok || abort_set(sm))) {
+        const bool ok = mbar_wait(&sm.scales_ready[uq], (uint32_t)(ku / UQ) & 1u, wait_ns);
+        if (barrier_or(qbar, 4 * 32, !ok || abort_set(sm))) {
             set_abort(sm);
             break;
         }
@@ -529,22 +516,34 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                 s1 = fp8_scale(__uint_as_float(l0 + 1 < L ? ld_relaxed_gpu(row + l0 + 1) : 0u));
             }
         };
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            if (j >= mine)
-                break;
+        bool fail = false;
+        for (int kt = (q - i0) & 1; kt < u.ntiles; kt += 2) {
+            const int i = i0 + kt, slot = i % RC;
             const int ob = nq & 1;
             ++nq;
-            const int tr0 = u.r0 + (kt0 + 2 * j) * TP; // the tile's first position
-            const int p0 = tr0 + 32 * w;                 // this warp's first position
-            uint32_t q0[8], q1[8]; // lines l0, l0+1: 32 position bytes each
+            // a failed wait is carried to the barrier below, where the quad
+            // stops together (the data read meanwhile is never stored)
+            fail = !__all_sync(0xffffffffu, mbar_wait(&sm.cfull[slot], (uint32_t)(i / RC) & 1u, wait_ns));
+            const uint32_t *tile = reinterpret_cast<const uint32_t *>(sm.cin[slot]) + (w * 32) * (TL / 2) + lane;
+            uint32_t v[32];
+            uint32_t dep = 0u;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                v[r] = tile[r * (TL / 2)];
+                dep ^= v[r];
+            }
+            if (!fail) // a slot whose fill never landed is not handed back
+                release_slot_after(&sm.cempty[slot], dep);
+            const int tr0 = u.r0 + kt * TP; // the tile's first position
+            const int p0 = tr0 + 32 * w;    // this warp's first position
+            uint32_t q0[8], q1[8];          // lines l0, l0+1: 32 position bytes each
             const int g = p0 < u.r1 ? jag::group_of(soffs, G, p0) : u.gl;
             if (p0 < u.r1 && soffs[g] >= p0 + 32) {
                 float s0, s1;
                 scales(g, s0, s1);
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
-                    const uint32_t *r = v[j] + 4 * jj;
+                    const uint32_t *r = v + 4 * jj;
                     q0[jj] = e4m3x2(__fmul_rn(bf16_lo(r[0]), s0), __fmul_rn(bf16_lo(r[1]), s0)) |
                              (e4m3x2(__fmul_rn(bf16_lo(r[2]), s0), __fmul_rn(bf16_lo(r[3]), s0)) << 16);
                     q1[jj] = e4m3x2(__fmul_rn(bf16_hi(r[0]), s1), __fmul_rn(bf16_hi(r[1]), s1)) |
@@ -570,11 +569,11 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                     float s0, s1;
                     scales(gg, s0, s1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i >= r && i < re) {
-                            const uint32_t x = v[j][i];
-                            q0[i >> 2] |= e4m3x2(__fmul_rn(bf16_lo(x), s0), 0.0f) << (8 * (i & 3));
-                            q1[i >> 2] |= e4m3x2(__fmul_rn(bf16_hi(x), s1), 0.0f) << (8 * (i & 3));
+                    for (int ii = 0; ii < 32; ++ii)
+                        if (ii >= r && ii < re) {
+                            const uint32_t x = v[ii];
+                            q0[ii >> 2] |= e4m3x2(__fmul_rn(bf16_lo(x), s0), 0.0f) << (8 * (ii & 3));
+                            q1[ii >> 2] |= e4m3x2(__fmul_rn(bf16_hi(x), s1), 0.0f) << (8 * (ii & 3));
                         }
                     r = re;
                 }
@@ -604,7 +603,7 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                     sts_v4(ob_addr + row * 128 + chunk * 16, val);
                 }
                 fence_proxy_async_smem();
-            } else {
+            } else if (!fail) {
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
                     const int l = l0 + bb;
@@ -619,12 +618,19 @@ __global__ void __launch_bounds__(jg1::THREADS, 1)
                     }
                 }
             }
-            named_barrier(qbar, 4 * 32);
+            if (barrier_or(qbar, 4 * 32, fail || abort_set(sm))) {
+                fail = true;
+                break;
+            }
             if (store_thread && full_tile) {
                 tma_store_2d(&tm_out, sm.out[q][ob], tr0, u.s * TL);
                 bulk_commit();
             }
             prev_stored = full_tile;
+        }
+        if (fail) {
+            set_abort(sm);
+            break;
         }
         __syncwarp();
         if (lane == 0)
