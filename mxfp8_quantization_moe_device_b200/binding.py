@@ -39,6 +39,8 @@ SIGNATURES = {
     "mx_quant_3d_colwise": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "fp8_grouped_gemm_rowwise": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
     "fp8_grouped_gemm_wgrad": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
+    "fp8_grouped_gemm_wgrad_ld": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i32, _vp,
+                                                 _vp]),
     "fp8_grouped_gemm_rowwise_strided": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _vp, _i32,
                                                         _vp, _vp]),
     "mx_grouped_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp]),
@@ -484,14 +486,17 @@ def fp8_grouped_gemm_wgrad(a, inv_a, b, inv_b, offs, *, out=None):
     g] . b[:, group g]^T) * inv_a[g][:, None] * inv_b[g][None, :]. a (N, M)
     and b (K, M) e4m3 with M contiguous (the buffers of
     fp8_quant_jagged_rowwise on grad_out^T and fp8_quant_jagged_colwise on the
-    input), inv_a (G, N), inv_b (G, K), offs (G,) ends along M. Returns out
-    (G, N, K) bf16."""
-    for t, n in ((a, "a"), (inv_a, "inv_a"), (b, "b"), (inv_b, "inv_b")):
+    input; row strides of at least M bytes, multiples of 16, e.g. column
+    slices [:, :M] of wider buffers), inv_a (G, N), inv_b (G, K), offs (G,)
+    ends along M. Returns out (G, N, K) bf16."""
+    for t, n in ((inv_a, "inv_a"), (inv_b, "inv_b")):
         _cuda(t, n)
         if not t.is_contiguous():
             raise TypeError(f"{n} must be contiguous")
-    if a.element_size() != 1 or b.element_size() != 1 or a.dim() != 2 or b.dim() != 2:
-        raise TypeError("a must be (N, M) and b (K, M), one byte per element (e4m3)")
+    for t, n in ((a, "a"), (b, "b")):
+        _cuda(t, n)
+        if t.dim() != 2 or t.element_size() != 1 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
+            raise TypeError(f"{n} must be a 2-D one-byte (e4m3) tensor with contiguous rows")
     if inv_a.dtype != torch.float32 or inv_b.dtype != torch.float32:
         raise TypeError("inv_a and inv_b must be float32")
     dev = a.device
@@ -503,7 +508,8 @@ def fp8_grouped_gemm_wgrad(a, inv_a, b, inv_b, offs, *, out=None):
         raise TypeError("shape mismatch between a, b, inv_a, inv_b and offs")
     if out is None:
         out = torch.empty((G, N, K), dtype=torch.bfloat16, device=dev)
-    _call("fp8_grouped_gemm_wgrad", dev, _ptr(a), _ptr(inv_a), _ptr(b), _ptr(inv_b), N, K, M, _ptr(offs), G, _ptr(out))
+    _call("fp8_grouped_gemm_wgrad_ld", dev, _ptr(a), _ptr(inv_a), _ptr(b), _ptr(inv_b), N, K, M, a.stride(0),
+          b.stride(0), _ptr(offs), G, _ptr(out))
     return out
 
 

@@ -310,34 +310,52 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
 // the MMA and the contraction of group g runs over its own positions.
 //
 // Same roles as above, on (group, n-tile, k-tile) items. The producer streams
-// 128-position chunks of the group starting at the 16-aligned position at or
-// below its first one (TMA coordinates must be 16-byte aligned); where a chunk
-// reaches outside the group, the MMA warp zeroes those position columns of
-// both tiles in shared memory (the bytes past the last group are not data),
-// fences the async proxy, and only then issues the MMAs. Items of empty
-// groups write zeros.
+// 128-position chunks of the group starting at the 128-aligned position at
+// or below its first one (so that every 128-byte row of a box is one L2
+// line: unaligned boxes read two lines per row and made the kernel L2
+// bound); where a chunk reaches outside the group, the MMA warp issues only
+// the K-32 slices that hold group positions, zeroes the bytes outside the
+// group within the two edge slices of both tiles in shared memory (the
+// bytes past the last group are not data), fences the async proxy, and
+// only then issues the MMAs. Items of empty groups write zeros.
 // ---------------------------------------------------------------------------
 namespace gm {
 
-// zero position columns outside [lo, hi) of a `rows` x 128-byte tile stored
-// with the 128-byte swizzle (byte c of row r at r*128 + ((c/16) ^ (r%8))*16 +
-// c%16); lane l of the warp takes rows l, l+32, ...
-MXQ_DEV void zero_outside(uint8_t *tile, int rows, int lo, int hi)
+// zero byte columns [b0, b1) (b1 - b0 <= 32) of a `rows` x 128-byte tile
+// stored with the 128-byte swizzle (byte c of row r at r*128 + ((c/16) ^
+// (r%8))*16 + c%16); lane l of the warp takes rows l, l+32, ... and every
+// 16-byte chunk the range touches: a whole chunk is stored as zeros, a
+// partial one is read, masked bytewise and written back
+MXQ_DEV void zero_cols(uint8_t *tile, int rows, int b0, int b1)
 {
+    if (b1 <= b0)
+        return;
     const int lane = threadIdx.x & 31;
+    const int c0 = b0 >> 4, c1 = (b1 - 1) >> 4; // the range's chunks (at most 3)
 #pragma unroll 1
-    for (int r = lane; r < rows; r += 32) {
-        uint8_t *row = tile + r * 128;
+    for (int c = c0; c <= c1; ++c) {
+        const int z0 = max(b0 - 16 * c, 0), z1 = min(b1 - 16 * c, 16); // bytes [z0, z1) of the chunk
+        uint32_t keep[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int a = min(max(z0 - 4 * w, 0), 4), b = min(max(z1 - 4 * w, 0), 4);
+            const uint32_t lo_m = a >= 4 ? 0xffffffffu : (1u << (8 * a)) - 1u; // bytes below a
+            const uint32_t hi_m = b >= 4 ? 0u : ~((1u << (8 * b)) - 1u);       // bytes from b on
+            keep[w] = lo_m | hi_m;
+        }
+        const bool whole = z0 == 0 && z1 == 16;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-            uint8_t *chunk = row + ((c ^ (r & 7)) << 4);
-            const int b0 = 16 * c, b1 = b0 + 16;
-            if (b1 <= lo || b0 >= hi) {
-                *reinterpret_cast<uint4 *>(chunk) = make_uint4(0u, 0u, 0u, 0u);
-            } else if (b0 < lo || b1 > hi) {
-                for (int j = 0; j < 16; ++j)
-                    if (b0 + j < lo || b0 + j >= hi)
-                        chunk[j] = 0;
+        for (int r = lane; r < rows; r += 32) {
+            uint4 *chunk = reinterpret_cast<uint4 *>(tile + r * 128 + ((c ^ (r & 7)) << 4));
+            if (whole) {
+                *chunk = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                uint4 v = *chunk;
+                v.x &= keep[0];
+                v.y &= keep[1];
+                v.z &= keep[2];
+                v.w &= keep[3];
+                *chunk = v;
             }
         }
     }
@@ -401,7 +419,7 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
         q.kt = rem - q.nt * ktn;
         q.s = q.g ? offs[q.g - 1] : 0;
         q.e = offs[q.g];
-        q.x0 = q.s & ~int64_t(15);
+        q.x0 = q.s & ~int64_t(BK - 1); // 128-byte aligned chunks: a box row is one L2 line
         q.nch = q.e > q.s ? (q.e - q.x0 + BK - 1) / BK : 0;
         return q;
     };
@@ -452,12 +470,19 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
                     break;
                 const int64_t c0 = q.x0 + j * BK;
                 const int lo = (int)max((int64_t)0, q.s - c0), hi = (int)min((int64_t)BK, q.e - c0);
-                if (lo > 0 || hi < BK) {
-                    // both tiles: positions past offs[G-1] were never written
-                    // by the quantization and may hold any byte, NaN codes
-                    // included, and 0 * NaN is NaN
-                    zero_outside(sm.a[s], BM, lo, hi);
-                    zero_outside(sm.b[s], BN, lo, hi);
+                // the K-32 slices holding some of the group's positions
+                // [lo, hi) of this chunk (never empty: the chunks span the
+                // group); slices wholly outside are not issued, and the
+                // bytes outside the group in the two edge slices are zeroed
+                // in both tiles: positions past offs[G-1] were never written
+                // by the quantization and may hold any byte, NaN codes
+                // included, and 0 * NaN is NaN
+                const int k_lo = lo >> 5, k_hi = (hi + 31) >> 5;
+                if ((lo & 31) || (hi & 31)) {
+                    zero_cols(sm.a[s], BM, 32 * k_lo, lo);
+                    zero_cols(sm.a[s], BM, hi, 32 * k_hi);
+                    zero_cols(sm.b[s], BN, 32 * k_lo, lo);
+                    zero_cols(sm.b[s], BN, hi, 32 * k_hi);
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
@@ -467,7 +492,8 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
                     const uint64_t bd = smem_desc_k128(smem_u32(sm.b[s]));
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k)
-                        tc_mma(d, ad + 2 * k, bd + 2 * k, IDESC, (j > 0 || k > 0) ? 1u : 0u);
+                        if (k >= k_lo && k < k_hi)
+                            tc_mma(d, ad + 2 * k, bd + 2 * k, IDESC, (j > 0 || k > k_lo) ? 1u : 0u);
                     tc_commit(&sm.empty[s]);
                 }
                 issued = true;

@@ -571,9 +571,9 @@ int mx_grouped_gemm(const void *a, const void *sfa, const void *w, const void *s
                   offs, (int)num_groups, static_cast<uint16_t *>(out), wait_ns());
 }
 
-int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, const float *inv_b, int64_t N,
-                           int64_t K, int64_t M, const int32_t *offs, int32_t num_groups, void *out,
-                           cudaStream_t stream)
+int fp8_grouped_gemm_wgrad_ld(const void *a, const float *inv_a, const void *b, const float *inv_b, int64_t N,
+                              int64_t K, int64_t M, int64_t lda, int64_t ldb, const int32_t *offs, int32_t num_groups,
+                              void *out, cudaStream_t stream)
 {
     if (M < 0 || N < 0 || K < 0 || num_groups < 1 || N % gm::BM || K % 128 || M % 16)
         return MXQ_ERR_SHAPE;
@@ -582,6 +582,8 @@ int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, con
     if (!a || !inv_a || !b || !inv_b || !offs || !out)
         return MXQ_ERR_NULL;
     if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(inv_a, 4) || !aligned(inv_b, 4))
+        return MXQ_ERR_ALIGN;
+    if (lda < M || ldb < M || lda % 16 || ldb % 16)
         return MXQ_ERR_ALIGN;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return MXQ_ERR_UNSUPPORTED;
@@ -593,14 +595,15 @@ int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, con
     CUtensorMap ta, tb;
     const uint64_t mm = (uint64_t)std::max<int64_t>(M, 16); // a map needs a non-zero extent
     const uint64_t da[2] = {mm, (uint64_t)N};
-    const uint64_t sa[1] = {mm};
+    const uint64_t sa[1] = {(uint64_t)std::max<int64_t>(lda, 16)};
     const uint32_t boxa[2] = {gm::BK, gm::BM};
     rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, boxa, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
     const uint64_t db[2] = {mm, (uint64_t)K};
+    const uint64_t sb[1] = {(uint64_t)std::max<int64_t>(ldb, 16)};
     const uint32_t boxb[2] = {gm::BK, (uint32_t)bn};
-    rc = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, db, sa, boxb, CU_TENSOR_MAP_SWIZZLE_128B);
+    rc = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, db, sb, boxb, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != MXQ_OK)
         return rc;
     const int64_t items = (int64_t)num_groups * (N / gm::BM) * (K / bn);
@@ -612,6 +615,13 @@ int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, con
     return launch(k_fp8_grouped_gemm_wgrad<128>, dim3((unsigned)grid), dim3(gm::THREADS), gm::smem_fixed<128>(),
                   stream, false, ta, tb, inv_a, inv_b, N, K, M, offs, (int)num_groups, static_cast<uint16_t *>(out),
                   wait_ns());
+}
+
+int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, const float *inv_b, int64_t N,
+                           int64_t K, int64_t M, const int32_t *offs, int32_t num_groups, void *out,
+                           cudaStream_t stream)
+{
+    return fp8_grouped_gemm_wgrad_ld(a, inv_a, b, inv_b, N, K, M, M, M, offs, num_groups, out, stream);
 }
 
 int mx_quant_3d_colwise(const void *in, int64_t E, int64_t N, int64_t K, int32_t mode, void *out, uint8_t *scales,
