@@ -247,9 +247,8 @@ int fp8_grouped_gemm_wgrad(const void *a, const float *inv_a, const void *b, con
 
 /* fp8_grouped_gemm_wgrad with the operands' row strides given (bytes): a
  * row n at a + n * lda, b row k at b + k * ldb; lda, ldb >= M and multiples
- * of 16 (MXQ_ERR_ALIGN otherwise). Rows a power of two bytes apart (M =
- * 65536 for example) load markedly slower than rows a few lines longer,
- * which the jagged ops' *_ld variants can write. */
+ * of 16 (MXQ_ERR_ALIGN otherwise), so that row-strided views (a slice of
+ * wider buffers, for example) are consumed in place. */
 int fp8_grouped_gemm_wgrad_ld(const void *a, const float *inv_a, const void *b, const float *inv_b,
                               int64_t N, int64_t K, int64_t M, int64_t lda, int64_t ldb,
                               const int32_t *offs, int32_t num_groups, void *out,

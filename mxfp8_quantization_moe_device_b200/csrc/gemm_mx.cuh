@@ -37,7 +37,14 @@ namespace mxq {
 namespace gmx {
 
 constexpr int BM = gm::BM, BK = gm::BK;
-constexpr int STAGES = gm::STAGES, THREADS = gm::THREADS;
+constexpr int STAGES = gm::STAGES;
+// warps 0-3 and 6-9 drain the accumulator (warp w reads TMEM lanes
+// 32 (w % 4) ..; warps 0-3 take the tile's first BN/2 columns, 6-9 the
+// rest), warp 4 loads, warp 5 issues: with one accumulator at BN 256 the
+// next tile's MMAs wait for the whole drain, which two warps per lane
+// quadrant halve
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (EPI_WARPS + 2) * 32;
 constexpr int A_BYTES = BM * BK;
 constexpr int SF_BYTES = 512;           // one 128 x 4 blocked scale tile
 constexpr int TMEM_COLS = 512;
@@ -133,7 +140,7 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
         }
         for (int i = 0; i < ACC; ++i) {
             mbar_init(&sm.acc_full[i], 1);
-            mbar_init(&sm.acc_empty[i], 4);
+            mbar_init(&sm.acc_empty[i], EPI_WARPS);
         }
         mbar_init(&sm.mma_done, 1);
         sm.abort_flag = 0;
@@ -210,22 +217,31 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
                 }
                 gm::tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BN);
-                bool ok = true;
-                for (int64_t kb = 0; kb < nkb; ++kb, ++seq) {
+                // the scales of stage `seq` into its slot's own TMEM columns,
+                // once the stage has landed (its slot's previous MMAs have
+                // then completed: the producer refilled the slot after them)
+                auto land_scales = [&](int sq) {
+                    const int ss = sq % STAGES;
+                    if (!mbar_wait(&sm.full[ss], (uint32_t)(sq / STAGES) & 1u, wait_ns))
+                        return false;
+                    gm::tc_fence_after();
+                    const uint32_t sft = tmem + (uint32_t)(SF_COL + ss * SF_STAGE_COLS);
+                    tc_cp_sf(sft, sf_desc(smem_u32(sm.sfa[ss])));
+#pragma unroll
+                    for (int h = 0; h < BN / 128; ++h) // W rows 128h.. of the tile: 4 columns each
+                        tc_cp_sf(sft + 4 + 4 * h, sf_desc(smem_u32(sm.sfb[ss] + h * SF_BYTES)));
+                    return true;
+                };
+                bool ok = land_scales(seq);
+                for (int64_t kb = 0; ok && kb < nkb; ++kb, ++seq) {
                     const int s = seq % STAGES;
-                    if (!mbar_wait(&sm.full[s], (uint32_t)(seq / STAGES) & 1u, wait_ns)) {
+                    // the next stage's scale copies go ahead of this stage's
+                    // MMAs, so that they are done before the MMAs that read them
+                    if (kb + 1 < nkb && !land_scales(seq + 1)) {
                         ok = false;
                         break;
                     }
-                    gm::tc_fence_after();
-                    // this stage's scales into its own TMEM columns; the copy and
-                    // the MMAs below run in issue order, and the columns are
-                    // rewritten only after this stage's MMAs have committed
                     const uint32_t sft = tmem + (uint32_t)(SF_COL + s * SF_STAGE_COLS);
-                    tc_cp_sf(sft, sf_desc(smem_u32(sm.sfa[s])));
-#pragma unroll
-                    for (int h = 0; h < BN / 128; ++h) // W rows 128h.. of the tile: 4 columns each
-                        tc_cp_sf(sft + 4 + 4 * h, sf_desc(smem_u32(sm.sfb[s] + h * SF_BYTES)));
                     const uint64_t ad = gm::smem_desc_k128(smem_u32(sm.a[s]));
                     const uint64_t bd = gm::smem_desc_k128(smem_u32(sm.b[s]));
 #pragma unroll
@@ -251,7 +267,8 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 0-3, TMEM lanes 32w..32w+31)
+        // ------------------------------------------------ epilogue (warps 0-3 and 6-9)
+        const int quad = warp & 3, c_begin = warp < 4 ? 0 : BN / 64; // TMEM lanes 32 quad.., 32-column chunks
         int t = 0;
         for (int64_t it = blockIdx.x; it < total; it += gridDim.x, ++t) {
             const int acc = t % ACC;
@@ -265,27 +282,30 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
             const int64_t mt = it / ntn, nt = it - mt * ntn;
             const int g = tile_group(mt);
             const int64_t gs = g ? offs[g - 1] : 0, ge = offs[g];
-            const int64_t m = gs + (mt - T[g]) * BM + 32 * warp + lane;
+            const int64_t m = gs + (mt - T[g]) * BM + 32 * quad + lane;
             const bool row_ok = m < ge;
-            uint16_t *dst = out + m * N + nt * BN;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                gm::tc_ld32(tmem + (uint32_t)(acc * BN + c * 32) + ((uint32_t)(32 * warp) << 16), r);
-                if (row_ok) {
-                    uint32_t pk[16];
+            uint16_t *dst = out + m * N + nt * BN + 32 * c_begin;
+            // the warp's half row into registers at once, the accumulator
+            // released, and only then the rounding and the stores: the next
+            // tile's MMAs wait for the TMEM reads alone
+            uint32_t r[BN / 2];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        pk[j] = gm::pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        st_v4(dst + c * 32 + 8 * j, pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-                }
-            }
+            for (int c = 0; c < BN / 64; ++c)
+                gm::tc_ld32_nowait(tmem + (uint32_t)(acc * BN + (c_begin + c) * 32) + ((uint32_t)(32 * quad) << 16),
+                                   r + 32 * c);
+            gm::tc_wait_ld();
             gm::tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sm.acc_empty[acc]);
+            if (row_ok) {
+#pragma unroll
+                for (int j = 0; j < BN / 16; ++j)
+                    st_v4(dst + 8 * j, gm::pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                          gm::pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                          gm::pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                          gm::pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
+            }
         }
     }
 

@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
         }
         for (int i = 0; i < ACC; ++i) {
             mbar_init(&sm.acc_full[i], 1);
-            mbar_init(&sm.acc_empty[i], 4);
+            mbar_init(&sm.acc_empty[i], EPI_WARPS);
         }
         mbar_init(&sm.mma_done, 1);
         sm.abort_flag = 0;
@@ -312,19 +312,28 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
                 }
                 gm::tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(acc * BN);
-                bool ok = true;
-                for (int j = 0; j < q.nch; ++j, ++seq) {
+                // scales of stage `sq` into its slot's TMEM columns once it has
+                // landed; the next stage's go ahead of this stage's MMAs
+                auto land_scales = [&](int sq) {
+                    const int ss = sq % STAGES;
+                    if (!mbar_wait(&sm.full[ss], (uint32_t)(sq / STAGES) & 1u, wait_ns))
+                        return false;
+                    gm::tc_fence_after();
+                    const uint32_t sft = tmem + (uint32_t)(SF_COL + ss * SF_STAGE_COLS);
+                    tc_cp_sf(sft, sf_desc(smem_u32(sm.sfa[ss])));
+#pragma unroll
+                    for (int h = 0; h < BN / 128; ++h)
+                        tc_cp_sf(sft + 4 + 4 * h, sf_desc(smem_u32(sm.sfb[ss] + h * SF_BYTES)));
+                    return true;
+                };
+                bool ok = land_scales(seq);
+                for (int j = 0; ok && j < q.nch; ++j, ++seq) {
                     const int s = seq % STAGES;
-                    if (!mbar_wait(&sm.full[s], (uint32_t)(seq / STAGES) & 1u, wait_ns)) {
+                    if (j + 1 < q.nch && !land_scales(seq + 1)) {
                         ok = false;
                         break;
                     }
-                    gm::tc_fence_after();
                     const uint32_t sft = tmem + (uint32_t)(SF_COL + s * SF_STAGE_COLS);
-                    tc_cp_sf(sft, sf_desc(smem_u32(sm.sfa[s])));
-#pragma unroll
-                    for (int h = 0; h < BN / 128; ++h)
-                        tc_cp_sf(sft + 4 + 4 * h, sf_desc(smem_u32(sm.sfb[s] + h * SF_BYTES)));
                     const uint64_t ad = gm::smem_desc_k128(smem_u32(sm.a[s]));
                     const uint64_t bd = gm::smem_desc_k128(smem_u32(sm.b[s]));
 #pragma unroll
@@ -349,14 +358,15 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (warps 0-3, TMEM lanes 32w..32w+31)
+        // ------------------------------------------------ epilogue (warps 0-3 and 6-9)
+        const int quad = warp & 3, c_begin = warp < 4 ? 0 : BN / 64; // TMEM lanes 32 quad.., 32-column chunks
         int t = 0;
         for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
             const Item q = item(it);
-            const int64_t n = q.nt * BM + 32 * warp + lane; // this thread's output row
+            const int64_t n = q.nt * BM + 32 * quad + lane; // this thread's output row
             uint16_t *dst = out + ((int64_t)q.g * N + n) * K + q.kt * BN;
             if (q.nch == 0) { // empty group: the sum is zero
-                for (int c = 0; c < BN; c += 8)
+                for (int c = 32 * c_begin; c < 32 * c_begin + BN / 2; c += 8)
                     st_v4(dst + c, 0u, 0u, 0u, 0u);
                 continue;
             }
@@ -368,22 +378,25 @@ __global__ void __launch_bounds__(gmx::THREADS, 1)
                 break;
             }
             gm::tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                gm::tc_ld32(tmem + (uint32_t)(acc * BN + c * 32) + ((uint32_t)(32 * warp) << 16), r);
-                uint32_t pk[16];
+            // the warp's half row into registers, the accumulator released,
+            // then the rounding and the stores (as in the forward MX GEMM)
+            uint32_t r[BN / 2];
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    pk[j] = gm::pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    st_v4(dst + c * 32 + 8 * j, pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            }
+            for (int c = 0; c < BN / 64; ++c)
+                gm::tc_ld32_nowait(tmem + (uint32_t)(acc * BN + (c_begin + c) * 32) + ((uint32_t)(32 * quad) << 16),
+                                   r + 32 * c);
+            gm::tc_wait_ld();
             gm::tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sm.acc_empty[acc]);
+            uint16_t *d0 = dst + 32 * c_begin;
+#pragma unroll
+            for (int j = 0; j < BN / 16; ++j)
+                st_v4(d0 + 8 * j, gm::pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                      gm::pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                      gm::pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                      gm::pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
             ++t;
         }
     }

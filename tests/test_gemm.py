@@ -145,6 +145,27 @@ def test_wgrad_gemm_vs_oracle(M, N, K, ends):
 
 
 
+@pytest.mark.parametrize("ends", [
+    [5, 37, 64, 96, 100, 228, 300, 1024],   # groups inside one K-32 slice, on slice edges, across chunks
+    [1024],
+])
+def test_wgrad_gemm_row_strided_operands(ends):
+    """Operands viewed out of wider buffers whose extra bytes hold NaN codes
+    (0xFF): the row-stride entry point gives the contiguous call's bits, and
+    both meet the oracle's bound."""
+    M, N, K = 1024, 128, 256
+    a, ia, b, ib, offs = _wgrad_operands(M, N, K, ends, seed=17)
+    want = mxq.fp8_grouped_gemm_wgrad(a, ia, b, ib, offs)
+    wa = torch.full((N, M + 272), 0xFF, dtype=torch.uint8, device=DEV)
+    wb = torch.full((K, M + 144), 0xFF, dtype=torch.uint8, device=DEV)
+    wa[:, :M] = a
+    wb[:, :M] = b
+    got = mxq.fp8_grouped_gemm_wgrad(wa[:, :M], ia, wb[:, :M], ib, offs)
+    assert mxq.device_status() == 0
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    _check_wgrad(got, a, ia, b, ib, offs)
+
+
 # ---------------------------------------------------------------- MXFP8 block-scaled
 
 def _mx_operands(M, N, K, E, ends, mode, seed):
