@@ -473,11 +473,17 @@ int mxq_version(void);
  *                              3 single-read kernel (cooperative launch).
  *   MXQ_TESTING_GEMM_TILE_N    mx_grouped_gemm (and mx_grouped_gemm_wgrad)
  *                              tile width: 0 automatic (256
- *                              when N % 256 == 0, else 128), 128 forced. */
+ *                              when N % 256 == 0, else 128), 128 forced.
+ *   MXQ_TESTING_BLOCKED_PATH   mx_scales_to_blocked_grouped(_k): 0
+ *                              automatic (the TMA ring kernels when the
+ *                              scale rows are a multiple of 16 bytes and
+ *                              at least one box wide, 128 bytes along rows
+ *                              and 144 along K), 1 the word-load kernels. */
 #define MXQ_TESTING_WAIT_LIMIT_NS 1
 #define MXQ_TESTING_SKIP_ARRIVAL 2
 #define MXQ_TESTING_FORCE_PATH 3
 #define MXQ_TESTING_GEMM_TILE_N 4
+#define MXQ_TESTING_BLOCKED_PATH 5
 int mxq_testing_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

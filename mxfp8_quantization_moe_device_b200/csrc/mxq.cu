@@ -12,6 +12,7 @@
 #include "jagged.cuh"
 #include "jagged1.cuh"
 #include "blocked.cuh"
+#include "blockedt.cuh"
 #include "gemm.cuh"
 #include "gemm_mx.cuh"
 #include "mxj.cuh"
@@ -24,6 +25,7 @@ std::atomic<int64_t> g_wait_ns{1000000000LL};
 std::atomic<int> g_drop_load{0};
 std::atomic<int> g_force_path{0};
 std::atomic<int> g_mx_bn{0}; // MX grouped GEMM tile width: 0 automatic, 128 forced
+std::atomic<int> g_blocked_words{0}; // blocked layouts: 1 forces the word-load kernels
 
 uint64_t wait_ns() { return (uint64_t)g_wait_ns.load(); }
 
@@ -125,7 +127,11 @@ int device_info(const DevInfo **out)
             cudaFuncSetAttribute(k_mx_grouped_gemm_wgrad<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(gmx::smem_fixed<128>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_mx_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(gmx::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess)
+                                 (int)(gmx::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_blocked_grouped_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(blkt::smem_fixed<blkt::R_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_blocked_grouped_k_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(blkt::smem_fixed<blkt::K_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess)
             return MXQ_ERR_CUDA;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.amx_per_sm, k_jagged_amax, jag::amx::THREADS, 0) !=
                 cudaSuccess ||
@@ -717,6 +723,26 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
     int rc = device_info(&di);
     if (rc != MXQ_OK)
         return rc;
+    if (rows > 0 && cols >= blkt::R_BOX_X && cols % 16 == 0 && aligned(scales, 16) && rows < (int64_t(1) << 31) &&
+        g_blocked_words.load() == 0) {
+        // TMA ring: rows of 16-byte multiples, at least one full box wide
+        CUtensorMap tm;
+        const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+        const uint64_t strides[1] = {(uint64_t)cols};
+        const uint32_t box[2] = {blkt::R_BOX_X, blkt::ROWS};
+        rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, scales, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc != MXQ_OK)
+            return rc;
+        const size_t smem = blkt::smem_fixed<blkt::R_STAGE>() + (size_t)num_groups * sizeof(int);
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_blocked_grouped_tma, blkt::THREADS, smem) !=
+            cudaSuccess)
+            return MXQ_ERR_CUDA;
+        const int64_t units = out_rows_capacity / 128 * ((tiles_c + blkt::TILES - 1) / blkt::TILES);
+        const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(units, (int64_t)di->sms * std::max(per_sm, 1)));
+        return launch(k_blocked_grouped_tma, dim3((unsigned)grid), dim3(blkt::THREADS), smem, stream, false, tm, rows,
+                      cols, offs, (int)num_groups, out, out_group_row_starts, out_rows_capacity / 128, wait_ns());
+    }
     const int64_t gx = std::max<int64_t>((tiles_c + blk::TILES - 1) / blk::TILES, 1);
     // enough CTAs to fill the GPU; each walks tile rows with stride gy
     const int64_t tile_rows = std::max<int64_t>(out_rows_capacity / 128, 1);
@@ -758,6 +784,26 @@ int mx_scales_to_blocked_grouped_k(const uint8_t *scales, int64_t rows, int64_t 
     if (rc != MXQ_OK)
         return rc;
     const int64_t tiles_c = out_cols_capacity / 4;
+    if (rows > 0 && cols >= blkt::K_BOX_X && cols % 16 == 0 && aligned(scales, 16) && cols < (int64_t(1) << 31) &&
+        g_blocked_words.load() == 0) {
+        // TMA ring: rows of 16-byte multiples, at least one box wide
+        CUtensorMap tm;
+        const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+        const uint64_t strides[1] = {(uint64_t)cols};
+        const uint32_t box[2] = {blkt::K_BOX_X, blkt::ROWS};
+        rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, scales, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc != MXQ_OK)
+            return rc;
+        const size_t smem = blkt::smem_fixed<blkt::K_STAGE>() + (size_t)num_groups * sizeof(int);
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_blocked_grouped_k_tma, blkt::THREADS, smem) !=
+            cudaSuccess)
+            return MXQ_ERR_CUDA;
+        const int64_t units = rows_p / 128 * ((tiles_c + blkt::TILES - 1) / blkt::TILES);
+        const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(units, (int64_t)di->sms * std::max(per_sm, 1)));
+        return launch(k_blocked_grouped_k_tma, dim3((unsigned)grid), dim3(blkt::THREADS), smem, stream, false, tm,
+                      rows, cols, offs, (int)num_groups, out, out_group_col_starts, out_cols_capacity, wait_ns());
+    }
     const int64_t gx = std::max<int64_t>((tiles_c + blk::TILES - 1) / blk::TILES, 1);
     const int64_t tile_rows = std::max<int64_t>(rows_p / 128, 1);
     const int64_t want = std::max<int64_t>((int64_t)di->sms * 8 / gx, 1);
@@ -1057,6 +1103,11 @@ int mxq_testing_set(int32_t what, int64_t value)
         if (value != 0 && value != 128)
             return MXQ_ERR_UNSUPPORTED;
         g_mx_bn.store((int)value);
+        return MXQ_OK;
+    case MXQ_TESTING_BLOCKED_PATH:
+        if (value != 0 && value != 1)
+            return MXQ_ERR_UNSUPPORTED;
+        g_blocked_words.store((int)value);
         return MXQ_OK;
     default: return MXQ_ERR_UNSUPPORTED;
     }

@@ -529,11 +529,23 @@ BLOCKED = [
     (1000, 33, [1, 2, 3, 500, 0, 494]),
     (64, 224, [64]),
     (4096, 300, [4000, 96]),
+    # rows of 16-byte multiples: the TMA ring kernel unless the word-load
+    # kernel is forced
+    (1000, 160, [1, 2, 3, 500, 0, 494]),  # a partial second column chunk, one-row groups
+    (700, 128, [0, 0, 129, 129, 300]),    # leading and inner empty groups, rows past the last group
+    (2000, 256, [128, 256, 1000, 616]),   # groups on tile boundaries
 ]
 
 
+@pytest.fixture(params=[0, 1], ids=["auto", "words"])
+def blocked_path(request):
+    mxq.testing_set(mxq.TESTING_BLOCKED_PATH, request.param)
+    yield request.param
+    mxq.testing_set(mxq.TESTING_BLOCKED_PATH, 0)
+
+
 @pytest.mark.parametrize("rows,cols,sizes", BLOCKED)
-def test_blocked_grouped_vs_oracle(rows, cols, sizes):
+def test_blocked_grouped_vs_oracle(rows, cols, sizes, blocked_path):
     s = synth.uniform_u8((rows, cols), 0, 254, seed=rows + cols)
     offs = torch.tensor(np.cumsum(sizes), dtype=torch.int32)
     ref, ref_starts = oracle.mx_scales_to_blocked_grouped(s.numpy(), offs.numpy())
@@ -548,7 +560,7 @@ def test_blocked_grouped_vs_oracle(rows, cols, sizes):
 
 @pytest.mark.parametrize("R,C", [(65536, 224), (8192, 512), (5120, 1024), (7168, 2048), (2048, 32768),
                                  (8192, 4096)])
-def test_blocked_grouped_config_shapes(R, C):
+def test_blocked_grouped_config_shapes(R, C, blocked_path):
     """The MX activation scales (65536, 224) with G=64 Dirichlet(0.3) groups and
     the scale-sweep shapes with G=8 Dirichlet(1.0) groups."""
     if (R, C) == (65536, 224):
@@ -571,11 +583,17 @@ BLOCKED_K = [
     (64, 40, [30]),                      # columns past the last group
     (1000, 600, [131, 1, 200, 268]),     # several 32-tile chunks per row tile
     (257, 4, [4]),
+    # rows of 16-byte multiples, at least 144 bytes: the TMA ring kernel
+    # unless the word-load kernel is forced
+    (1000, 608, [131, 1, 200, 276]),     # chunks starting at every byte phase
+    (300, 144, [1, 2, 3, 4, 5, 6, 7, 116]),
+    (129, 512, [0, 17, 0, 255, 240]),    # empty groups, a group of 1 tile column
+    (64, 160, [30]),                     # columns past the last group
 ]
 
 
 @pytest.mark.parametrize("rows,cols,sizes", BLOCKED_K)
-def test_blocked_grouped_k_vs_oracle(rows, cols, sizes):
+def test_blocked_grouped_k_vs_oracle(rows, cols, sizes, blocked_path):
     s = synth.uniform_u8((rows, cols), 0, 254, seed=rows * 3 + cols)
     offs = torch.tensor(np.cumsum(sizes), dtype=torch.int32)
     ref, ref_starts = oracle.mx_scales_to_blocked_grouped_k(s.numpy(), offs.numpy())
@@ -591,7 +609,7 @@ def test_blocked_grouped_k_vs_oracle(rows, cols, sizes):
 
 
 @pytest.mark.parametrize("R,C", [(8192, 512), (2048, 32768), (5120, 4096)])
-def test_blocked_grouped_k_sweep_shapes(R, C):
+def test_blocked_grouped_k_sweep_shapes(R, C, blocked_path):
     """The pages' scale-sweep shapes with G=8 Dirichlet(1.0) groups along K,
     capacity C + 4G (their byte count)."""
     s, offs = synth.scale_sweep_k(R, C)
