@@ -443,14 +443,67 @@ def flush_l2_clean(torch, buf, sink):
     torch.sum(buf.view(torch.int64), dim=0, out=sink)
 
 
+GRAPH_BELOW_BYTES = 512 << 20  # shapes timed again inside a CUDA graph
+
+
+def graph_us(torch, fn, flush, calls=10, reps=5):
+    """Device time per call of `fn` with the per-launch host and event
+    overhead amortised away (about 5 us on B200 for a single timed call):
+    two CUDA graphs, one of `calls` x (clean L2 flush, fn) and one of `calls`
+    x (clean L2 flush) alone, each replayed `reps` times; the median
+    difference divided by `calls`. The L2 is cold and clean before every
+    call, as for "us_clean". None if the call cannot be captured."""
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                fn()
+                flush()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graphs = []
+        for with_fn in (True, False):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(calls):
+                    flush()
+                    if with_fn:
+                        fn()
+            g.replay()
+            graphs.append(g)
+        torch.cuda.synchronize()
+        diffs = []
+        for _ in range(reps):
+            t = []
+            for g in graphs:
+                torch.cuda._sleep(200000)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                t.append(a.elapsed_time(b) * 1e3)
+            diffs.append((t[0] - t[1]) / calls)
+        del graphs
+        return round(statistics.median(diffs), 3)
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+
+
 def per_shape_sweep(wl, reps):
     """us/call and GB/s per config shape after 5 warm-up calls: the median of
     `reps` calls with the L2 flushed (256 MB write) before each ("us"); the
     median of `reps` calls after the same write followed by a read of the
     flush buffer, so that the L2 is cold but holds no dirty lines the call
     would first have to write back ("us_clean"); the median of `reps`
-    back-to-back calls with a hot L2 ("us_hot", labelled as such); and the
-    median host time to enqueue one call ("enqueue_us")."""
+    back-to-back calls with a hot L2 ("us_hot", labelled as such); the
+    median host time to enqueue one call ("enqueue_us"); and, for shapes
+    under 512 MB, the per-call device time from CUDA graphs with a clean L2
+    flush before every call ("us_graph", see graph_us), which a single timed
+    call overstates by the launch and event overhead (about 5 us on B200)."""
     torch, mxq = wl.torch, wl.mxq
     from mxfp8_quantization_moe_device_b200 import synth
     dev = wl.dev
@@ -487,10 +540,15 @@ def per_shape_sweep(wl, reps):
         us = statistics.median(ts)
         gbs = nbytes / (us * 1e-6) / 1e9
         usc = statistics.median(clean)
-        rows.append({"op": name, "shape": shape, "us": round(us, 3), "GB/s": round(gbs, 1),
-                     "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4),
-                     "us_clean": round(usc, 3), "frac_measured_clean": round(nbytes / (usc * 1e-6) / 1e9 / peak, 4),
-                     "us_hot": round(statistics.median(hot), 3), "enqueue_us": round(statistics.median(enq), 1)})
+        row = {"op": name, "shape": shape, "us": round(us, 3), "GB/s": round(gbs, 1),
+               "frac_measured": round(gbs / peak, 4), "frac_8TBs": round(gbs / 8000.0, 4),
+               "us_clean": round(usc, 3), "frac_measured_clean": round(nbytes / (usc * 1e-6) / 1e9 / peak, 4),
+               "us_hot": round(statistics.median(hot), 3), "enqueue_us": round(statistics.median(enq), 1)}
+        if nbytes < GRAPH_BELOW_BYTES:
+            row["us_graph"] = graph_us(torch, fn, lambda: flush_l2_clean(torch, flush, sink))
+            if row["us_graph"]:
+                row["frac_measured_graph"] = round(nbytes / (row["us_graph"] * 1e-6) / 1e9 / peak, 4)
+        rows.append(row)
 
     run.rows = rows
 

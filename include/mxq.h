@@ -478,12 +478,17 @@ int mxq_version(void);
  *                              automatic (the TMA ring kernels when the
  *                              scale rows are a multiple of 16 bytes and
  *                              at least one box wide, 128 bytes along rows
- *                              and 144 along K), 1 the word-load kernels. */
+ *                              and 144 along K), 1 the word-load kernels.
+ *   MXQ_TESTING_GEMM_ONE_SM    fp8_grouped_gemm_wgrad(_ld): 0 automatic
+ *                              (CTA pairs with 256 x 256 tiles when N and
+ *                              K are multiples of 256), 1 the one-SM
+ *                              kernel. */
 #define MXQ_TESTING_WAIT_LIMIT_NS 1
 #define MXQ_TESTING_SKIP_ARRIVAL 2
 #define MXQ_TESTING_FORCE_PATH 3
 #define MXQ_TESTING_GEMM_TILE_N 4
 #define MXQ_TESTING_BLOCKED_PATH 5
+#define MXQ_TESTING_GEMM_ONE_SM 6
 int mxq_testing_set(int32_t what, int64_t value);
 
 #ifdef __cplusplus

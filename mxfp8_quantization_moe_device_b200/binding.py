@@ -20,6 +20,7 @@ ERR_BAD_OFFSETS, ERR_TIMEOUT, ERR_WORKSPACE, ERR_CUDA = 6, 7, 8, 9
 FLOOR, RCEIL = 0, 1
 TESTING_WAIT_LIMIT_NS, TESTING_SKIP_ARRIVAL, TESTING_FORCE_PATH, TESTING_GEMM_TILE_N = 1, 2, 3, 4
 TESTING_BLOCKED_PATH = 5
+TESTING_GEMM_ONE_SM = 6
 
 _lib = None
 

@@ -550,17 +550,30 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
             }
             tc_fence_after();
             const float sa = __ldg(inv_a + (int64_t)q.g * N + n);
+            // the tile's column scales, one per lane and 32-column chunk
+            // (one coalesced load per chunk), handed to the row-owning
+            // lanes by shuffles: per-element loads of a scale every lane
+            // shares would queue in the load/store unit
             const float *sb = inv_b + (int64_t)q.g * K + q.kt * BN;
+            float sbl[BN / 32];
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+                sbl[c] = __ldg(sb + c * 32 + lane);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tc_ld32(tmem + (uint32_t)(acc * BN + c * 32) + ((uint32_t)(32 * warp) << 16), r);
+                float cs = sbl[0];
+#pragma unroll
+                for (int cc = 1; cc < BN / 32; ++cc)
+                    cs = c == cc ? sbl[cc] : cs;
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(r[2 * j]), sa), __ldg(sb + c * 32 + 2 * j));
+                    const float v0 =
+                        __fmul_rn(__fmul_rn(__uint_as_float(r[2 * j]), sa), __shfl_sync(0xffffffffu, cs, 2 * j));
                     const float v1 =
-                        __fmul_rn(__fmul_rn(__uint_as_float(r[2 * j + 1]), sa), __ldg(sb + c * 32 + 2 * j + 1));
+                        __fmul_rn(__fmul_rn(__uint_as_float(r[2 * j + 1]), sa), __shfl_sync(0xffffffffu, cs, 2 * j + 1));
                     pk[j] = pack_bf16x2(v0, v1);
                 }
 #pragma unroll

@@ -15,6 +15,7 @@
 #include "blockedt.cuh"
 #include "gemm.cuh"
 #include "gemm_mx.cuh"
+#include "gemm2.cuh"
 #include "mxj.cuh"
 
 using namespace mxq;
@@ -26,6 +27,7 @@ std::atomic<int> g_drop_load{0};
 std::atomic<int> g_force_path{0};
 std::atomic<int> g_mx_bn{0}; // MX grouped GEMM tile width: 0 automatic, 128 forced
 std::atomic<int> g_blocked_words{0}; // blocked layouts: 1 forces the word-load kernels
+std::atomic<int> g_gemm_one_sm{0};   // weight-gradient GEMM: 1 forces the one-SM kernel
 
 uint64_t wait_ns() { return (uint64_t)g_wait_ns.load(); }
 
@@ -82,6 +84,7 @@ struct DevInfo {
     int cst_per_sm = 0;   // resident CTAs of the jagged cast pass
     int sg_per_sm = 0;    // resident CTAs of the single-read jagged kernel
     int rb_per_sm = 0;    // resident CTAs of the 1x128 kernel
+    int wg2_pairs = 0;    // co-resident CTA pairs of the pair weight-gradient GEMM
     int mx32_per_sm = 0;  // resident CTAs of the 1x32 kernel
     int mxb_per_sm = 0;   // resident CTAs of the 1x32 kernel with blocked scales
     int mxj_per_sm = 0;   // resident CTAs of the padded MX jagged kernel (at MAX_G groups)
@@ -89,6 +92,28 @@ struct DevInfo {
 
 DevInfo g_dev[128];
 std::mutex g_dev_mu;
+
+// co-resident clusters of two for a kernel with `smem` dynamic bytes
+template <typename... K>
+int max_pairs(void (*kernel)(K...), dim3 block, size_t smem, int *pairs)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(pairs, (void *)kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+}
 
 int device_info(const DevInfo **out)
 {
@@ -131,7 +156,11 @@ int device_info(const DevInfo **out)
             cudaFuncSetAttribute(k_blocked_grouped_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(blkt::smem_fixed<blkt::R_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_blocked_grouped_k_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(blkt::smem_fixed<blkt::K_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess)
+                                 (int)(blkt::smem_fixed<blkt::K_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+            cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)g2::SMEM_BYTES) != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        if (max_pairs(k_fp8_grouped_gemm_wgrad_2sm, dim3(g2::THREADS), g2::SMEM_BYTES, &di.wg2_pairs) != MXQ_OK)
             return MXQ_ERR_CUDA;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&di.amx_per_sm, k_jagged_amax, jag::amx::THREADS, 0) !=
                 cudaSuccess ||
@@ -176,6 +205,31 @@ int launch(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_
     }
     return MXQ_OK;
 }
+
+// launch in clusters of two CTAs along x (grid.x even)
+template <typename... K, typename... A>
+int launch_pairs(void (*kernel)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, A &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MXQ_ERR_LAUNCH;
+    }
+    return MXQ_OK;
+}
+
 
 // ------------------------------------------------------------ jagged plan
 struct JaggedPlan {
@@ -600,6 +654,25 @@ int fp8_grouped_gemm_wgrad_ld(const void *a, const float *inv_a, const void *b, 
     const int bn = K % 256 == 0 ? 256 : 128;
     CUtensorMap ta, tb;
     const uint64_t mm = (uint64_t)std::max<int64_t>(M, 16); // a map needs a non-zero extent
+    if (N % g2::BM == 0 && K % g2::BN == 0 && di->wg2_pairs > 0 && g_gemm_one_sm.load() == 0) {
+        // CTA pairs: 256 x 256 tiles, each CTA loading 128 rows of a and of b
+        const uint64_t da[2] = {mm, (uint64_t)N};
+        const uint64_t sa[1] = {(uint64_t)std::max<int64_t>(lda, 16)};
+        const uint32_t box[2] = {g2::BK, g2::HALF};
+        rc = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a, da, sa, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc != MXQ_OK)
+            return rc;
+        const uint64_t db[2] = {mm, (uint64_t)K};
+        const uint64_t sb[1] = {(uint64_t)std::max<int64_t>(ldb, 16)};
+        rc = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, b, db, sb, box, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (rc != MXQ_OK)
+            return rc;
+        const int64_t items = (int64_t)num_groups * (N / g2::BM) * (K / g2::BN);
+        const int64_t pairs = std::max<int64_t>(1, std::min<int64_t>(items, di->wg2_pairs));
+        return launch_pairs(k_fp8_grouped_gemm_wgrad_2sm, dim3((unsigned)(2 * pairs)), dim3(g2::THREADS),
+                            g2::SMEM_BYTES, stream, ta, tb, inv_a, inv_b, N, K, M, offs, (int)num_groups,
+                            static_cast<uint16_t *>(out), wait_ns());
+    }
     const uint64_t da[2] = {mm, (uint64_t)N};
     const uint64_t sa[1] = {(uint64_t)std::max<int64_t>(lda, 16)};
     const uint32_t boxa[2] = {gm::BK, gm::BM};
@@ -1108,6 +1181,11 @@ int mxq_testing_set(int32_t what, int64_t value)
         if (value != 0 && value != 1)
             return MXQ_ERR_UNSUPPORTED;
         g_blocked_words.store((int)value);
+        return MXQ_OK;
+    case MXQ_TESTING_GEMM_ONE_SM:
+        if (value != 0 && value != 1)
+            return MXQ_ERR_UNSUPPORTED;
+        g_gemm_one_sm.store((int)value);
         return MXQ_OK;
     default: return MXQ_ERR_UNSUPPORTED;
     }

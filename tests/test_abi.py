@@ -147,8 +147,9 @@ def test_testing_hooks_accept_only_their_documented_values(lib):
     assert lib.mxq_testing_set(binding.TESTING_FORCE_PATH, -1) == binding.ERR_UNSUPPORTED
     assert lib.mxq_testing_set(binding.TESTING_GEMM_TILE_N, 64) == binding.ERR_UNSUPPORTED
     assert lib.mxq_testing_set(binding.TESTING_BLOCKED_PATH, 2) == binding.ERR_UNSUPPORTED
+    assert lib.mxq_testing_set(binding.TESTING_GEMM_ONE_SM, 2) == binding.ERR_UNSUPPORTED
     for hook, value in ((binding.TESTING_FORCE_PATH, 2), (binding.TESTING_FORCE_PATH, 3),
-                        (binding.TESTING_GEMM_TILE_N, 128), (binding.TESTING_BLOCKED_PATH, 1),
+                        (binding.TESTING_GEMM_TILE_N, 128), (binding.TESTING_BLOCKED_PATH, 1), (binding.TESTING_GEMM_ONE_SM, 1),
                         (binding.TESTING_WAIT_LIMIT_NS, 5_000_000), (binding.TESTING_SKIP_ARRIVAL, 1)):
         assert lib.mxq_testing_set(hook, value) == binding.OK
         assert lib.mxq_testing_set(hook, 0) == binding.OK

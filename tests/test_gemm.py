@@ -145,6 +145,27 @@ def test_wgrad_gemm_vs_oracle(M, N, K, ends):
 
 
 
+@pytest.mark.parametrize("one_sm", [0, 1], ids=["pairs", "one_sm"])
+@pytest.mark.parametrize("M,N,K,ends", [
+    (1008, 256, 256, [3, 250, 251, 700, 992]),          # unaligned starts and ends, a one-row group, tail positions
+    (4096, 512, 512, [0, 1000, 1016, 3000, 4096]),      # an empty first group, several pair tiles
+    (2048, 256, 768, [5, 37, 64, 96, 100, 228, 2048]),  # groups inside one K-32 slice and on slice edges
+])
+def test_wgrad_gemm_pair_tiles_vs_oracle(M, N, K, ends, one_sm):
+    """N and K multiples of 256: the CTA-pair kernel (256 x 256 tiles,
+    tcgen05 cta_group::2), and the one-SM kernel forced on the same data."""
+    a, ia, b, ib, offs = _wgrad_operands(M, N, K, ends, seed=M + N + K)
+    mxq.testing_set(mxq.TESTING_GEMM_ONE_SM, one_sm)
+    try:
+        out = mxq.fp8_grouped_gemm_wgrad(a, ia, b, ib, offs)
+    finally:
+        mxq.testing_set(mxq.TESTING_GEMM_ONE_SM, 0)
+    assert mxq.device_status() == 0
+    _check_wgrad(out, a, ia, b, ib, offs)
+    if ends[0] == 0:
+        assert bool((out[0] == 0).all())
+
+
 @pytest.mark.parametrize("ends", [
     [5, 37, 64, 96, 100, 228, 300, 1024],   # groups inside one K-32 slice, on slice edges, across chunks
     [1024],
