@@ -32,9 +32,9 @@
 //   epilogue (both)  drains its own 128 TMEM lanes x 256 columns, scales,
 //                    rounds, stores, and arrives on the leader's
 //                    accumulator-empty barrier (count 8).
-// No TMA load uses cluster multicast. Every wait is bounded; a CTA that
-// gives up records MXQ_ERR_TIMEOUT and stops its roles, and both meet at
-// the closing cluster barrier before TMEM is freed.
+// Every TMA load fills the loading CTA's own shared memory. Every wait is
+// bounded; a CTA that gives up records MXQ_ERR_TIMEOUT and stops its roles,
+// and both meet at the closing cluster barrier before TMEM is freed.
 #pragma once
 
 #include "gemm.cuh"
