@@ -73,10 +73,11 @@ MXQ_DEV uint32_t lds32(uint32_t addr)
     return v;
 }
 
-// barrier init, padded starts into T (dynamic smem after the fixed part),
-// and the group starts of CTA 0; false on bad offsets
+// barrier init, padded starts into T and the offsets into so (dynamic
+// shared memory after the fixed part: the per-unit group lookups then touch
+// no global memory), and the group starts of CTA 0; false on bad offsets
 template <int STAGE_BYTES>
-MXQ_DEV bool setup(Smem<STAGE_BYTES> &sm, int *T, const int32_t *offs, int G, int64_t extent, int shift,
+MXQ_DEV bool setup(Smem<STAGE_BYTES> &sm, int *T, int *so, const int32_t *offs, int G, int64_t extent, int shift,
                    int32_t *starts_out, int start_mul)
 {
     if (threadIdx.x == 0) {
@@ -89,6 +90,9 @@ MXQ_DEV bool setup(Smem<STAGE_BYTES> &sm, int *T, const int32_t *offs, int G, in
     }
     if (!padded_starts(offs, G, extent, shift, T, &sm.Tend))
         return false;
+    for (int g = threadIdx.x; g < G; g += blockDim.x)
+        so[g] = offs[g];
+    __syncthreads();
     if (blockIdx.x == 0 && starts_out)
         for (int g = threadIdx.x; g < G; g += blockDim.x)
             starts_out[g] = T[g] * start_mul;
@@ -127,8 +131,8 @@ __global__ void __launch_bounds__(blkt::THREADS) k_blocked_grouped_tma(const __g
     using SM = Smem<R_STAGE>;
     extern __shared__ uint8_t smem_raw[];
     SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int *T = reinterpret_cast<int *>(&sm + 1);
-    if (!setup(sm, T, offs, G, rows, 7, starts_out, 128))
+    int *T = reinterpret_cast<int *>(&sm + 1), *so = T + G;
+    if (!setup(sm, T, so, offs, G, rows, 7, starts_out, 128))
         return;
     const int Tend = sm.Tend;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,7 +149,7 @@ __global__ void __launch_bounds__(blkt::THREADS) k_blocked_grouped_tma(const __g
                 const int64_t rt = u / nch, ch = u - rt * nch;
                 if (rt < Tend) {
                     const int g = owner(T, G, rt);
-                    const int64_t src0 = (g ? offs[g - 1] : 0) + (rt - T[g]) * ROWS;
+                    const int64_t src0 = (g ? so[g - 1] : 0) + (rt - T[g]) * ROWS;
                     mbar_arrive_expect_tx(&sm.full[s], R_STAGE);
                     tma_load_2d(sm.in[s], &tm_in, &sm.full[s], (int)(ch * R_BOX_X), (int)src0);
                 } else {
@@ -166,8 +170,8 @@ __global__ void __launch_bounds__(blkt::THREADS) k_blocked_grouped_tma(const __g
         int nvalid = 0;
         if (rt < Tend) {
             const int g = owner(T, G, rt);
-            const int64_t src0 = (g ? offs[g - 1] : 0) + (rt - T[g]) * ROWS;
-            nvalid = (int)min((int64_t)ROWS, (int64_t)offs[g] - src0);
+            const int64_t src0 = (g ? so[g - 1] : 0) + (rt - T[g]) * ROWS;
+            nvalid = (int)min((int64_t)ROWS, (int64_t)so[g] - src0);
         }
         const int ntiles = (int)min((int64_t)TILES, tiles_c - ch * TILES);
         bool ok = mbar_wait(&sm.full[s], (uint32_t)(it / STAGES) & 1u, wait_ns);
@@ -214,8 +218,8 @@ __global__ void __launch_bounds__(blkt::THREADS) k_blocked_grouped_k_tma(const _
     using SM = Smem<K_STAGE>;
     extern __shared__ uint8_t smem_raw[];
     SM &sm = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int *T = reinterpret_cast<int *>(&sm + 1);
-    if (!setup(sm, T, offs, G, cols, 2, starts_out, 4))
+    int *T = reinterpret_cast<int *>(&sm + 1), *so = T + G;
+    if (!setup(sm, T, so, offs, G, cols, 2, starts_out, 4))
         return;
     const int Tend = sm.Tend;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -225,9 +229,9 @@ __global__ void __launch_bounds__(blkt::THREADS) k_blocked_grouped_k_tma(const _
     // source byte of output tile column tc (< Tend) and the bytes it holds
     auto column = [&](int64_t tc, int64_t &src, int &nv) {
         const int g = owner(T, G, tc);
-        const int64_t gs = g ? offs[g - 1] : 0;
+        const int64_t gs = g ? so[g - 1] : 0;
         src = gs + (tc - T[g]) * 4;
-        nv = (int)min((int64_t)4, (int64_t)offs[g] - src);
+        nv = (int)min((int64_t)4, (int64_t)so[g] - src);
     };
 
     if (warp == CWARPS) {

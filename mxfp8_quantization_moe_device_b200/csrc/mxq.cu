@@ -154,9 +154,9 @@ int device_info(const DevInfo **out)
             cudaFuncSetAttribute(k_mx_grouped_gemm_wgrad<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(gmx::smem_fixed<256>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_blocked_grouped_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(blkt::smem_fixed<blkt::R_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+                                 (int)(blkt::smem_fixed<blkt::R_STAGE>() + 2 * blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_blocked_grouped_k_tma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(blkt::smem_fixed<blkt::K_STAGE>() + blk::MAX_G * sizeof(int))) != cudaSuccess ||
+                                 (int)(blkt::smem_fixed<blkt::K_STAGE>() + 2 * blk::MAX_G * sizeof(int))) != cudaSuccess ||
             cudaFuncSetAttribute(k_fp8_grouped_gemm_wgrad_2sm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)g2::SMEM_BYTES) != cudaSuccess)
             return MXQ_ERR_CUDA;
@@ -806,7 +806,7 @@ int mx_scales_to_blocked_grouped(const uint8_t *scales, int64_t rows, int64_t co
         rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, scales, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
         if (rc != MXQ_OK)
             return rc;
-        const size_t smem = blkt::smem_fixed<blkt::R_STAGE>() + (size_t)num_groups * sizeof(int);
+        const size_t smem = blkt::smem_fixed<blkt::R_STAGE>() + 2 * (size_t)num_groups * sizeof(int);
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_blocked_grouped_tma, blkt::THREADS, smem) !=
             cudaSuccess)
@@ -867,7 +867,7 @@ int mx_scales_to_blocked_grouped_k(const uint8_t *scales, int64_t rows, int64_t 
         rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, scales, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc != MXQ_OK)
             return rc;
-        const size_t smem = blkt::smem_fixed<blkt::K_STAGE>() + (size_t)num_groups * sizeof(int);
+        const size_t smem = blkt::smem_fixed<blkt::K_STAGE>() + 2 * (size_t)num_groups * sizeof(int);
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_blocked_grouped_k_tma, blkt::THREADS, smem) !=
             cudaSuccess)
