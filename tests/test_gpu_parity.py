@@ -84,6 +84,10 @@ JAGGED = [
     # single-read kernel keeps 8 groups of a unit in shared memory and the
     # rest (here also one spanning two units) in the global table
     (1024, 136, [10, 20, 30, 40, 50, 60, 70, 80, 90, 100, 200, 300, 1024]),
+    # one group over all 16384 positions: every unit of every strip shares it
+    (16384, 256, [16384]),
+    # the same positions with empty groups before and after the only real one
+    (16384, 256, [0, 0, 16384, 16384]),
 ]
 
 
